@@ -1,0 +1,242 @@
+"""Seeded synthetic workloads: sequence layouts and input tensors.
+
+This module is the only code shared by the CUDA library's callers (tests,
+bench) and the fp64 oracle.  It holds configuration and random-number
+generation only -- none of the attention, RoPE, pooling or selection
+arithmetic.  Inputs are drawn in float32 from numpy's PCG64 with a fixed seed
+and, for bf16 workloads, rounded to bfloat16 (round to nearest even) once;
+the same bits go to the GPU and to the oracle.
+
+Layouts follow the sequence order [conditioning frames (t<0) | video | audio
+| text] of one batch item.  Audio tokens use the 21/218 temporal scale that
+makes 218 audio tokens span 21 latent frames (SkyReels-V4 digest, novelty 5).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import Dict, List, Optional, Tuple
+
+import numpy as np
+
+SEG_VIDEO, SEG_AUDIO, SEG_TEXT = 0, 1, 2
+ORDER_RASTER, ORDER_BLOCK444 = 0, 1
+AUDIO_T_NUM, AUDIO_T_DEN = 21, 218
+
+
+def video(T, H, W, t0=0, order=ORDER_RASTER):
+    return dict(kind=SEG_VIDEO, n_tokens=T * H * W, T=T, H=H, W=W, t0=t0,
+                t_num=1, t_den=1, order=order)
+
+
+def audio(n, t0=0):
+    return dict(kind=SEG_AUDIO, n_tokens=n, T=n, H=1, W=1, t0=t0,
+                t_num=AUDIO_T_NUM, t_den=AUDIO_T_DEN, order=ORDER_RASTER)
+
+
+def text(n):
+    return dict(kind=SEG_TEXT, n_tokens=n, T=n, H=1, W=1, t0=0, t_num=1,
+                t_den=1, order=ORDER_RASTER)
+
+
+@dataclass
+class Workload:
+    name: str
+    segments: List[dict]
+    batch: int
+    heads: int
+    head_dim: int
+    dtype: str                   # "bf16" or "f32"
+    seed: int
+    qk_std: float                # std of the N(0, std^2) background of Q and K
+    v_std: float
+    planted_regions: int = 0     # Gaussian "hot" regions added to Q and K
+    planted_amp: float = 0.0
+    mask: bool = False           # carry a channel-concat mask (never applied)
+    sparse: bool = False         # block-sparse video self-attention
+    top_k: int = 32
+    top_p: float = 0.9
+    theta: float = 10000.0
+    extra: Dict = field(default_factory=dict)
+
+    @property
+    def n_tokens(self) -> int:
+        return sum(s["n_tokens"] for s in self.segments)
+
+    @property
+    def n_video(self) -> int:
+        """Tokens of the video stream (conditioning frames included)."""
+        return sum(s["n_tokens"] for s in self.segments if s["kind"] == SEG_VIDEO)
+
+    @property
+    def n_audio(self) -> int:
+        return sum(s["n_tokens"] for s in self.segments if s["kind"] == SEG_AUDIO)
+
+    def video_range(self) -> Tuple[int, int]:
+        return _kind_range(self.segments, SEG_VIDEO)
+
+    def audio_range(self) -> Tuple[int, int]:
+        return _kind_range(self.segments, SEG_AUDIO)
+
+
+def _kind_range(segs, kind):
+    start = 0
+    lo = hi = None
+    for s in segs:
+        if s["kind"] == kind:
+            if lo is None:
+                lo = start
+            elif hi != start:
+                raise ValueError("segments of one kind must be contiguous")
+            hi = start + s["n_tokens"]
+        start += s["n_tokens"]
+    if lo is None:
+        return (0, 0)
+    return (lo, hi)
+
+
+INV_SQRT_128 = float(1.0 / np.sqrt(128.0))
+
+# The five workloads of the benchmark.  Sizes follow the 480p / 720p / 1080p
+# 21-latent-frame shapes; 218 audio tokens span the 21 frames.
+WORKLOADS: Dict[str, Workload] = {
+    "tiny_f32": Workload(
+        "tiny_f32", [video(1, 4, 4, t0=-1), video(3, 4, 4), audio(32), text(16)],
+        batch=1, heads=2, head_dim=64, dtype="f32", seed=0, qk_std=1.0, v_std=1.0),
+    "480p": Workload(
+        "480p", [video(21, 30, 52), audio(218), text(512)],
+        batch=1, heads=24, head_dim=128, dtype="bf16", seed=1,
+        qk_std=INV_SQRT_128, v_std=INV_SQRT_128),
+    "720p": Workload(
+        "720p", [video(21, 45, 80), audio(218), text(512)],
+        batch=1, heads=24, head_dim=128, dtype="bf16", seed=2,
+        qk_std=INV_SQRT_128, v_std=INV_SQRT_128),
+    "720p_cond_b2": Workload(
+        "720p_cond_b2", [video(2, 45, 80, t0=-2), video(21, 45, 80), audio(218), text(512)],
+        batch=2, heads=24, head_dim=128, dtype="bf16", seed=3,
+        qk_std=INV_SQRT_128, v_std=INV_SQRT_128, mask=True),
+    "1080p_sparse": Workload(
+        "1080p_sparse", [video(21, 68, 120, order=ORDER_BLOCK444), audio(218)],
+        batch=1, heads=24, head_dim=128, dtype="bf16", seed=4,
+        qk_std=1.0, v_std=1.0, planted_regions=8, planted_amp=2.0, sparse=True),
+}
+
+
+def reduced(name: str, T: int, H: int, W: int, n_audio: Optional[int] = None,
+            n_text: Optional[int] = None, heads: int = 2, seed_offset: int = 100,
+            batch: Optional[int] = None) -> Workload:
+    """A smaller workload with the structure of ``name``: every video segment
+    gets the grid (T', H, W) with T' = T for the target video and the original
+    frame count for conditioning frames."""
+    w = WORKLOADS[name]
+    segs = []
+    for s in w.segments:
+        if s["kind"] == SEG_VIDEO:
+            tt = s["T"] if s["t0"] < 0 else T
+            segs.append(video(tt, H, W, t0=s["t0"], order=s["order"]))
+        elif s["kind"] == SEG_AUDIO:
+            segs.append(audio(n_audio if n_audio is not None else s["n_tokens"]))
+        else:
+            segs.append(text(n_text if n_text is not None else s["n_tokens"]))
+    return Workload(f"{name}_reduced_{T}x{H}x{W}", segs, batch or w.batch, heads,
+                    w.head_dim, w.dtype, w.seed + seed_offset, w.qk_std, w.v_std,
+                    w.planted_regions, w.planted_amp, w.mask, w.sparse, w.top_k,
+                    w.top_p, w.theta)
+
+
+# ---------------------------------------------------------------------------
+# bf16 helpers (storage conversion only)
+# ---------------------------------------------------------------------------
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 to bfloat16, nearest even; returns uint16 bit patterns."""
+    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    r = ((b >> 16) & 1) + np.uint32(0x7FFF)
+    return ((b + r) >> 16).astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+# ---------------------------------------------------------------------------
+# generators
+# ---------------------------------------------------------------------------
+
+def _block_major_permutation(T: int, H: int, W: int) -> np.ndarray:
+    """Raster index of every token of a T x H x W grid, listed in 4x4x4
+    block-major storage order (blocks in (tb, hb, wb) raster order, tokens
+    inside a block in (t, h, w) raster order over the block's real extent)."""
+    idx = np.arange(T * H * W, dtype=np.int64).reshape(T, H, W)
+    parts = []
+    for t0 in range(0, T, 4):
+        for h0 in range(0, H, 4):
+            for w0 in range(0, W, 4):
+                parts.append(idx[t0:t0 + 4, h0:h0 + 4, w0:w0 + 4].reshape(-1))
+    return np.concatenate(parts)
+
+
+def _planted_bump(seg: dict, n_regions: int, amp: float, rng) -> np.ndarray:
+    """max over regions of amp * exp(-|(x - c) / sigma|^2 / 2) on the grid of
+    a video segment, in the segment's storage order (float32, [n_tokens]).
+    Centres are uniform in the grid; sigma per axis = extent / 8."""
+    T, H, W = seg["T"], seg["H"], seg["W"]
+    tt, hh, ww = np.meshgrid(np.arange(T), np.arange(H), np.arange(W), indexing="ij")
+    bump = np.zeros((T, H, W), np.float32)
+    sig = np.array([T, H, W], np.float64) / 8.0
+    for _ in range(n_regions):
+        c = rng.uniform(0, 1, 3) * np.array([T, H, W])
+        d2 = (((tt - c[0]) / sig[0]) ** 2 + ((hh - c[1]) / sig[1]) ** 2
+              + ((ww - c[2]) / sig[2]) ** 2)
+        bump = np.maximum(bump, (amp * np.exp(-0.5 * d2)).astype(np.float32))
+    flat = bump.reshape(-1)
+    if seg["order"] == ORDER_BLOCK444:
+        flat = flat[_block_major_permutation(T, H, W)]
+    return flat
+
+
+def _mask(w: Workload, rng) -> np.ndarray:
+    """uint8 [B, frames, H, W]: axis-aligned boxes with uniform corners added
+    until at least 30% of the tokens are covered."""
+    vids = [s for s in w.segments if s["kind"] == SEG_VIDEO]
+    F = sum(s["T"] for s in vids)
+    H, W = vids[0]["H"], vids[0]["W"]
+    m = np.zeros((w.batch, F, H, W), np.uint8)
+    for b in range(w.batch):
+        while m[b].mean() < 0.30:
+            lo = [rng.integers(0, n) for n in (F, H, W)]
+            hi = [rng.integers(l, n) + 1 for l, n in zip(lo, (F, H, W))]
+            m[b, lo[0]:hi[0], lo[1]:hi[1], lo[2]:hi[2]] = 1
+    return m
+
+
+def generate(w: Workload) -> Dict[str, np.ndarray]:
+    """Q, K, V [B, N, heads, d] (+ mask).  bf16 workloads return uint16 bit
+    patterns under 'q','k','v'; f32 workloads return float32 arrays."""
+    rng = np.random.Generator(np.random.PCG64(w.seed))
+    shape = (w.batch, w.n_tokens, w.heads, w.head_dim)
+    out = {}
+    for name, std in (("q", w.qk_std), ("k", w.qk_std), ("v", w.v_std)):
+        x = rng.standard_normal(shape, dtype=np.float32)
+        x *= np.float32(std)
+        out[name] = x
+    if w.planted_regions:
+        start = 0
+        for s in w.segments:
+            if s["kind"] == SEG_VIDEO:
+                bump = _planted_bump(s, w.planted_regions, w.planted_amp, rng)
+                for name in ("q", "k"):
+                    out[name][:, start:start + s["n_tokens"]] += bump[None, :, None, None]
+            start += s["n_tokens"]
+    if w.dtype == "bf16":
+        for name in ("q", "k", "v"):
+            out[name] = f32_to_bf16_bits(out[name])
+    if w.mask:
+        out["mask"] = _mask(w, rng)
+    return out
+
+
+def as_f64(x: np.ndarray, dtype: str) -> np.ndarray:
+    """The exact values a generated tensor holds, as float64."""
+    if dtype == "bf16":
+        return bf16_bits_to_f32(x).astype(np.float64)
+    return np.asarray(x, np.float64)

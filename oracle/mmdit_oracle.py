@@ -1,0 +1,352 @@
+"""Plain fp64 CPU oracle for the joint video/audio attention hot path.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may call it.  It shares no code, table or helper with the CUDA
+library; the only thing both sides share is the seeded input generator, which
+holds none of the method's arithmetic.
+
+Every function is written straight from the definitions, in float64, with no
+blocking, fusion or reordering beyond what the definition states, so that a
+reader can check it against the sources by eye:
+
+* Sources (cited by page title and section):
+  - [SKY-D] "SkyReels-V4: Multi-modal Video-Audio Generation, Inpainting and
+    Editing model" -- Chinese digest of arXiv 2602.21818: workflow steps 1-6
+    and the list of novelties (4th: time-offset 3D RoPE with negative
+    temporal indices; 5th: audio RoPE frequency scaling 21/218).
+  - [SKY-B] "SkyReels-V4: dual-stream MMDiT ..." -- trdm.cn blog, sections
+    2.1 (dual stream then single stream, joint self-attention) and 2.2
+    (bidirectional audio<->video cross-attention in every block; 21 video
+    frames aligned with 218 audio tokens through RoPE frequency scaling).
+  - [PRISM] "Prism: dynamic sparse attention for native 2K joint video-audio
+    generation" -- reading guide of arXiv 2610.05416, Method section 3
+    (mean-pooled key blocks, block probabilities P_i, and the attended set
+    S_i = Top-k(P_i, k) U Top-p(P_i, p)); scope rule in the Method preamble
+    (only video self-attention is sparsified, cross-attention stays dense).
+
+Readings where the sources are silent are stated at each function; the
+complete list is kept with the design notes of the repository.
+
+Pins: every function here is checked by ``tests/test_oracle_*.py`` against
+closed forms, invariants, worked values and brute force -- never against the
+CUDA path.  The model-level output beyond attention is not computed here.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import List, Sequence, Tuple
+
+import numpy as np
+
+SEG_VIDEO = 0
+SEG_AUDIO = 1
+SEG_TEXT = 2
+
+ORDER_RASTER = 0
+ORDER_BLOCK444 = 1
+
+BLOCK_EDGE = 4  # 4x4x4 token blocks of the sparse mode
+
+
+@dataclass
+class Segment:
+    """One contiguous run of tokens of a per-batch sequence.
+
+    kind     : SEG_VIDEO / SEG_AUDIO / SEG_TEXT
+    n_tokens : number of tokens in the run
+    T, H, W  : video grid (T frames of H x W latent tokens); unused otherwise
+    t0       : first temporal index; negative for conditioning/reference
+               latents ([SKY-D] step 1: reference latents are concatenated in
+               time and told apart from the target by negative time indices)
+    t_num, t_den : audio temporal scale t = t0 + j * t_num / t_den
+               ([SKY-D] novelty 5: 218 audio tokens span 21 latent frames)
+    order    : ORDER_RASTER or ORDER_BLOCK444 (video only)
+    """
+
+    kind: int
+    n_tokens: int
+    T: int = 0
+    H: int = 0
+    W: int = 0
+    t0: int = 0
+    t_num: int = 1
+    t_den: int = 1
+    order: int = ORDER_RASTER
+
+
+@dataclass
+class Layout:
+    segments: List[Segment] = field(default_factory=list)
+
+    @property
+    def n_tokens(self) -> int:
+        return sum(s.n_tokens for s in self.segments)
+
+
+# ---------------------------------------------------------------------------
+# a1: positions
+# ---------------------------------------------------------------------------
+
+def _block_major_coords(T: int, H: int, W: int) -> np.ndarray:
+    """(t, h, w) of every token of a T x H x W grid stored block-major.
+
+    Blocks of 4x4x4 tokens are visited in (tb, hb, wb) raster order; inside a
+    block the tokens are visited in (t, h, w) raster order over the block's
+    real extent.  Blocks on the far edge of an axis that does not divide by 4
+    are short and hold only their real tokens (no padding in memory).
+    """
+    e = BLOCK_EDGE
+    out = []
+    for tb in range(-(-T // e)):
+        for hb in range(-(-H // e)):
+            for wb in range(-(-W // e)):
+                for t in range(tb * e, min(T, tb * e + e)):
+                    for h in range(hb * e, min(H, hb * e + e)):
+                        for w in range(wb * e, min(W, wb * e + e)):
+                            out.append((t, h, w))
+    return np.asarray(out, dtype=np.float64).reshape(-1, 3)
+
+
+def positions(layout: Layout) -> np.ndarray:
+    """Per-token RoPE positions (t, h, w) as float64, shape [N, 3].
+
+    * video, raster order: token n -> (t0 + n // (H W), (n // W) % H, n % W)
+    * video, block-major: see ``_block_major_coords``; t shifted by t0
+    * audio token j -> (t0 + j * t_num / t_den, 0, 0)       [SKY-D] novelty 5
+    * text -> (0, 0, 0)   (reading: the sources give text no 3D position)
+    """
+    rows = []
+    for s in layout.segments:
+        if s.kind == SEG_VIDEO:
+            if s.n_tokens != s.T * s.H * s.W:
+                raise ValueError("video segment size != T*H*W")
+            if s.order == ORDER_RASTER:
+                n = np.arange(s.n_tokens)
+                p = np.stack([s.t0 + n // (s.H * s.W), (n // s.W) % s.H, n % s.W], 1)
+                p = p.astype(np.float64)
+            else:
+                p = _block_major_coords(s.T, s.H, s.W)
+                p[:, 0] += s.t0
+            rows.append(p)
+        elif s.kind == SEG_AUDIO:
+            j = np.arange(s.n_tokens, dtype=np.float64)
+            p = np.zeros((s.n_tokens, 3))
+            p[:, 0] = s.t0 + j * s.t_num / s.t_den
+            rows.append(p)
+        elif s.kind == SEG_TEXT:
+            rows.append(np.zeros((s.n_tokens, 3)))
+        else:
+            raise ValueError("unknown segment kind")
+    if not rows:
+        return np.zeros((0, 3))
+    return np.concatenate(rows, 0)
+
+
+# ---------------------------------------------------------------------------
+# a2: 3D RoPE
+# ---------------------------------------------------------------------------
+
+def rope_bands(head_dim: int) -> Tuple[int, int, int]:
+    """Channel split (d_t, d_h, d_w) of the 3D RoPE.
+
+    Reading: h and w get 2*floor(d/6) channels each and t the rest, which is
+    44/42/42 at d=128 and 24/20/20 at d=64.
+    """
+    dh = 2 * (head_dim // 6)
+    return head_dim - 2 * dh, dh, dh
+
+
+def rope(x: np.ndarray, pos: np.ndarray, theta: float = 10000.0,
+         bands: Tuple[int, int, int] | None = None) -> np.ndarray:
+    """Rotate every head of x by its token's (t, h, w) position.
+
+    x   : [..., N, heads, d] (any float dtype; computed in float64)
+    pos : [N, 3]
+    Channels are split into consecutive bands [t | h | w]; inside band b of
+    width d_b, channel pair (2i, 2i+1) -- pairs interleaved, i counted from
+    the band start -- is treated as the complex number x_2i + 1j*x_2i+1 and
+    multiplied by exp(1j * pos_b * theta**(-2i/d_b)).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    if bands is None:
+        bands = rope_bands(d)
+    if sum(bands) != d or any(b % 2 for b in bands):
+        raise ValueError("bad RoPE bands")
+    z = x[..., 0::2] + 1j * x[..., 1::2]            # [..., N, heads, d/2]
+    angle = np.zeros((pos.shape[0], d // 2))
+    start = 0
+    for axis, db in enumerate(bands):
+        i = np.arange(db // 2, dtype=np.float64)
+        omega = theta ** (-2.0 * i / db)
+        angle[:, start // 2:(start + db) // 2] = pos[:, axis:axis + 1] * omega[None, :]
+        start += db
+    z = z * np.exp(1j * angle)[:, None, :]
+    out = np.empty_like(x)
+    out[..., 0::2] = z.real
+    out[..., 1::2] = z.imag
+    return out
+
+
+# ---------------------------------------------------------------------------
+# a3 / a4: attention
+# ---------------------------------------------------------------------------
+
+def attn(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float):
+    """softmax(q k^T * scale) v for one head, float64, no mask.
+
+    q [Nq, d], k [Nk, d], v [Nk, dv] -> (o [Nq, dv], lse [Nq]) where lse is
+    the natural-log sum of exp of the scaled scores of each row.
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    s = (q @ k.T) * scale
+    m = s.max(axis=1, keepdims=True)
+    e = np.exp(s - m)
+    l = e.sum(axis=1, keepdims=True)
+    o = (e @ v) / l
+    lse = (m + np.log(l))[:, 0]
+    return o, lse
+
+
+def attn_bshd(q, k, v, scale):
+    """attn for every (batch, head) of [B, N, H, d] tensors."""
+    q = np.asarray(q, np.float64)
+    B, Nq, H, _ = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, Nq, H, dv))
+    lse = np.zeros((B, Nq, H))
+    for b in range(B):
+        for h in range(H):
+            o[b, :, h], lse[b, :, h] = attn(q[b, :, h], k[b, :, h], v[b, :, h], scale)
+    return o, lse
+
+
+def joint_attn(q, k, v, scale):
+    """Joint self-attention over the whole concatenated sequence.
+
+    [SKY-D] step 3 and [SKY-B] 2.1: video(/audio) and text tokens are
+    projected separately and then attend jointly in one softmax; the
+    dual-stream and single-stream blocks run the same attention math.  The
+    binary mask M of step 2 is an input channel, not an attention mask, so it
+    does not enter here.
+    """
+    return attn_bshd(q, k, v, scale)
+
+
+def av_cross_attn(qv, kv, vv, qa, ka, va, scale):
+    """Bidirectional audio<->video cross-attention ([SKY-D] step 3,
+    [SKY-B] 2.2): video queries attend to the audio keys/values and audio
+    queries attend to the video keys/values.  Returns (o_video, o_audio)."""
+    o_v, _ = attn_bshd(qv, ka, va, scale)
+    o_a, _ = attn_bshd(qa, kv, vv, scale)
+    return o_v, o_a
+
+
+# ---------------------------------------------------------------------------
+# a5 - a7: block-sparse mode
+# ---------------------------------------------------------------------------
+
+def video_blocks(T: int, H: int, W: int):
+    """Token ranges of the 4x4x4 blocks of a block-major video segment.
+
+    Returns a list of (start, length) in block order (tb, hb, wb raster);
+    a block's tokens are contiguous in the block-major storage."""
+    e = BLOCK_EDGE
+    out = []
+    start = 0
+    for tb in range(-(-T // e)):
+        for hb in range(-(-H // e)):
+            for wb in range(-(-W // e)):
+                n = ((min(T, tb * e + e) - tb * e) * (min(H, hb * e + e) - hb * e)
+                     * (min(W, wb * e + e) - wb * e))
+                out.append((start, n))
+                start += n
+    return out
+
+
+def pool(x: np.ndarray, blocks) -> np.ndarray:
+    """Mean over the real tokens of each block ([PRISM] Method 3: keys are
+    mean-pooled into block representatives; the query is pooled the same way
+    -- a reading).  x [B, N, H, d] -> [B, H, nblocks, d] float64."""
+    x = np.asarray(x, np.float64)
+    B, _, Hh, d = x.shape
+    out = np.zeros((B, Hh, len(blocks), d))
+    for i, (s, n) in enumerate(blocks):
+        out[:, :, i, :] = x[:, s:s + n].mean(axis=1)
+    return out
+
+
+def select_row(qbar_i: np.ndarray, kbar: np.ndarray, top_k: int, top_p: float,
+               scale: float) -> np.ndarray:
+    """Attended key-block set of one query block ([PRISM] Method 3).
+
+    P_i = softmax_j(qbar_i . kbar_j * scale).  Blocks are ordered by P
+    descending, ties by block id ascending.  Top-k takes the first
+    min(k, n) blocks; Top-p takes the shortest prefix whose cumulative
+    probability reaches p (the block that crosses p is included; if
+    rounding keeps the sum below p, every block).  S_i is their union,
+    returned in ascending block id.
+    """
+    s = (kbar @ qbar_i) * scale
+    e = np.exp(s - s.max())
+    P = e / e.sum()
+    n = P.shape[0]
+    order = sorted(range(n), key=lambda j: (-P[j], j))
+    n_k = min(top_k, n)
+    csum = 0.0
+    n_p = n
+    for r, j in enumerate(order):
+        csum += P[j]
+        if csum >= top_p:
+            n_p = r + 1
+            break
+    chosen = order[:max(n_k, n_p)]
+    return np.asarray(sorted(chosen), dtype=np.int64)
+
+
+def block_probs(qbar_i, kbar, scale):
+    """P_i of ``select_row`` (exposed for tie analysis in the tests)."""
+    s = (kbar @ qbar_i) * scale
+    e = np.exp(s - s.max())
+    return e / e.sum()
+
+
+def block_select(qbar, kbar, top_k, top_p, scale):
+    """``select_row`` for every (batch, head, query block).
+
+    qbar, kbar [B, H, nblk, d] -> nested list sel[b][h][i] of int arrays."""
+    B, Hh, nq, _ = qbar.shape
+    return [[[select_row(qbar[b, h, i], kbar[b, h], top_k, top_p, scale)
+              for i in range(nq)] for h in range(Hh)] for b in range(B)]
+
+
+def sparse_attn_rows(q, k, v, blocks, sel, scale, b: int, h: int, qblk: int):
+    """Sparse attention for the tokens of one query block: the tokens of
+    query block ``qblk`` attend only to the tokens of the key blocks in
+    ``sel`` (the attended set S_i), with one softmax over all of them
+    ([PRISM] Method 3, online-softmax attention over S_i)."""
+    s0, n = blocks[qblk]
+    kk = np.concatenate([k[b, blocks[j][0]:blocks[j][0] + blocks[j][1], h] for j in sel], 0)
+    vv = np.concatenate([v[b, blocks[j][0]:blocks[j][0] + blocks[j][1], h] for j in sel], 0)
+    o, lse = attn(q[b, s0:s0 + n, h], kk, vv, scale)
+    return o, lse
+
+
+def sparse_attn(q, k, v, blocks, sel, scale):
+    """``sparse_attn_rows`` for every (batch, head, query block);
+    q, k, v [B, N, H, d] block-major; sel as returned by block_select."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    B, N, Hh, _ = q.shape
+    o = np.zeros((B, N, Hh, v.shape[-1]))
+    for b in range(B):
+        for h in range(Hh):
+            for i, (s0, n) in enumerate(blocks):
+                o[b, s0:s0 + n, h], _ = sparse_attn_rows(q, k, v, blocks, sel[b][h][i],
+                                                         scale, b, h, i)
+    return o
