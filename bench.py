@@ -1,0 +1,497 @@
+"""Benchmark of the joint video/audio attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl reference]
+
+One step is one pass of the layer's attention hot path over one batch of the
+workload: 3D RoPE of Q and K, then (dense workloads) joint self-attention over
+the whole sequence or (block-sparse workload) block selection and sparse
+video self-attention, then the bidirectional audio<->video cross-attention.
+Inputs are seeded synthetic tensors of the workload's shape, resident in HBM
+before timing; they are larger than L2 (126 MB), so no flush is needed.
+
+The JSON line reports algorithmic TFLOP/s (4 * Nq * Nkv * d per head for
+every attention; for sparse attention only the selected token pairs), video
+tokens/s, an end-to-end figure through the same C-ABI calls with pinned host
+buffers copied in and results copied out every step, the live roofline of
+the dominant kernel (CUDA events around its launches), SM clocks sampled
+during the timed region, and the fp64 oracle timed on a bounded sample on
+the host cores (CPU baseline).
+
+``--impl reference`` times the fp64 oracle instead (the reference arm): each
+step is a bounded sample of the same workload on the host cores.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own copy of
+the workload with no collective on the data path (weak scaling); ranks meet
+only at the barriers around the timed region and the max-over-ranks time
+reduction.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from joint_video_audio_rope_b200 import workloads as WL  # noqa: E402
+
+METRIC = "joint A/V attention TFLOP/s & video tokens/s per layer, % of B200 bf16 TC peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------- ranks
+
+def dist_env():
+    """(rank, world, local_rank) from the torchrun environment."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity on one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ----------------------------------------------------------------- work model
+
+def attn_flops(nq: int, nkv: int, d: int, heads: int, batch: int) -> float:
+    return 4.0 * nq * nkv * d * heads * batch
+
+
+def dense_step_flops(w: WL.Workload) -> dict:
+    n, d, H, B = w.n_tokens, w.head_dim, w.heads, w.batch
+    nv, na = w.n_video, w.n_audio
+    return {"joint": attn_flops(n, n, d, H, B),
+            "cross": attn_flops(nv, na, d, H, B) + attn_flops(na, nv, d, H, B)}
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi SM clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- oracle (CPU)
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_sample(w: WL.Workload, host: dict, rows: int, seed: int = 0):
+    """Run the fp64 oracle on a bounded sample of one step: RoPE of every key
+    and of `rows` sampled query rows, those rows' joint attention (or, for the
+    sparse workload, their block-sparse attention after pooling and selection
+    on all blocks), and the cross-attention of `rows` video rows plus every
+    audio row.  Returns (seconds, algorithmic flops of the sample)."""
+    import oracle as O
+    rng = np.random.default_rng(seed)
+    lay = O.Layout([O.Segment(s["kind"], s["n_tokens"], s["T"], s["H"], s["W"], s["t0"],
+                              s["t_num"], s["t_den"], s["order"]) for s in w.segments])
+    d, H = w.head_dim, w.heads
+    scale = 1.0 / math.sqrt(d)
+    t0 = time.perf_counter()
+    flops = 0.0
+    pos = O.positions(lay)
+    q = WL.as_f64(host["q"][0], w.dtype)
+    k = O.rope(WL.as_f64(host["k"][0], w.dtype), pos, w.theta)
+    v = WL.as_f64(host["v"][0], w.dtype)
+    sel_rows = np.sort(rng.choice(w.n_tokens, size=min(rows, w.n_tokens), replace=False))
+    qr = O.rope(q[sel_rows], pos[sel_rows], w.theta)
+    v0, v1 = w.video_range()
+    a0, a1 = w.audio_range()
+    if not w.sparse:
+        for h in range(H):
+            O.attn(qr[:, h], k[:, h], v[:, h], scale)
+        flops += attn_flops(len(sel_rows), w.n_tokens, d, H, 1)
+    else:
+        seg = w.segments[0]
+        blocks = O.video_blocks(seg["T"], seg["H"], seg["W"])
+        qfull = O.rope(q[v0:v1], pos[v0:v1], w.theta)
+        qb, kb = O.pool(qfull[None], blocks), O.pool(k[None, v0:v1], blocks)
+        starts = np.array([s for s, _ in blocks])
+        for r in sel_rows[sel_rows < v1]:
+            i = int(np.searchsorted(starts, r, side="right") - 1)
+            for h in range(H):
+                sel = O.select_row(qb[0, h, i], kb[0, h], w.top_k, float(np.float32(w.top_p)), scale)
+                kk = np.concatenate([k[blocks[j][0]:blocks[j][0] + blocks[j][1], h] for j in sel])
+                vv = np.concatenate([v[blocks[j][0]:blocks[j][0] + blocks[j][1], h] for j in sel])
+                O.attn(qr[sel_rows == r][:, h], kk, vv, scale)
+                flops += attn_flops(1, len(kk), d, 1, 1)
+    # cross-attention: sampled video rows over the audio keys, every audio row
+    # over the video keys
+    vrows = sel_rows[(sel_rows >= v0) & (sel_rows < v1)]
+    if a1 > a0:
+        qa = O.rope(q[a0:a1], pos[a0:a1], w.theta)
+        for h in range(H):
+            O.attn(qr[np.isin(sel_rows, vrows)][:, h], k[a0:a1, h], v[a0:a1, h], scale)
+            O.attn(qa[:, h], k[v0:v1, h], v[v0:v1, h], scale)
+        flops += attn_flops(len(vrows), a1 - a0, d, H, 1) + attn_flops(a1 - a0, v1 - v0, d, H, 1)
+    return time.perf_counter() - t0, flops
+
+
+def cpu_baseline(w: WL.Workload, host: dict, target_s: float = 15.0) -> dict:
+    """Time the oracle as it stands on a bounded sample (about `target_s`)."""
+    probe_rows = 16
+    dt, _ = oracle_sample(w, host, probe_rows, seed=1)
+    rows = int(max(8, min(w.n_tokens, probe_rows * target_s / max(dt, 1e-3))))
+    dt, flops = oracle_sample(w, host, rows, seed=2)
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{rows} sampled query rows x {w.heads} heads (+ all audio rows for the "
+                      f"cross-attention), keys RoPE'd in full; {dt:.1f} s fp64 numpy",
+            "seconds": dt}
+
+
+# ----------------------------------------------------------------- GPU arm
+
+def run_gpu(args) -> int:
+    import torch
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    if rank == 0:
+        from joint_video_audio_rope_b200 import build
+        build.build()
+    barrier(world, dev)
+    from joint_video_audio_rope_b200 import mmdit as M
+
+    w = WL.WORKLOADS[args.workload]
+    x = WL.generate(w)
+    to_dev = lambda a: (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+                        .to(dev, non_blocking=False))
+    q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
+    o = torch.empty_like(q)
+    o_cross = torch.empty_like(q)  # video and audio slices receive the cross outputs
+    desc = M.desc_of(q)
+    lay = M.make_layout(w.segments)
+    rope = M.rope_params(w.theta, 44, 42, 42)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    v0, v1 = w.video_range()
+    a0, a1 = w.audio_range()
+    dv, da = M.desc_of(q[:, v0:v1]), M.desc_of(q[:, a0:a1])
+    ws_cross = M.av_cross_attn_workspace_size(dv, da)
+    sparse = w.sparse
+    if sparse:
+        vlay = M.make_layout([s for s in w.segments if s["kind"] == WL.SEG_VIDEO])
+        vd = M.desc_of(q[:, v0:v1])
+        nb = M.num_blocks(vlay)
+        idx = torch.empty((w.batch, w.heads, nb, nb), dtype=torch.int32, device=dev)
+        cnt = torch.empty((w.batch, w.heads, nb), dtype=torch.int32, device=dev)
+        ws_sel = M.block_select_workspace_size(vd, vlay)
+        ws_sp = M.sparse_attn_workspace_size(vd, vlay, nb)
+    else:
+        ws_sel = ws_sp = 0
+    ws = torch.empty(max(ws_cross, ws_sel, ws_sp, 256), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        M.rope_apply(q, k, desc, lay, rope, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        if sparse:
+            M.block_select(q[:, v0:v1], k[:, v0:v1], vd, vlay, w.top_k, w.top_p, scale, nb, idx,
+                           cnt, ws, ws.numel(), stream)
+            if ev is not None:
+                ev[2].record(stream)
+            M.sparse_attn(q[:, v0:v1], k[:, v0:v1], v[:, v0:v1], o[:, v0:v1], vd, vlay, idx, cnt,
+                          nb, scale, ws, ws.numel(), stream)
+        else:
+            if ev is not None:
+                ev[2].record(stream)
+            M.joint_attn(q, k, v, o, desc, lay, scale, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+        M.av_cross_attn(q[:, v0:v1], k[:, v0:v1], v[:, v0:v1], q[:, a0:a1], k[:, a0:a1],
+                        v[:, a0:a1], o_cross[:, v0:v1], o_cross[:, a0:a1], dv, da, scale, ws,
+                        ws.numel(), stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+    # launches of this library's kernels per step
+    launches_per_step = 1 + (2 + 3 if sparse else 1) + 2
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if M.device_status(stream) != 0:
+        raise RuntimeError("device status after warm-up: " + M.last_error())
+
+    flops = dense_step_flops(w)
+    if sparse:
+        # algorithmic work of sparse attention: selected token pairs only
+        cnt_h = cnt.cpu().numpy()
+        idx_h = idx.cpu().numpy()
+        seg = w.segments[0]
+        blen = np.array([_block_len(seg["T"], seg["H"], seg["W"], b) for b in range(nb)], np.int64)
+        pairs = 0
+        for b in range(w.batch):
+            for h in range(w.heads):
+                for i in range(nb):
+                    pairs += blen[i] * blen[idx_h[b, h, i, :cnt_h[b, h, i]]].sum()
+        flops = {"joint": 4.0 * pairs * w.head_dim, "cross": flops["cross"]}
+        density = float(cnt_h.mean() / nb)
+    step_flops = flops["joint"] + flops["cross"]
+
+    # ---------------------------------------------------------- timed region
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    barrier(world, dev)
+    if M.device_status(stream) != 0:
+        raise RuntimeError("device status after timing: " + M.last_error())
+    ms_total = reduce_max(t_start.elapsed_time(t_end), world, dev)
+    ms_step = ms_total / args.steps
+    part_ms = {name: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
+               for j, name in enumerate(["rope", "select" if sparse else "none",
+                                         "sparse" if sparse else "joint", "cross"])}
+
+    # ---------------------------------------------------------- end to end
+    pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hq, hk, hv = pin(x["q"]), pin(x["k"]), pin(x["v"])
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hoc = torch.empty(o_cross.shape, dtype=o.dtype).pin_memory()
+    e2e_steps = max(1, min(args.steps, 5))
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        step()
+        ho.copy_(o, non_blocking=True)
+        hoc.copy_(o_cross, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = reduce_max(e0.elapsed_time(e1), world, dev) / e2e_steps
+    h2d = 3 * q.numel() * q.element_size()
+    d2h = 2 * o.numel() * o.element_size()
+
+    # ---------------------------------------------------------- report
+    peaks, peak_src = read_peaks()
+    dom = "sparse" if sparse else "joint"
+    dom_ms = part_ms[dom]
+    achieved = flops["joint"] / (dom_ms / 1e3) / 1e12
+    peak = peaks.get("bf16_tflops_sustained") or FALLBACK_PEAKS["bf16_tflops_sustained"]
+    value = step_flops * world / (ms_step / 1e3) / 1e12
+    tokens_s = w.batch * w.n_video * world / (ms_step / 1e3)
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return 0
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.n_tokens,
+                   "video_tokens": w.n_video, "audio_tokens": w.n_audio, "heads": w.heads,
+                   "head_dim": w.head_dim, "parallelism": f"replica x{world} (no collective)",
+                   "l2": "inputs larger than L2 (no flush needed)",
+                   "step": ("rope+select+sparse+cross" if sparse else "rope+joint+cross")},
+        "video_tokens_per_s": round(tokens_s, 1),
+        "frac_of_peak": round(value / world / peak, 4),
+        "parts_ms": {k_: round(v_, 4) for k_, v_ in part_ms.items() if k_ != "none"},
+        "flops_per_step": {k_: v_ for k_, v_ in flops.items()},
+        "e2e": {"value": round(step_flops * world / (e2e_ms / 1e3) / 1e12, 2), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 3)},
+        "gpu_launches": launches_per_step * args.steps,
+        "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (" + dom + ")",
+                     "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": f"bf16_tflops_sustained of {peak_src}"},
+        "clocks": clocks,
+    }
+    if sparse:
+        line["block_density"] = round(density, 4)
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, x, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _block_len(T, H, W, b):
+    nhb, nwb = -(-H // 4), -(-W // 4)
+    tb, r = divmod(b, nhb * nwb)
+    hb, wb = divmod(r, nwb)
+    return min(4, T - 4 * tb) * min(4, H - 4 * hb) * min(4, W - 4 * wb)
+
+
+# ----------------------------------------------------------------- reference arm
+
+def run_reference(args) -> int:
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = WL.WORKLOADS[args.workload]
+    x = WL.generate(w)
+    cores = blas_threads()
+    # calibrate one step to about args.ref_step_seconds of oracle work
+    dt, _ = oracle_sample(w, x, 16, seed=1)
+    rows = int(max(8, min(w.n_tokens, 16 * args.ref_step_seconds / max(dt, 1e-3))))
+    for i in range(args.warmup):
+        oracle_sample(w, x, rows, seed=100 + i)
+    tot_s, tot_f = 0.0, 0.0
+    for i in range(args.steps):
+        s, f = oracle_sample(w, x, rows, seed=1000 + i)
+        tot_s += s
+        tot_f += f
+    value = tot_f / tot_s / 1e12
+    sample = (f"{rows} sampled query rows x {w.heads} heads per step (+ all audio rows for the "
+              f"cross-attention), fp64 numpy oracle")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.n_tokens,
+                   "video_tokens": w.n_video, "audio_tokens": w.n_audio, "heads": w.heads,
+                   "head_dim": w.head_dim, "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="480p", choices=sorted(WL.WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=6.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,253 @@
+/*
+ * mmdit.h -- C ABI of the joint video/audio attention hot path (sm_100a).
+ *
+ * The library implements the attention layer of a dual-stream MMDiT video +
+ * audio diffusion transformer as described for SkyReels-V4:
+ *   - "SkyReels-V4: Multi-modal Video-Audio Generation, Inpainting and
+ *     Editing model" (Chinese digest of arXiv 2602.21818), workflow steps 1-3
+ *     and novelties 4-5;
+ *   - "SkyReels-V4: dual-stream MMDiT ..." (trdm.cn blog), sections 2.1-2.2;
+ * plus an optional block-sparse mode after
+ *   - "Prism: dynamic sparse attention for native 2K joint video-audio
+ *     generation" (reading guide of arXiv 2610.05416), Method section 3.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Tensors are BSHD: element (b, n, h, c) of a tensor described by
+ * mmdit_tensor_desc d sits at  b*d.stride_batch + n*d.stride_tok + h*d.head_dim + c
+ * elements from the base pointer (heads are packed, channels contiguous).
+ * Strides are in elements; for bf16 tensors stride_tok*2 and stride_batch*2
+ * must be multiples of 16 bytes and the base pointer 16-byte aligned.
+ *
+ * Ownership: every pointer is caller-owned device memory (except the
+ * descriptor / layout structs, which are host memory read during the call).
+ * The library never allocates device memory on these calls: scratch comes
+ * from the caller's `workspace`, sized by the matching *_workspace_size query.
+ *
+ * Streams: every call only enqueues work on `stream` (a cudaStream_t; NULL is
+ * the legacy default stream) and returns without synchronising.
+ *
+ * Errors: calls return an mmdit_status.  Arguments are validated before any
+ * launch; on error nothing is launched and mmdit_last_error() describes the
+ * problem (thread-local string).  Device-side waits are bounded: a wait that
+ * runs out records MMDIT_ETIMEOUT in a per-device flag, the kernel releases its
+ * resources and returns; mmdit_device_status() reads and clears that flag.
+ */
+#ifndef MMDIT_H_
+#define MMDIT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MMDIT_API __attribute__((visibility("default")))
+#else
+#define MMDIT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* mmdit_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  MMDIT_OK = 0,
+  MMDIT_EINVAL = 1,       /* bad pointer, shape, stride, layout or parameter   */
+  MMDIT_EUNSUPPORTED = 2, /* dtype / head_dim / architecture not supported     */
+  MMDIT_EWORKSPACE = 3,   /* workspace missing or smaller than the size query  */
+  MMDIT_ECUDA = 4,        /* a CUDA runtime/driver call failed                 */
+  MMDIT_ETIMEOUT = 5      /* a bounded device-side wait ran out                */
+} mmdit_status;
+
+enum { MMDIT_BF16 = 0, MMDIT_F32 = 1 };
+enum { MMDIT_SEG_VIDEO = 0, MMDIT_SEG_AUDIO = 1, MMDIT_SEG_TEXT = 2 };
+enum { MMDIT_ORDER_RASTER = 0, MMDIT_ORDER_BLOCK444 = 1 };
+#define MMDIT_MAX_SEGMENTS 8
+
+/*
+ * One contiguous run of tokens in the per-batch-item sequence.  The sequence
+ * of one batch item is the concatenation of the layout's segments; the usual
+ * order is [conditioning frames | video | audio | text] but any order works.
+ *
+ *  kind = VIDEO: n_tokens = T*H*W latent tokens of T frames.  Token
+ *      positions are (t0 + t, h, w).  Conditioning / reference latents are a
+ *      video segment with t0 < 0 (SkyReels-V4 digest, step 1 and novelty 4:
+ *      reference latents are concatenated along time with negative temporal
+ *      indices).  order = RASTER stores tokens in (t, h, w) raster order;
+ *      order = BLOCK444 stores them block-major: 4x4x4 blocks in (tb, hb, wb)
+ *      raster order, tokens inside a block in (t, h, w) raster order over the
+ *      block's real extent (short edge blocks hold only their real tokens).
+ *  kind = AUDIO: token j has position (t0 + j*t_num/t_den, 0, 0).  With
+ *      t_num/t_den = 21/218, 218 audio tokens span 21 latent frames
+ *      (digest novelty 5; blog section 2.2).  T, H, W are ignored.
+ *  kind = TEXT: position (0, 0, 0): the identity rotation.
+ */
+typedef struct {
+  int32_t kind;
+  int32_t n_tokens;
+  int32_t T, H, W;
+  int32_t t0;
+  int32_t t_num, t_den;
+  int32_t order;
+} mmdit_segment;
+
+typedef struct {
+  int32_t n_seg;                          /* 1..MMDIT_MAX_SEGMENTS */
+  mmdit_segment seg[MMDIT_MAX_SEGMENTS];  /* same for every batch item */
+} mmdit_layout;
+
+typedef struct {
+  int32_t batch;      /* B >= 1 */
+  int32_t n_tokens;   /* N >= 0 (tokens per batch item) */
+  int32_t heads;      /* >= 1 */
+  int32_t head_dim;   /* 128 (bf16 or f32) or 64 (f32 only) */
+  int32_t dtype;      /* MMDIT_BF16 or MMDIT_F32 */
+  int64_t stride_tok;   /* elements between consecutive tokens (>= heads*head_dim) */
+  int64_t stride_batch; /* elements between consecutive batch items */
+} mmdit_tensor_desc;
+
+/* 3D RoPE parameters: theta and the channel split over the t / h / w axes
+ * (dim_t + dim_h + dim_w = head_dim, each even).  44/42/42 at head_dim 128. */
+typedef struct {
+  float theta;
+  int32_t dim_t, dim_h, dim_w;
+} mmdit_rope_params;
+
+/*
+ * mmdit_rope_apply -- 3D RoPE over (t, h, w), in place on q and/or k.
+ *   Digest novelty 4 (time-offset 3D RoPE) and 5 (audio scaling 21/218);
+ *   blog section 2.2.  Channels are split into bands [t | h | w]; in band b of
+ *   width d_b the interleaved pair (2i, 2i+1) (i counted from the band start)
+ *   is rotated by angle pos_b * theta^(-2i/d_b).  Positions come from
+ *   `layout` (never stored).
+ *   q, k   : device [B, N, heads, head_dim] described by `desc`; either may be
+ *            NULL (skipped), not both.  Updated in place.
+ *   layout : segments must sum to desc->n_tokens.
+ *   Errors : EINVAL (NULL both, bad layout/desc/bands), EUNSUPPORTED (dtype),
+ *            ECUDA.
+ */
+MMDIT_API int mmdit_rope_apply(void* q, void* k, const mmdit_tensor_desc* desc,
+                     const mmdit_layout* layout, const mmdit_rope_params* rope,
+                     mmdit_stream_t stream);
+
+/*
+ * mmdit_joint_attn -- joint self-attention over the whole concatenated
+ *   sequence of each batch item: O = softmax(Q K^T * scale) V per (batch,
+ *   head), no causal mask (digest step 3; blog section 2.1: video/audio and
+ *   text tokens attend jointly in one softmax, in both the dual-stream and the
+ *   single-stream blocks).
+ *   q, k, v, o : device [B, N, heads, head_dim], all described by `desc`
+ *                (o may not alias q, k or v).
+ *   lse        : NULL or device float [B, heads, N]: natural-log sum of exp of
+ *                the scaled scores of each query row.
+ *   rope_q     : NULL, or RoPE parameters to rotate Q by `layout` positions as
+ *                it is loaded (K must then already be rotated, e.g. by
+ *                mmdit_rope_apply with q = NULL).  bf16 only.
+ *   cond_mask  : NULL or device uint8 [B, F, H, W] with F the frames of all
+ *                video segments; the binary channel-concat mask M of digest
+ *                step 2.  It is an input channel of the patch embedding, not an
+ *                attention mask: it is shape-checked (mask_elems must equal
+ *                B*F*H*W) and never read or applied.
+ *   workspace  : may be NULL; mmdit_joint_attn_workspace_size() returns 0.
+ *   Errors     : EINVAL, EUNSUPPORTED, EWORKSPACE, ECUDA.
+ */
+MMDIT_API int mmdit_joint_attn(const void* q, const void* k, const void* v, void* o, float* lse,
+                     const mmdit_tensor_desc* desc, const mmdit_layout* layout,
+                     float scale, const mmdit_rope_params* rope_q,
+                     const uint8_t* cond_mask, int64_t mask_elems,
+                     void* workspace, size_t ws_bytes, mmdit_stream_t stream);
+MMDIT_API size_t mmdit_joint_attn_workspace_size(const mmdit_tensor_desc* desc);
+
+/*
+ * mmdit_av_cross_attn -- bidirectional audio<->video cross-attention (digest
+ *   step 3; blog section 2.2), both directions in one call:
+ *     o_video = softmax(qv ka^T * scale) va     (video queries, audio keys)
+ *     o_audio = softmax(qa kv^T * scale) vv     (audio queries, video keys)
+ *   qv, kv, vv, o_video : device, described by `video` (N = video tokens,
+ *                         conditioning frames included)
+ *   qa, ka, va, o_audio : device, described by `audio`
+ *   Both descriptors must agree on batch, heads, head_dim and dtype.  Inputs
+ *   are expected to be RoPE-rotated already.  The audio-query direction
+ *   splits the video keys across CTAs and merges partial results through the
+ *   workspace (size from mmdit_av_cross_attn_workspace_size).
+ *   Errors : EINVAL, EUNSUPPORTED, EWORKSPACE, ECUDA.
+ */
+MMDIT_API int mmdit_av_cross_attn(const void* qv, const void* kv, const void* vv,
+                        const void* qa, const void* ka, const void* va,
+                        void* o_video, void* o_audio,
+                        const mmdit_tensor_desc* video, const mmdit_tensor_desc* audio,
+                        float scale, void* workspace, size_t ws_bytes,
+                        mmdit_stream_t stream);
+MMDIT_API size_t mmdit_av_cross_attn_workspace_size(const mmdit_tensor_desc* video,
+                                          const mmdit_tensor_desc* audio);
+
+/*
+ * mmdit_block_select -- hybrid top-k / top-p key-block selection of the
+ *   block-sparse mode (Prism guide, Method section 3).
+ *   Q and K of one block-major video segment are mean-pooled per 4x4x4 block
+ *   (fp32, over each block's real tokens) into Qbar, Kbar.  For query block i
+ *   of each (batch, head): P_i = softmax_j(Qbar_i . Kbar_j * scale), and
+ *   S_i = TopK(P_i, top_k) U TopP(P_i, top_p), where blocks are ranked by P
+ *   descending (ties: lower block id first), TopK is the first min(top_k, n)
+ *   blocks and TopP the shortest prefix whose cumulative probability reaches
+ *   top_p (the crossing block included; all blocks if it never does).
+ *   q, k      : device [B, N, heads, 128] bf16, N = the video segment's tokens
+ *   layout    : exactly one VIDEO segment with order BLOCK444
+ *   cap       : row capacity of block_idx; must be >= the number of blocks
+ *               (a list is never truncated)
+ *   block_idx : device int32 [B, heads, nblocks, cap]: S_i in ascending block
+ *               id, entries past block_cnt are left unwritten
+ *   block_cnt : device int32 [B, heads, nblocks]: |S_i|
+ *   workspace : size from mmdit_block_select_workspace_size (pooled blocks)
+ *   Errors    : EINVAL (layout, cap, top_k < 0, top_p outside [0, 1]),
+ *               EUNSUPPORTED, EWORKSPACE, ECUDA.
+ */
+MMDIT_API int mmdit_block_select(const void* q, const void* k, const mmdit_tensor_desc* desc,
+                       const mmdit_layout* layout, int top_k, float top_p, float scale,
+                       int cap, int32_t* block_idx, int32_t* block_cnt,
+                       void* workspace, size_t ws_bytes, mmdit_stream_t stream);
+MMDIT_API size_t mmdit_block_select_workspace_size(const mmdit_tensor_desc* desc,
+                                         const mmdit_layout* layout);
+
+/*
+ * mmdit_sparse_attn -- attention restricted to selected key blocks (Prism
+ *   guide, Method section 3: online-softmax attention over S_i only).  Every
+ *   token of query block i attends, in one softmax, to the tokens of the key
+ *   blocks listed in block_idx[b, h, i, 0:block_cnt[b, h, i]].
+ *   q, k, v, o : device [B, N, heads, 128] bf16, block-major video segment
+ *   block_idx, block_cnt : as written by mmdit_block_select (ids must be
+ *               ascending and < nblocks; counts in [0, nblocks]); a query block
+ *               with an empty list gets a zero output row
+ *   workspace  : size from mmdit_sparse_attn_workspace_size (per-CTA merged
+ *               block lists)
+ *   Errors     : EINVAL, EUNSUPPORTED, EWORKSPACE, ECUDA.
+ */
+MMDIT_API int mmdit_sparse_attn(const void* q, const void* k, const void* v, void* o,
+                      const mmdit_tensor_desc* desc, const mmdit_layout* layout,
+                      const int32_t* block_idx, const int32_t* block_cnt, int cap,
+                      float scale, void* workspace, size_t ws_bytes,
+                      mmdit_stream_t stream);
+MMDIT_API size_t mmdit_sparse_attn_workspace_size(const mmdit_tensor_desc* desc,
+                                        const mmdit_layout* layout, int cap);
+
+/* Number of 4x4x4 blocks of the single BLOCK444 video segment of `layout`
+ * (0 if the layout is not a single such segment). */
+MMDIT_API int mmdit_num_blocks(const mmdit_layout* layout);
+
+/* Reads and clears the device error flag of the current device after
+ * synchronising `stream`: MMDIT_OK, or MMDIT_ETIMEOUT if a bounded wait ran out
+ * in a kernel since the last call, or MMDIT_ECUDA. */
+MMDIT_API int mmdit_device_status(mmdit_stream_t stream);
+
+/* Thread-local description of the last error returned on this thread. */
+MMDIT_API const char* mmdit_last_error(void);
+
+/* Library version string. */
+MMDIT_API const char* mmdit_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MMDIT_H_ */

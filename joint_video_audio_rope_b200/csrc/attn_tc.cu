@@ -1,0 +1,588 @@
+// Flash-style attention on the sm_100a tensor cores (tcgen05 + tensor memory).
+//
+// Computes O = softmax(Q K^T * scale) V for bf16 Q/K/V with head_dim 128 and
+// fp32 accumulation and softmax state.  One kernel serves every attention of
+// the layer:
+//   * joint self-attention over the concatenated sequence (SkyReels-V4 digest,
+//     arXiv 2602.21818, workflow step 3; SkyReels-V4 blog, section 2.1);
+//   * both directions of the audio<->video cross-attention (same sources;
+//     blog section 2.2), the audio-query direction with the video keys split
+//     across CTAs and merged afterwards (split-KV);
+//   * block-sparse attention restricted to selected key blocks (Prism guide,
+//     arXiv 2610.05416, Method section 3: online-softmax attention over S_i).
+//
+// CTA organisation (320 threads, one CTA per SM):
+//   warps 0-3  softmax warpgroup for Q tile 0 (128 query rows; thread = row)
+//   warps 4-7  softmax warpgroup for Q tile 1
+//   warp 8     TMA producer: Q tiles once, then K/V tiles into a 4-slot ring
+//   warp 9     tensor-memory allocator and single-thread tcgen05.mma issuer
+// Tensor memory (512 columns x 128 lanes of 32 bit):
+//   [0,128) S0 / P0   [128,256) S1 / P1   [256,384) O0   [384,512) O1
+// S = Q K^T lands in TMEM; the softmax warps read it (tcgen05.ld), write the
+// bf16 probabilities P back over the first 64 columns of S (tcgen05.st), and
+// the MMA warp computes O += P V with P as the tensor-memory A operand.  The
+// two Q tiles ping-pong: while one warpgroup runs its softmax, the tensor core
+// works on the other tile.  The running row max is only moved (and O
+// rescaled) when it grows by more than 2^8 in probability units, so O is
+// rarely touched by the softmax warps.
+//
+// Shared-memory tiles use the 128-byte swizzle: a 128 x 128 bf16 tile is two
+// column halves of 64 channels (128 bytes per row); TMA writes them as 64-row
+// boxes.  Q and K are K-major MMA operands; V is an MN-major operand.
+// No TMA multicast is used anywhere.
+#include <math.h>
+
+#include "internal.h"
+
+namespace mmdit {
+
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kStages = 4;                // K/V ring slots (one 128 x 128 tile each)
+constexpr int kTileBytes = 128 * 128 * 2; // 32 KB
+constexpr int kHalfCol = 128 * 128;       // bytes of one 64-channel column half
+constexpr int kBoxBytes = 64 * 128;       // one TMA box: 64 rows x 64 channels
+constexpr int kQOff = 0;
+constexpr int kKVOff = 2 * kTileBytes;
+constexpr int kBarOff = kKVOff + kStages * kTileBytes;
+constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + barriers + alignment slack
+constexpr float kRescaleLog2 = 8.0f;      // move the max only beyond a factor 2^8
+
+// barrier indices (8 bytes each)
+enum {
+  B_QFULL = 0,    // 2: Q tile landed (TMA)
+  B_QREADY = 2,   // 2: Q tile rotated in place (fused RoPE), 128 arrivals
+  B_KVFULL = 4,   // 4: ring slot landed (TMA)
+  B_KVEMPTY = 8,  // 4: ring slot consumed (tcgen05.commit)
+  B_SFULL = 12,   // 2: S tile ready in TMEM
+  B_PFULL = 14,   // 2: P tile written to TMEM (128 arrivals)
+  B_OFULL = 16,   // 2: last PV of the tile done
+  B_MMADONE = 18, // 1: every MMA of the CTA done (teardown)
+  B_COUNT = 19
+};
+
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0, 0);  // Q, K: K-major
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 0, 1);  // P (TMEM), V: MN-major
+
+struct Work {
+  int prob, b, h, split, qtile;
+  int q0;       // first query token of the CTA (row 0 of Q tile 0)
+  int q_valid;  // valid query rows of the CTA (<= 256)
+  int kv_lo, kv_hi;  // dense: key range
+  int nkv;      // number of 128-row key tiles
+  long long ubase;   // sparse: offset of the merged list
+  int g_first, g_nblk;
+};
+
+__device__ __forceinline__ Work decode_work(const AttnParams& P) {
+  Work w;
+  int idx = blockIdx.x;
+  w.prob = 0;
+  if (P.n_prob > 1 && idx >= P.prob[0].ctas) {
+    idx -= P.prob[0].ctas;
+    w.prob = 1;
+  }
+  const AttnProblem& pr = P.prob[w.prob];
+  w.qtile = idx % pr.n_qtiles;
+  idx /= pr.n_qtiles;
+  w.split = idx % pr.n_splits;
+  idx /= pr.n_splits;
+  w.h = idx % pr.H;
+  w.b = idx / pr.H;
+  if (pr.mode == kModeDense) {
+    w.q0 = w.qtile * 256;
+    w.q_valid = min(256, pr.Nq - w.q0);
+    w.kv_lo = w.split * pr.kv_per_split;
+    w.kv_hi = min(pr.Nkv, w.kv_lo + pr.kv_per_split);
+    w.nkv = w.kv_hi > w.kv_lo ? (w.kv_hi - w.kv_lo + 127) / 128 : 0;
+    w.ubase = 0;
+    w.g_first = w.g_nblk = 0;
+  } else {
+    const int4 g = pr.groups[w.qtile];
+    w.g_first = g.x;
+    w.g_nblk = g.y;
+    w.q0 = g.z;
+    w.q_valid = g.w;
+    w.kv_lo = 0;
+    w.kv_hi = pr.Nkv;
+    const long long lid = ((long long)w.b * pr.H + w.h) * pr.n_qtiles + w.qtile;
+    w.ubase = lid * pr.ucap;
+    const int cnt = pr.ucnt[lid];
+    w.nkv = (cnt + 1) / 2;
+  }
+  return w;
+}
+
+// Token start of the two 64-row halves of key tile j, and (sparse) the
+// merged-list entries they come from.
+__device__ __forceinline__ void kv_tile(const AttnProblem& pr, const Work& w, int j, int& s0,
+                                        int& s1, uint32_t& e0, uint32_t& e1) {
+  if (pr.mode == kModeDense) {
+    s0 = w.kv_lo + j * 128;
+    s1 = s0 + 64;
+    e0 = e1 = 0;
+  } else {
+    const int cnt = pr.ucnt[((long long)w.b * pr.H + w.h) * pr.n_qtiles + w.qtile];
+    e0 = pr.ulist[w.ubase + 2 * j];
+    e1 = (2 * j + 1 < cnt) ? pr.ulist[w.ubase + 2 * j + 1] : 0u;
+    int len;
+    block_extent(pr.vT, pr.vH, pr.vW, (int)(e0 & 0xFFFFu), s0, len);
+    if (2 * j + 1 < cnt)
+      block_extent(pr.vT, pr.vH, pr.vW, (int)(e1 & 0xFFFFu), s1, len);
+    else
+      s1 = s0;  // loaded but fully masked
+  }
+}
+
+__device__ __forceinline__ void tma_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                         int h, int b, int s0, int s1) {
+  tma_load_4d(dst, map, bar, 0, h, s0, b);
+  tma_load_4d(dst + kBoxBytes, map, bar, 0, h, s1, b);
+  tma_load_4d(dst + kHalfCol, map, bar, 64, h, s0, b);
+  tma_load_4d(dst + kHalfCol + kBoxBytes, map, bar, 64, h, s1, b);
+}
+
+// S_t = Q_t K^T : M=128 (query rows), N=128 (key rows), K=128 (channels) as
+// 8 MMAs of K=16.  Both operands K-major, 128-byte swizzle; stepping K by 16
+// channels moves the start address 32 bytes inside the swizzle atom, and the
+// second 64-channel half lives kHalfCol bytes further.
+__device__ __forceinline__ void mma_qk(uint32_t s_tmem, uint32_t q_smem, uint32_t k_smem) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t off = (kk >> 2) * kHalfCol + (kk & 3) * 32;
+    const uint64_t a = smem_desc_sw128(q_smem + off, 16, 1024);
+    const uint64_t b = smem_desc_sw128(k_smem + off, 16, 1024);
+    tc_mma_ss(s_tmem, a, b, kIdescQK, kk > 0);
+  }
+}
+
+// O_t (+)= P_t V : M=128, N=128 (channels), K=128 (key rows).  P comes from
+// tensor memory (16 bf16 per row = 8 columns per K step).  V is MN-major:
+// 64-channel halves are LBO = kHalfCol apart, 8-row groups SBO = 1024 apart,
+// and 16 key rows (one K step) are 2048 bytes.
+__device__ __forceinline__ void mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem,
+                                       bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint64_t b = smem_desc_sw128(v_smem + kk * 2048, kHalfCol, 1024);
+    tc_mma_ts(o_tmem, p_tmem + kk * 8, b, kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+// Rotate this thread's Q row (row r of the tile at q_smem) in place by the
+// 3D RoPE angles of token `tok`.
+__device__ void rope_row_smem(uint8_t* q_tile, int r, int tok, const DevLayout& L,
+                              const RopeTab& tab) {
+  float pt, ph, pw;
+  token_position(L, tok, pt, ph, pw);
+#pragma unroll 1
+  for (int j = 0; j < 16; ++j) {  // 16 chunks of 8 channels
+    const int half = j >> 3, jj = j & 7;
+    uint4* p = reinterpret_cast<uint4*>(q_tile + half * kHalfCol + r * 128 +
+                                        ((jj ^ (r & 7)) << 4));
+    uint4 raw = *p;
+    __nv_bfloat162* x = reinterpret_cast<__nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int m = j * 4 + i;
+      const float pos = m < tab.pt ? pt : (m < tab.ph ? ph : pw);
+      float sn, cs;
+      sincosf(pos * tab.omega[m], &sn, &cs);
+      const float2 v = __bfloat1622float2(x[i]);
+      x[i] = __float22bfloat162_rn(make_float2(v.x * cs - v.y * sn, v.x * sn + v.y * cs));
+    }
+    *p = raw;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ AttnParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bars = sbase + kBarOff;
+  auto bar = [&](int i) { return bars + 8u * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + 8 * B_COUNT);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Work w = decode_work(P);
+  const AttnProblem& pr = P.prob[w.prob];
+  int* err = P.err;
+  const bool skip = *(volatile int*)err != 0;  // an earlier kernel timed out
+
+  if (threadIdx.x == 0) {
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(B_QFULL + t), 1);
+      mbar_init(bar(B_QREADY + t), 128);
+      mbar_init(bar(B_SFULL + t), 1);
+      mbar_init(bar(B_PFULL + t), 128);
+      mbar_init(bar(B_OFULL + t), 1);
+    }
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(B_KVFULL + s), 1);
+      mbar_init(bar(B_KVEMPTY + s), 1);
+    }
+    mbar_init(bar(B_MMADONE), 1);
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int nkv = skip ? 0 : w.nkv;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && !skip) {
+      tma_prefetch_desc(&pr.tmQ);
+      tma_prefetch_desc(&pr.tmK);
+      tma_prefetch_desc(&pr.tmV);
+      for (int t = 0; t < 2; ++t) {
+        mbar_expect_tx(bar(B_QFULL + t), kTileBytes);
+        const int s0 = w.q0 + t * 128;
+        tma_tile(sbase + kQOff + t * kTileBytes, &pr.tmQ, bar(B_QFULL + t), w.h, w.b, s0,
+                 s0 + 64);
+      }
+      int last[kStages] = {-1, -1, -1, -1};
+      bool ok = true;
+      for (int j = 0; j < nkv && ok; ++j) {
+        int s0, s1;
+        uint32_t e0, e1;
+        kv_tile(pr, w, j, s0, s1, e0, e1);
+        for (int kind = 0; kind < 2; ++kind) {
+          const int i = 2 * j + kind;
+          const int slot = i % kStages;
+          if (!mbar_wait(bar(B_KVEMPTY + slot), ((i / kStages) & 1) ^ 1, err)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(bar(B_KVFULL + slot), kTileBytes);
+          tma_tile(sbase + kKVOff + slot * kTileBytes, kind ? &pr.tmV : &pr.tmK,
+                   bar(B_KVFULL + slot), w.h, w.b, s0, s1);
+          last[slot] = i;
+        }
+      }
+      // every copy issued must land before the CTA's shared memory goes away
+      for (int t = 0; t < 2; ++t) mbar_wait(bar(B_QFULL + t), 0, err);
+      for (int s = 0; s < kStages; ++s)
+        if (last[s] >= 0) mbar_wait(bar(B_KVFULL + s), (last[s] / kStages) & 1, err);
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && !skip) {
+      bool ok = true;
+      const uint32_t q_s[2] = {sbase + kQOff, sbase + kQOff + kTileBytes};
+      const uint32_t s_t[2] = {tmem, tmem + 128};
+      const uint32_t o_t[2] = {tmem + 256, tmem + 384};
+      const int qbar = pr.rope_q ? B_QREADY : B_QFULL;
+      for (int t = 0; t < 2 && ok; ++t) ok = mbar_wait(bar(qbar + t), 0, err);
+      if (ok && nkv > 0) {
+        // prologue: S_t = Q_t K_0^T for both tiles
+        ok = mbar_wait(bar(B_KVFULL + 0), 0, err);
+        if (ok) {
+          tc_fence_after();
+          mma_qk(s_t[0], q_s[0], sbase + kKVOff);
+          tc_commit(bar(B_SFULL + 0));
+          mma_qk(s_t[1], q_s[1], sbase + kKVOff);
+          tc_commit(bar(B_SFULL + 1));
+          tc_commit(bar(B_KVEMPTY + 0));
+        }
+        for (int j = 0; j < nkv && ok; ++j) {
+          const int iv = 2 * j + 1, ik = 2 * j + 2;
+          const int sv = iv % kStages, sk = ik % kStages;
+          const uint32_t v_smem = sbase + kKVOff + sv * kTileBytes;
+          const uint32_t k_smem = sbase + kKVOff + sk * kTileBytes;
+          const bool more = j + 1 < nkv;
+          if (!(ok = mbar_wait(bar(B_KVFULL + sv), (iv / kStages) & 1, err))) break;
+          if (!(ok = mbar_wait(bar(B_PFULL + 0), j & 1, err))) break;
+          tc_fence_after();
+          mma_pv(o_t[0], s_t[0], v_smem, j > 0);
+          if (more) {
+            if (!(ok = mbar_wait(bar(B_KVFULL + sk), (ik / kStages) & 1, err))) break;
+            tc_fence_after();
+            mma_qk(s_t[0], q_s[0], k_smem);
+            tc_commit(bar(B_SFULL + 0));
+          }
+          if (!(ok = mbar_wait(bar(B_PFULL + 1), j & 1, err))) break;
+          tc_fence_after();
+          mma_pv(o_t[1], s_t[1], v_smem, j > 0);
+          tc_commit(bar(B_KVEMPTY + sv));
+          if (more) {
+            mma_qk(s_t[1], q_s[1], k_smem);
+            tc_commit(bar(B_SFULL + 1));
+            tc_commit(bar(B_KVEMPTY + sk));
+          }
+        }
+      }
+      tc_commit(bar(B_OFULL + 0));
+      tc_commit(bar(B_OFULL + 1));
+      tc_commit(bar(B_MMADONE));
+      mbar_wait(bar(B_MMADONE), 0, err);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int t = warp >> 2;                  // Q tile of this warpgroup
+    const int r = (warp & 3) * 32 + lane;     // row inside the tile == TMEM lane
+    const int row = t * 128 + r;              // row inside the CTA
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t s_addr = tmem + lane_off + t * 128;
+    const uint32_t o_addr = tmem + lane_off + 256 + t * 128;
+    const float sl2 = P.scale_log2;
+    const float thresh = kRescaleLog2 / sl2;  // in raw score units
+    bool ok = !skip;
+
+    if (ok && pr.rope_q) {
+      ok = mbar_wait(bar(B_QFULL + t), 0, err);
+      if (ok) {
+        rope_row_smem(smem + kQOff + t * kTileBytes, r, w.q0 + row, P.layout, P.rope);
+        fence_proxy_async_smem();
+      }
+      mbar_arrive(bar(B_QREADY + t));
+    }
+
+    // sparse mode: which query block of the group this row belongs to
+    int qb = 0;
+    if (pr.mode == kModeSparse) {
+      int acc = 0;
+      qb = 31;  // rows past the group: member of nothing
+      for (int i = 0; i < w.g_nblk; ++i) {
+        int st, len;
+        block_extent(pr.vT, pr.vH, pr.vW, w.g_first + i, st, len);
+        if (row < acc + len) {
+          qb = i;
+          break;
+        }
+        acc += len;
+      }
+    }
+
+    float m_used = -INFINITY, l = 0.f;
+    for (int j = 0; j < nkv; ++j) {
+      ok = ok && mbar_wait(bar(B_SFULL + t), j & 1, err);
+      if (__any_sync(0xffffffffu, !ok)) {
+        ok = false;
+        break;
+      }
+      __syncwarp();
+      tc_fence_after();
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(s_addr + c * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(v[i]);
+      }
+      // valid key columns of each 64-row half for this row
+      int len0, len1;
+      if (pr.mode == kModeDense) {
+        const int s0 = w.kv_lo + j * 128;
+        len0 = max(0, min(64, w.kv_hi - s0));
+        len1 = max(0, min(64, w.kv_hi - s0 - 64));
+      } else {
+        const int cnt = pr.ucnt[((long long)w.b * pr.H + w.h) * pr.n_qtiles + w.qtile];
+        const uint32_t e0 = pr.ulist[w.ubase + 2 * j];
+        const uint32_t e1 = (2 * j + 1 < cnt) ? pr.ulist[w.ubase + 2 * j + 1] : 0u;
+        int st;
+        block_extent(pr.vT, pr.vH, pr.vW, (int)(e0 & 0xFFFFu), st, len0);
+        len0 = ((e0 >> 16) >> qb) & 1u ? len0 : 0;
+        if (2 * j + 1 < cnt) {
+          block_extent(pr.vT, pr.vH, pr.vW, (int)(e1 & 0xFFFFu), st, len1);
+          len1 = ((e1 >> 16) >> qb) & 1u ? len1 : 0;
+        } else {
+          len1 = 0;
+        }
+      }
+      if (len0 < 64 || len1 < 64) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          if (c >= len0) s[c] = -INFINITY;
+          if (c >= len1) s[64 + c] = -INFINITY;
+        }
+      }
+      float mt = s[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mt = fmaxf(mt, s[c]);
+      const bool grow = mt > m_used + thresh || (m_used == -INFINITY && mt > -INFINITY);
+      float alpha = 1.f;
+      if (grow) {
+        alpha = (m_used == -INFINITY) ? 0.f : ex2_approx((m_used - mt) * sl2);
+        m_used = mt;
+        l *= alpha;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        // rescale the running O of this row (previous PV is complete: it was
+        // issued before the QK whose completion released this S tile)
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld32(o_addr + c * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+          tmem_st32(o_addr + c * 32, v);
+        }
+        tmem_wait_st();
+      }
+      const float mref = (m_used == -INFINITY) ? 0.f : m_used * sl2;
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = ex2_approx(fmaf(s[c * 64 + 2 * i], sl2, -mref));
+          const float p1 = ex2_approx(fmaf(s[c * 64 + 2 * i + 1], sl2, -mref));
+          v[i] = pack_bf16x2(p0, p1);
+          sum += p0 + p1;
+        }
+        tmem_st32(s_addr + c * 32, v);
+      }
+      tmem_wait_st();
+      l += sum;
+      tc_fence_before();
+      mbar_arrive(bar(B_PFULL + t));
+    }
+
+    // ------------------------------------------------------------ epilogue
+    if (ok && nkv > 0) ok = mbar_wait(bar(B_OFULL + t), 0, err);
+    const bool all_ok = !__any_sync(0xffffffffu, !ok);
+    __syncwarp();
+    if (all_ok && !skip) {
+      tc_fence_after();
+      const bool valid_row = row < w.q_valid;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const int qrow = w.q0 + row;
+      if (pr.part_o != nullptr) {
+        // split-KV partial: unnormalised O, running max (log2 units) and sum
+        const long long prow =
+            (((long long)w.split * pr.B + w.b) * pr.H + w.h) * (long long)(pr.n_qtiles * 256) +
+            (long long)w.qtile * 256 + row;
+        float* dst = pr.part_o + prow * 128;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          if (nkv > 0) {
+            tmem_ld32(o_addr + c * 32, v);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
+          }
+          if (valid_row) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(dst + c * 32 + i) =
+                  make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                              __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+          }
+        }
+        if (valid_row) {
+          pr.part_ml[prow * 2 + 0] = (m_used == -INFINITY) ? -INFINITY : m_used * sl2;
+          pr.part_ml[prow * 2 + 1] = l;
+        }
+      } else {
+        __nv_bfloat16* dst = pr.o + (long long)w.b * pr.o_sb + (long long)qrow * pr.o_st +
+                             (long long)w.h * 128;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          if (nkv > 0) {
+            tmem_ld32(o_addr + c * 32, v);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
+          }
+          if (valid_row) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              uint4 pk;
+              pk.x = pack_bf16x2(__uint_as_float(v[i + 0]) * inv, __uint_as_float(v[i + 1]) * inv);
+              pk.y = pack_bf16x2(__uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv);
+              pk.z = pack_bf16x2(__uint_as_float(v[i + 4]) * inv, __uint_as_float(v[i + 5]) * inv);
+              pk.w = pack_bf16x2(__uint_as_float(v[i + 6]) * inv, __uint_as_float(v[i + 7]) * inv);
+              *reinterpret_cast<uint4*>(dst + c * 32 + i) = pk;
+            }
+          }
+        }
+        if (pr.lse != nullptr && valid_row) {
+          const float mref = (m_used == -INFINITY) ? 0.f : m_used * sl2;
+          pr.lse[((long long)w.b * pr.H + w.h) * pr.Nq + qrow] =
+              l > 0.f ? (mref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Merge split-KV partials: O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
+__global__ void split_combine_kernel(const float* __restrict__ part_o,
+                                     const float* __restrict__ part_ml, __nv_bfloat16* o,
+                                     long long o_st, long long o_sb, int n_splits, int B, int H,
+                                     int Nq, int Nq_pad) {
+  const int row = blockIdx.x;  // over B * H * Nq
+  const int q = row % Nq;
+  const int h = (row / Nq) % H;
+  const int b = row / (Nq * H);
+  const int c = threadIdx.x;   // channel (128 threads)
+  float M = -INFINITY;
+  for (int s = 0; s < n_splits; ++s) {
+    const long long pr = (((long long)s * B + b) * H + h) * Nq_pad + q;
+    M = fmaxf(M, part_ml[pr * 2]);
+  }
+  float L = 0.f, acc = 0.f;
+  for (int s = 0; s < n_splits; ++s) {
+    const long long pr = (((long long)s * B + b) * H + h) * Nq_pad + q;
+    const float m = part_ml[pr * 2];
+    if (m == -INFINITY) continue;
+    const float f = exp2f(m - M);
+    L += f * part_ml[pr * 2 + 1];
+    acc += f * part_o[pr * 128 + c];
+  }
+  o[(long long)b * o_sb + (long long)q * o_st + (long long)h * 128 + c] =
+      __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
+}
+
+}  // namespace
+
+cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int ctas = p.prob[0].ctas + (p.n_prob > 1 ? p.prob[1].ctas : 0);
+  if (ctas == 0) return cudaSuccess;
+  attn_tc_kernel<<<ctas, kThreads, kSmemBytes, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_split_combine(const float* part_o, const float* part_ml, __nv_bfloat16* o,
+                                 long long o_st, long long o_sb, int n_splits, int B, int H,
+                                 int Nq, int Nq_pad, cudaStream_t s) {
+  if (B * H * Nq == 0) return cudaSuccess;
+  split_combine_kernel<<<B * H * Nq, 128, 0, s>>>(part_o, part_ml, o, o_st, o_sb, n_splits, B, H,
+                                                 Nq, Nq_pad);
+  return cudaGetLastError();
+}
+
+}  // namespace mmdit

@@ -1,0 +1,84 @@
+// Launchers shared between the C-ABI front end (mmdit_api.cu) and the kernel
+// translation units.  Host-only declarations; not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace mmdit {
+
+// RoPE (rope.cu)
+cudaError_t launch_rope(void* q, void* k, const mmdit_tensor_desc& d, const DevLayout& L,
+                        const RopeTab& tab, cudaStream_t s);
+
+// fp32 SIMT attention (attn_f32.cu): o = softmax(q k^T scale) v per (b, h);
+// optional lse [B, H, Nq].
+struct F32AttnArgs {
+  const float *q, *k, *v;
+  float* o;
+  float* lse;
+  int B, H, D, Nq, Nkv;
+  long long q_st, q_sb, k_st, k_sb, v_st, v_sb, o_st, o_sb;  // strides in elements
+  float scale;
+};
+cudaError_t launch_attn_f32(const F32AttnArgs& a, cudaStream_t s);
+
+// tcgen05 bf16 attention (attn_tc.cu)
+enum AttnMode { kModeDense = 0, kModeSparse = 1 };
+
+struct AttnProblem {
+  CUtensorMap tmQ, tmK, tmV;  // 4D maps {channel, head, token, batch}, box {64,1,64,1}
+  __nv_bfloat16* o;           // output (dense/sparse), or nullptr when writing partials
+  long long o_st, o_sb;       // output strides (elements)
+  float* lse;                 // [B, H, Nq] or nullptr
+  float* part_o;              // split-KV partials [split][B][H][Nq_pad][128] (unnormalised)
+  float* part_ml;             // split-KV partials [split][B][H][Nq_pad][2] (m*log2e*scale, l)
+  int Nq, Nkv, H, B;
+  int n_qtiles;               // ceil(Nq / 256) (dense) or number of groups (sparse)
+  int n_splits;               // KV splits per (q tile pair, head, batch)
+  int kv_per_split;           // tokens per split, multiple of 128
+  int ctas;                   // n_qtiles * H * B * n_splits
+  int mode;                   // AttnMode
+  // sparse mode: the query groups and the merged key-block lists
+  const int4* groups;         // per group: {first block, n blocks, start token, n tokens}
+  const uint32_t* ulist;      // [B][H][n_groups][ucap]: block id | member mask << 16
+  const int* ucnt;            // [B][H][n_groups]
+  int ucap;
+  int vT, vH, vW;             // block-major video grid (sparse mode)
+  int rope_q;                 // rotate Q tiles in shared memory after loading
+};
+
+struct AttnParams {
+  AttnProblem prob[2];
+  int n_prob;
+  float scale_log2;           // softmax scale * log2(e)
+  DevLayout layout;           // for fused Q RoPE
+  RopeTab rope;
+  int* err;                   // device error flag
+};
+
+cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s);
+cudaError_t launch_split_combine(const float* part_o, const float* part_ml, __nv_bfloat16* o,
+                                 long long o_st, long long o_sb, int n_splits, int B, int H,
+                                 int Nq, int Nq_pad, cudaStream_t s);
+
+// block selection (select.cu)
+cudaError_t launch_pool(const __nv_bfloat16* q, const __nv_bfloat16* k, const mmdit_tensor_desc& d,
+                        int T, int H, int W, int nblk, float* qbar, float* kbar, cudaStream_t s);
+cudaError_t launch_select(const float* qbar, const float* kbar, int B, int H, int nblk, int top_k,
+                          float top_p, float scale, int cap, int32_t* idx, int32_t* cnt,
+                          cudaStream_t s);
+size_t select_smem_bytes(int nblk);
+cudaError_t launch_groups(int T, int H, int W, int nblk, int4* groups, int* n_groups,
+                          cudaStream_t s);
+cudaError_t launch_union(const int32_t* idx, const int32_t* cnt, int cap, const int4* groups,
+                         int n_groups_max, const int* n_groups, int B, int H, int nblk,
+                         uint32_t* ulist, int* ucnt, cudaStream_t s);
+
+// helpers (mmdit_api.cu)
+int* device_error_flag();  // device address of this device's error word
+
+}  // namespace mmdit

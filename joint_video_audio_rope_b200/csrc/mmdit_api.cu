@@ -1,0 +1,573 @@
+// C-ABI front end of the library (declared in include/mmdit.h): argument
+// validation, TMA tensor-map encoding and kernel launches.  Every argument is
+// checked before anything is launched; no call allocates device memory.
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <mutex>
+#include <string>
+
+#include "internal.h"
+
+namespace mmdit {
+
+__device__ int g_device_error_word = 0;
+
+namespace {
+
+thread_local std::string t_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(MMDIT_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_desc(const mmdit_tensor_desc* d, const char* name) {
+  if (d == nullptr) return fail(MMDIT_EINVAL, "%s: descriptor is NULL", name);
+  if (d->batch < 1 || d->n_tokens < 0 || d->heads < 1)
+    return fail(MMDIT_EINVAL, "%s: batch=%d n_tokens=%d heads=%d out of range", name, d->batch,
+                d->n_tokens, d->heads);
+  if (d->dtype != MMDIT_BF16 && d->dtype != MMDIT_F32)
+    return fail(MMDIT_EUNSUPPORTED, "%s: dtype %d not supported", name, d->dtype);
+  if (d->dtype == MMDIT_BF16 && d->head_dim != 128)
+    return fail(MMDIT_EUNSUPPORTED, "%s: bf16 needs head_dim 128 (got %d)", name, d->head_dim);
+  if (d->dtype == MMDIT_F32 && d->head_dim != 64 && d->head_dim != 128)
+    return fail(MMDIT_EUNSUPPORTED, "%s: f32 needs head_dim 64 or 128 (got %d)", name,
+                d->head_dim);
+  const long long row = (long long)d->heads * d->head_dim;
+  if (d->stride_tok < row)
+    return fail(MMDIT_EINVAL, "%s: stride_tok %lld < heads*head_dim %lld", name, d->stride_tok, row);
+  if (d->batch > 1 && d->stride_batch < d->stride_tok * (long long)d->n_tokens)
+    return fail(MMDIT_EINVAL, "%s: stride_batch %lld overlaps batch items", name, d->stride_batch);
+  const int es = d->dtype == MMDIT_BF16 ? 2 : 4;
+  if ((d->stride_tok * es) % 16 != 0 || (d->stride_batch * es) % 16 != 0)
+    return fail(MMDIT_EINVAL, "%s: strides must be multiples of 16 bytes", name);
+  return MMDIT_OK;
+}
+
+int check_layout(const mmdit_layout* L, int n_tokens) {
+  if (L == nullptr) return fail(MMDIT_EINVAL, "layout is NULL");
+  if (L->n_seg < 1 || L->n_seg > MMDIT_MAX_SEGMENTS)
+    return fail(MMDIT_EINVAL, "layout: n_seg %d outside [1, %d]", L->n_seg, MMDIT_MAX_SEGMENTS);
+  long long total = 0;
+  for (int i = 0; i < L->n_seg; ++i) {
+    const mmdit_segment& s = L->seg[i];
+    if (s.n_tokens < 0) return fail(MMDIT_EINVAL, "layout: segment %d has n_tokens < 0", i);
+    if (s.kind == MMDIT_SEG_VIDEO) {
+      if (s.T < 1 || s.H < 1 || s.W < 1 || (long long)s.T * s.H * s.W != s.n_tokens)
+        return fail(MMDIT_EINVAL, "layout: video segment %d: T*H*W != n_tokens", i);
+      if (s.order != MMDIT_ORDER_RASTER && s.order != MMDIT_ORDER_BLOCK444)
+        return fail(MMDIT_EINVAL, "layout: segment %d: bad order %d", i, s.order);
+    } else if (s.kind == MMDIT_SEG_AUDIO) {
+      if (s.t_den < 1 || s.t_num < 0 || (long long)s.n_tokens * s.t_num > 0x7fffffffLL)
+        return fail(MMDIT_EINVAL, "layout: audio segment %d: bad t_num/t_den", i);
+    } else if (s.kind != MMDIT_SEG_TEXT) {
+      return fail(MMDIT_EINVAL, "layout: segment %d: bad kind %d", i, s.kind);
+    }
+    total += s.n_tokens;
+  }
+  if (total != n_tokens)
+    return fail(MMDIT_EINVAL, "layout: segments hold %lld tokens, tensor has %d", total, n_tokens);
+  return MMDIT_OK;
+}
+
+DevLayout to_dev(const mmdit_layout* L) {
+  DevLayout d{};
+  d.n_seg = L->n_seg;
+  int start = 0;
+  for (int i = 0; i < L->n_seg; ++i) {
+    const mmdit_segment& s = L->seg[i];
+    d.seg[i] = DevSeg{s.kind, start, s.n_tokens, s.T, s.H, s.W, s.t0, s.t_num, s.t_den, s.order};
+    start += s.n_tokens;
+  }
+  return d;
+}
+
+int make_rope_tab(const mmdit_rope_params* r, int head_dim, RopeTab& tab) {
+  if (r == nullptr) return fail(MMDIT_EINVAL, "rope parameters are NULL");
+  if (!(r->theta > 0.f) || r->dim_t < 0 || r->dim_h < 0 || r->dim_w < 0 || (r->dim_t & 1) ||
+      (r->dim_h & 1) || (r->dim_w & 1) || r->dim_t + r->dim_h + r->dim_w != head_dim)
+    return fail(MMDIT_EINVAL, "rope: need theta > 0 and even dims summing to head_dim %d",
+                head_dim);
+  tab = RopeTab{};
+  tab.pt = r->dim_t / 2;
+  tab.ph = (r->dim_t + r->dim_h) / 2;
+  tab.npairs = head_dim / 2;
+  const int dims[3] = {r->dim_t, r->dim_h, r->dim_w};
+  int m = 0;
+  for (int a = 0; a < 3; ++a)
+    for (int i = 0; i < dims[a] / 2; ++i, ++m)
+      tab.omega[m] = (float)pow((double)r->theta, -2.0 * i / (double)dims[a]);
+  return MMDIT_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 4D map {channel, head, token, batch} over a bf16 [B, N, heads, 128] tensor,
+// box {64, 1, 64, 1}, 128-byte swizzle, zero fill out of bounds.
+int make_map(CUtensorMap* m, const void* base, const mmdit_tensor_desc& d, int n_tokens,
+             const char* name) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(MMDIT_ECUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[4] = {128, (cuuint64_t)d.heads, (cuuint64_t)n_tokens, (cuuint64_t)d.batch};
+  cuuint64_t strides[3] = {128 * 2, (cuuint64_t)d.stride_tok * 2,
+                           (cuuint64_t)(d.batch > 1 ? d.stride_batch : d.stride_tok * n_tokens) * 2};
+  cuuint32_t box[4] = {64, 1, 64, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MMDIT_ECUDA, "%s: tensor map encoding failed (%d)", name, (int)r);
+  return MMDIT_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int check_sm100() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0)
+    return fail(MMDIT_EUNSUPPORTED, "device %d is sm_%d%d; this library targets sm_100a", dev,
+                major, minor);
+  return MMDIT_OK;
+}
+
+// single BLOCK444 video segment -> grid and block count
+int sparse_layout(const mmdit_layout* L, const mmdit_tensor_desc* d, int& T, int& H, int& W,
+                  int& nblk) {
+  int rc = check_layout(L, d->n_tokens);
+  if (rc) return rc;
+  if (L->n_seg != 1 || L->seg[0].kind != MMDIT_SEG_VIDEO || L->seg[0].order != MMDIT_ORDER_BLOCK444)
+    return fail(MMDIT_EINVAL, "block-sparse calls need exactly one BLOCK444 video segment");
+  T = L->seg[0].T;
+  H = L->seg[0].H;
+  W = L->seg[0].W;
+  const long long nb = (long long)((T + 3) / 4) * ((H + 3) / 4) * ((W + 3) / 4);
+  if (nb > 6000)
+    return fail(MMDIT_EUNSUPPORTED, "%lld blocks; at most 6000 are supported", nb);
+  nblk = (int)nb;
+  return MMDIT_OK;
+}
+
+int host_block_len(int T, int H, int W, int b) {
+  const int nhb = (H + 3) / 4, nwb = (W + 3) / 4;
+  const int tb = b / (nhb * nwb), r = b % (nhb * nwb), hb = r / nwb, wb = r % nwb;
+  return std::min(4, T - 4 * tb) * std::min(4, H - 4 * hb) * std::min(4, W - 4 * wb);
+}
+
+// greedy grouping of query blocks (<= 256 tokens, <= 16 blocks); the device
+// groups_kernel applies the same rule and writes the table.
+int host_group_count(int T, int H, int W, int nblk) {
+  int g = 0, nb = 0, tokens = 0;
+  for (int b = 0; b < nblk; ++b) {
+    const int len = host_block_len(T, H, W, b);
+    if (nb == 16 || tokens + len > 256) {
+      ++g;
+      nb = 0;
+      tokens = 0;
+    }
+    ++nb;
+    tokens += len;
+  }
+  return g + (nb > 0 ? 1 : 0);
+}
+
+struct CrossPlan {
+  int n_qtiles_a, splits, kv_per_split, nq_pad;
+  size_t part_o_bytes, part_ml_bytes;
+};
+
+CrossPlan plan_cross(const mmdit_tensor_desc* v, const mmdit_tensor_desc* a) {
+  CrossPlan p{};
+  p.n_qtiles_a = (a->n_tokens + 255) / 256;
+  const int tiles = (v->n_tokens + 127) / 128;
+  p.splits = std::max(1, (tiles + 31) / 32);
+  p.kv_per_split = ((tiles + p.splits - 1) / p.splits) * 128;
+  p.splits = std::max(1, (v->n_tokens + p.kv_per_split - 1) / p.kv_per_split);
+  p.nq_pad = p.n_qtiles_a * 256;
+  const size_t rows = (size_t)p.splits * a->batch * a->heads * p.nq_pad;
+  p.part_o_bytes = align256(rows * 128 * sizeof(float));
+  p.part_ml_bytes = align256(rows * 2 * sizeof(float));
+  return p;
+}
+
+}  // namespace
+
+int* device_error_flag() {
+  static int* cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (cache[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error_word) != cudaSuccess) return nullptr;
+    cache[dev] = static_cast<int*>(p);
+  }
+  return cache[dev];
+}
+
+}  // namespace mmdit
+
+using namespace mmdit;
+
+extern "C" {
+
+const char* mmdit_last_error(void) { return t_last_error.c_str(); }
+
+const char* mmdit_version(void) { return "mmdit-av-attn 0.1.0 (sm_100a)"; }
+
+int mmdit_num_blocks(const mmdit_layout* L) {
+  if (L == nullptr || L->n_seg != 1 || L->seg[0].kind != MMDIT_SEG_VIDEO ||
+      L->seg[0].order != MMDIT_ORDER_BLOCK444 || L->seg[0].T < 1 || L->seg[0].H < 1 ||
+      L->seg[0].W < 1)
+    return 0;
+  return ((L->seg[0].T + 3) / 4) * ((L->seg[0].H + 3) / 4) * ((L->seg[0].W + 3) / 4);
+}
+
+int mmdit_device_status(mmdit_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_error_word, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error flag");
+  if (v != 0) {
+    const int zero = 0;
+    cudaMemcpyToSymbol(g_device_error_word, &zero, sizeof(int));
+    return fail(v, "a bounded device wait ran out (status %d)", v);
+  }
+  return MMDIT_OK;
+}
+
+int mmdit_rope_apply(void* q, void* k, const mmdit_tensor_desc* desc, const mmdit_layout* layout,
+                     const mmdit_rope_params* rope, mmdit_stream_t stream) {
+  int rc = check_desc(desc, "rope");
+  if (rc) return rc;
+  if (q == nullptr && k == nullptr) return fail(MMDIT_EINVAL, "rope: q and k are both NULL");
+  if ((q && !aligned16(q)) || (k && !aligned16(k)))
+    return fail(MMDIT_EINVAL, "rope: tensors must be 16-byte aligned");
+  if ((rc = check_layout(layout, desc->n_tokens))) return rc;
+  RopeTab tab;
+  if ((rc = make_rope_tab(rope, desc->head_dim, tab))) return rc;
+  if (desc->n_tokens == 0) return MMDIT_OK;
+  cudaError_t e = launch_rope(q, k, *desc, to_dev(layout), tab, (cudaStream_t)stream);
+  return e == cudaSuccess ? MMDIT_OK : cuda_fail(e, "rope launch");
+}
+
+size_t mmdit_joint_attn_workspace_size(const mmdit_tensor_desc*) { return 0; }
+
+int mmdit_joint_attn(const void* q, const void* k, const void* v, void* o, float* lse,
+                     const mmdit_tensor_desc* desc, const mmdit_layout* layout, float scale,
+                     const mmdit_rope_params* rope_q, const uint8_t* cond_mask, int64_t mask_elems,
+                     void*, size_t, mmdit_stream_t stream) {
+  int rc = check_desc(desc, "joint_attn");
+  if (rc) return rc;
+  if (!q || !k || !v || !o) return fail(MMDIT_EINVAL, "joint_attn: q, k, v, o must be non-NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(MMDIT_EINVAL, "joint_attn: tensors must be 16-byte aligned");
+  if (o == q || o == k || o == v) return fail(MMDIT_EINVAL, "joint_attn: o aliases an input");
+  if (!(scale > 0.f) || !isfinite(scale)) return fail(MMDIT_EINVAL, "joint_attn: scale must be > 0");
+  if ((rc = check_layout(layout, desc->n_tokens))) return rc;
+  if (cond_mask != nullptr) {
+    // the channel-concat mask M: carried with the inputs, never applied
+    long long frames = 0;
+    int mh = -1, mw = -1;
+    for (int i = 0; i < layout->n_seg; ++i) {
+      const mmdit_segment& s = layout->seg[i];
+      if (s.kind != MMDIT_SEG_VIDEO) continue;
+      if (mh >= 0 && (s.H != mh || s.W != mw))
+        return fail(MMDIT_EINVAL, "joint_attn: video segments disagree on H, W for the mask");
+      mh = s.H;
+      mw = s.W;
+      frames += s.T;
+    }
+    const long long expect = mh < 0 ? 0 : (long long)desc->batch * frames * mh * mw;
+    if (mask_elems != expect)
+      return fail(MMDIT_EINVAL, "joint_attn: mask has %lld elements, expected B*F*H*W = %lld",
+                  (long long)mask_elems, expect);
+  }
+  RopeTab tab{};
+  if (rope_q != nullptr) {
+    if (desc->dtype != MMDIT_BF16)
+      return fail(MMDIT_EUNSUPPORTED, "joint_attn: fused Q RoPE needs bf16");
+    if ((rc = make_rope_tab(rope_q, desc->head_dim, tab))) return rc;
+  }
+  if (desc->n_tokens == 0) return MMDIT_OK;
+  if (desc->dtype == MMDIT_F32) {
+    F32AttnArgs a{(const float*)q, (const float*)k, (const float*)v, (float*)o, lse,
+                  desc->batch, desc->heads, desc->head_dim, desc->n_tokens, desc->n_tokens,
+                  desc->stride_tok, desc->stride_batch, desc->stride_tok, desc->stride_batch,
+                  desc->stride_tok, desc->stride_batch, desc->stride_tok, desc->stride_batch, scale};
+    cudaError_t e = launch_attn_f32(a, (cudaStream_t)stream);
+    return e == cudaSuccess ? MMDIT_OK : cuda_fail(e, "attn_f32 launch");
+  }
+  if ((rc = check_sm100())) return rc;
+  AttnParams p{};
+  AttnProblem& pr = p.prob[0];
+  if ((rc = make_map(&pr.tmQ, q, *desc, desc->n_tokens, "q")) ||
+      (rc = make_map(&pr.tmK, k, *desc, desc->n_tokens, "k")) ||
+      (rc = make_map(&pr.tmV, v, *desc, desc->n_tokens, "v")))
+    return rc;
+  pr.o = (__nv_bfloat16*)o;
+  pr.o_st = desc->stride_tok;
+  pr.o_sb = desc->stride_batch;
+  pr.lse = lse;
+  pr.Nq = pr.Nkv = desc->n_tokens;
+  pr.H = desc->heads;
+  pr.B = desc->batch;
+  pr.n_qtiles = (desc->n_tokens + 255) / 256;
+  pr.n_splits = 1;
+  pr.kv_per_split = ((desc->n_tokens + 127) / 128) * 128;
+  pr.ctas = pr.n_qtiles * pr.H * pr.B;
+  pr.mode = kModeDense;
+  pr.rope_q = rope_q != nullptr;
+  p.n_prob = 1;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.layout = to_dev(layout);
+  p.rope = tab;
+  p.err = device_error_flag();
+  if (p.err == nullptr) return fail(MMDIT_ECUDA, "device error flag unavailable");
+  cudaError_t e = launch_attn_tc(p, (cudaStream_t)stream);
+  return e == cudaSuccess ? MMDIT_OK : cuda_fail(e, "attn_tc launch");
+}
+
+size_t mmdit_av_cross_attn_workspace_size(const mmdit_tensor_desc* video,
+                                          const mmdit_tensor_desc* audio) {
+  if (video == nullptr || audio == nullptr || video->dtype != MMDIT_BF16) return 0;
+  if (check_desc(video, "video") || check_desc(audio, "audio")) return 0;
+  const CrossPlan c = plan_cross(video, audio);
+  return c.part_o_bytes + c.part_ml_bytes;
+}
+
+int mmdit_av_cross_attn(const void* qv, const void* kv, const void* vv, const void* qa,
+                        const void* ka, const void* va, void* o_video, void* o_audio,
+                        const mmdit_tensor_desc* video, const mmdit_tensor_desc* audio,
+                        float scale, void* workspace, size_t ws_bytes, mmdit_stream_t stream) {
+  int rc;
+  if ((rc = check_desc(video, "video")) || (rc = check_desc(audio, "audio"))) return rc;
+  if (video->batch != audio->batch || video->heads != audio->heads ||
+      video->head_dim != audio->head_dim || video->dtype != audio->dtype)
+    return fail(MMDIT_EINVAL, "av_cross: video and audio descriptors disagree");
+  const void* ptrs[8] = {qv, kv, vv, qa, ka, va, o_video, o_audio};
+  for (const void* p : ptrs) {
+    if (p == nullptr) return fail(MMDIT_EINVAL, "av_cross: every tensor must be non-NULL");
+    if (!aligned16(p)) return fail(MMDIT_EINVAL, "av_cross: tensors must be 16-byte aligned");
+  }
+  if (video->n_tokens < 1 || audio->n_tokens < 1)
+    return fail(MMDIT_EINVAL, "av_cross: both streams need at least one token");
+  if (!(scale > 0.f) || !isfinite(scale)) return fail(MMDIT_EINVAL, "av_cross: scale must be > 0");
+  cudaStream_t s = (cudaStream_t)stream;
+  if (video->dtype == MMDIT_F32) {
+    F32AttnArgs a1{(const float*)qv, (const float*)ka, (const float*)va, (float*)o_video, nullptr,
+                   video->batch, video->heads, video->head_dim, video->n_tokens, audio->n_tokens,
+                   video->stride_tok, video->stride_batch, audio->stride_tok, audio->stride_batch,
+                   audio->stride_tok, audio->stride_batch, video->stride_tok, video->stride_batch,
+                   scale};
+    F32AttnArgs a2{(const float*)qa, (const float*)kv, (const float*)vv, (float*)o_audio, nullptr,
+                   audio->batch, audio->heads, audio->head_dim, audio->n_tokens, video->n_tokens,
+                   audio->stride_tok, audio->stride_batch, video->stride_tok, video->stride_batch,
+                   video->stride_tok, video->stride_batch, audio->stride_tok, audio->stride_batch,
+                   scale};
+    cudaError_t e = launch_attn_f32(a1, s);
+    if (e == cudaSuccess) e = launch_attn_f32(a2, s);
+    return e == cudaSuccess ? MMDIT_OK : cuda_fail(e, "attn_f32 launch");
+  }
+  const CrossPlan c = plan_cross(video, audio);
+  if (workspace == nullptr || ws_bytes < c.part_o_bytes + c.part_ml_bytes)
+    return fail(MMDIT_EWORKSPACE, "av_cross: workspace needs %zu bytes", c.part_o_bytes + c.part_ml_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(MMDIT_EINVAL, "av_cross: workspace must be 256-byte aligned");
+  if ((rc = check_sm100())) return rc;
+  AttnParams p{};
+  // problem 0: audio queries over the video keys, split across CTAs
+  AttnProblem& a2v = p.prob[0];
+  if ((rc = make_map(&a2v.tmQ, qa, *audio, audio->n_tokens, "qa")) ||
+      (rc = make_map(&a2v.tmK, kv, *video, video->n_tokens, "kv")) ||
+      (rc = make_map(&a2v.tmV, vv, *video, video->n_tokens, "vv")))
+    return rc;
+  a2v.o = nullptr;
+  a2v.part_o = reinterpret_cast<float*>(workspace);
+  a2v.part_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + c.part_o_bytes);
+  a2v.Nq = audio->n_tokens;
+  a2v.Nkv = video->n_tokens;
+  a2v.H = audio->heads;
+  a2v.B = audio->batch;
+  a2v.n_qtiles = c.n_qtiles_a;
+  a2v.n_splits = c.splits;
+  a2v.kv_per_split = c.kv_per_split;
+  a2v.ctas = a2v.n_qtiles * a2v.n_splits * a2v.H * a2v.B;
+  a2v.mode = kModeDense;
+  // problem 1: video queries over the audio keys
+  AttnProblem& v2a = p.prob[1];
+  if ((rc = make_map(&v2a.tmQ, qv, *video, video->n_tokens, "qv")) ||
+      (rc = make_map(&v2a.tmK, ka, *audio, audio->n_tokens, "ka")) ||
+      (rc = make_map(&v2a.tmV, va, *audio, audio->n_tokens, "va")))
+    return rc;
+  v2a.o = (__nv_bfloat16*)o_video;
+  v2a.o_st = video->stride_tok;
+  v2a.o_sb = video->stride_batch;
+  v2a.Nq = video->n_tokens;
+  v2a.Nkv = audio->n_tokens;
+  v2a.H = video->heads;
+  v2a.B = video->batch;
+  v2a.n_qtiles = (video->n_tokens + 255) / 256;
+  v2a.n_splits = 1;
+  v2a.kv_per_split = ((audio->n_tokens + 127) / 128) * 128;
+  v2a.ctas = v2a.n_qtiles * v2a.H * v2a.B;
+  v2a.mode = kModeDense;
+  p.n_prob = 2;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.err = device_error_flag();
+  if (p.err == nullptr) return fail(MMDIT_ECUDA, "device error flag unavailable");
+  cudaError_t e = launch_attn_tc(p, s);
+  if (e == cudaSuccess)
+    e = launch_split_combine(a2v.part_o, a2v.part_ml, (__nv_bfloat16*)o_audio, audio->stride_tok,
+                             audio->stride_batch, c.splits, audio->batch, audio->heads,
+                             audio->n_tokens, c.nq_pad, s);
+  return e == cudaSuccess ? MMDIT_OK : cuda_fail(e, "av_cross launch");
+}
+
+size_t mmdit_block_select_workspace_size(const mmdit_tensor_desc* desc, const mmdit_layout* layout) {
+  int T, H, W, nblk;
+  if (check_desc(desc, "block_select") || sparse_layout(layout, desc, T, H, W, nblk)) return 0;
+  return 2 * align256((size_t)desc->batch * desc->heads * nblk * 128 * sizeof(float));
+}
+
+int mmdit_block_select(const void* q, const void* k, const mmdit_tensor_desc* desc,
+                       const mmdit_layout* layout, int top_k, float top_p, float scale, int cap,
+                       int32_t* block_idx, int32_t* block_cnt, void* workspace, size_t ws_bytes,
+                       mmdit_stream_t stream) {
+  int rc = check_desc(desc, "block_select");
+  if (rc) return rc;
+  if (desc->dtype != MMDIT_BF16) return fail(MMDIT_EUNSUPPORTED, "block_select: bf16 only");
+  if (!q || !k || !block_idx || !block_cnt)
+    return fail(MMDIT_EINVAL, "block_select: q, k, block_idx, block_cnt must be non-NULL");
+  if (!aligned16(q) || !aligned16(k)) return fail(MMDIT_EINVAL, "block_select: 16-byte alignment");
+  int T, H, W, nblk;
+  if ((rc = sparse_layout(layout, desc, T, H, W, nblk))) return rc;
+  if (cap < nblk) return fail(MMDIT_EINVAL, "block_select: cap %d < number of blocks %d", cap, nblk);
+  if (top_k < 0) return fail(MMDIT_EINVAL, "block_select: top_k < 0");
+  if (!(top_p >= 0.f && top_p <= 1.f)) return fail(MMDIT_EINVAL, "block_select: top_p outside [0, 1]");
+  if (!(scale > 0.f) || !isfinite(scale)) return fail(MMDIT_EINVAL, "block_select: scale must be > 0");
+  const size_t half = align256((size_t)desc->batch * desc->heads * nblk * 128 * sizeof(float));
+  if (workspace == nullptr || ws_bytes < 2 * half)
+    return fail(MMDIT_EWORKSPACE, "block_select: workspace needs %zu bytes", 2 * half);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(MMDIT_EINVAL, "block_select: workspace must be 256-byte aligned");
+  float* qbar = static_cast<float*>(workspace);
+  float* kbar = reinterpret_cast<float*>(static_cast<char*>(workspace) + half);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = launch_pool((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, *desc, T, H, W,
+                              nblk, qbar, kbar, s);
+  if (e == cudaSuccess)
+    e = launch_select(qbar, kbar, desc->batch, desc->heads, nblk, top_k, top_p, scale, cap,
+                      block_idx, block_cnt, s);
+  return e == cudaSuccess ? MMDIT_OK : cuda_fail(e, "block_select launch");
+}
+
+size_t mmdit_sparse_attn_workspace_size(const mmdit_tensor_desc* desc, const mmdit_layout* layout,
+                                        int) {
+  int T, H, W, nblk;
+  if (check_desc(desc, "sparse_attn") || sparse_layout(layout, desc, T, H, W, nblk)) return 0;
+  const int ng = host_group_count(T, H, W, nblk);
+  const size_t lists = (size_t)desc->batch * desc->heads * ng;
+  return align256(sizeof(int4) * ng) + align256(lists * nblk * sizeof(uint32_t)) +
+         align256(lists * sizeof(int));
+}
+
+int mmdit_sparse_attn(const void* q, const void* k, const void* v, void* o,
+                      const mmdit_tensor_desc* desc, const mmdit_layout* layout,
+                      const int32_t* block_idx, const int32_t* block_cnt, int cap, float scale,
+                      void* workspace, size_t ws_bytes, mmdit_stream_t stream) {
+  int rc = check_desc(desc, "sparse_attn");
+  if (rc) return rc;
+  if (desc->dtype != MMDIT_BF16) return fail(MMDIT_EUNSUPPORTED, "sparse_attn: bf16 only");
+  if (!q || !k || !v || !o || !block_idx || !block_cnt)
+    return fail(MMDIT_EINVAL, "sparse_attn: every pointer must be non-NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(MMDIT_EINVAL, "sparse_attn: 16-byte alignment");
+  if (o == q || o == k || o == v) return fail(MMDIT_EINVAL, "sparse_attn: o aliases an input");
+  int T, H, W, nblk;
+  if ((rc = sparse_layout(layout, desc, T, H, W, nblk))) return rc;
+  if (cap < nblk) return fail(MMDIT_EINVAL, "sparse_attn: cap %d < number of blocks %d", cap, nblk);
+  if (!(scale > 0.f) || !isfinite(scale)) return fail(MMDIT_EINVAL, "sparse_attn: scale must be > 0");
+  const int ng = host_group_count(T, H, W, nblk);
+  const size_t lists = (size_t)desc->batch * desc->heads * ng;
+  const size_t g_bytes = align256(sizeof(int4) * ng);
+  const size_t l_bytes = align256(lists * nblk * sizeof(uint32_t));
+  const size_t c_bytes = align256(lists * sizeof(int));
+  if (workspace == nullptr || ws_bytes < g_bytes + l_bytes + c_bytes)
+    return fail(MMDIT_EWORKSPACE, "sparse_attn: workspace needs %zu bytes", g_bytes + l_bytes + c_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(MMDIT_EINVAL, "sparse_attn: workspace must be 256-byte aligned");
+  if ((rc = check_sm100())) return rc;
+  char* ws = static_cast<char*>(workspace);
+  int4* groups = reinterpret_cast<int4*>(ws);
+  uint32_t* ulist = reinterpret_cast<uint32_t*>(ws + g_bytes);
+  int* ucnt = reinterpret_cast<int*>(ws + g_bytes + l_bytes);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = launch_groups(T, H, W, nblk, groups, nullptr, s);
+  if (e == cudaSuccess)
+    e = launch_union(block_idx, block_cnt, cap, groups, ng, nullptr, desc->batch, desc->heads, nblk,
+                     ulist, ucnt, s);
+  if (e != cudaSuccess) return cuda_fail(e, "sparse_attn prep launch");
+  AttnParams p{};
+  AttnProblem& pr = p.prob[0];
+  if ((rc = make_map(&pr.tmQ, q, *desc, desc->n_tokens, "q")) ||
+      (rc = make_map(&pr.tmK, k, *desc, desc->n_tokens, "k")) ||
+      (rc = make_map(&pr.tmV, v, *desc, desc->n_tokens, "v")))
+    return rc;
+  pr.o = (__nv_bfloat16*)o;
+  pr.o_st = desc->stride_tok;
+  pr.o_sb = desc->stride_batch;
+  pr.Nq = pr.Nkv = desc->n_tokens;
+  pr.H = desc->heads;
+  pr.B = desc->batch;
+  pr.n_qtiles = ng;
+  pr.n_splits = 1;
+  pr.kv_per_split = 0;
+  pr.ctas = ng * pr.H * pr.B;
+  pr.mode = kModeSparse;
+  pr.groups = groups;
+  pr.ulist = ulist;
+  pr.ucnt = ucnt;
+  pr.ucap = nblk;
+  pr.vT = T;
+  pr.vH = H;
+  pr.vW = W;
+  p.n_prob = 1;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.err = device_error_flag();
+  if (p.err == nullptr) return fail(MMDIT_ECUDA, "device error flag unavailable");
+  e = launch_attn_tc(p, s);
+  return e == cudaSuccess ? MMDIT_OK : cuda_fail(e, "sparse attn launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,341 @@
+// Block-sparse mode, selection side (Prism guide, arXiv 2610.05416, Method
+// section 3): key blocks (and, in this library, query blocks too) are
+// mean-pooled into representatives; each query block i gets block
+// probabilities P_i = softmax_j(Qbar_i . Kbar_j * scale) and attends to
+// S_i = TopK(P_i, k) U TopP(P_i, p).
+//
+// Kernels:
+//   pool_kernel    one CTA per (block, batch): coalesced 128-bit reads of the
+//                  block's <= 64 tokens of Q and K, fp32 sums, mean over the
+//                  block's real tokens.  HBM-bound: Q and K are read once.
+//   select_kernel  one CTA per (8 query blocks, head, batch): fp32 block
+//                  scores into shared memory, then one warp per row: fp32
+//                  probabilities, fp64 normaliser and prefix masses, value
+//                  thresholds of the k-th block (count search) and of the
+//                  top-p crossing block (mass search) by bisection on the
+//                  fp32 bit patterns, and an ascending-id compaction with
+//                  warp ballots.  Ranking is P descending, ties by lower id.
+//   groups_kernel  partitions the query blocks into CTA groups of <= 256
+//                  tokens and <= 16 blocks (greedy, in block order).
+//   union_kernel   per (group, head, batch): merges the groups' selected
+//                  lists into one ascending list whose entries carry a
+//                  16-bit membership mask (which query blocks of the group
+//                  selected the key block).  The attention kernel walks it.
+#include <math.h>
+
+#include "internal.h"
+
+namespace mmdit {
+
+namespace {
+
+__global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ q,
+                                                   const __nv_bfloat16* __restrict__ k, int H,
+                                                   long long st, long long sb, int T, int Hg,
+                                                   int Wg, int nblk, float* __restrict__ qbar,
+                                                   float* __restrict__ kbar) {
+  const int blk = blockIdx.x, b = blockIdx.y;
+  int start, len;
+  block_extent(T, Hg, Wg, blk, start, len);
+  const int npairs = H * 64;  // bf16 pairs per token row (head_dim 128)
+  const float inv = 1.f / (float)len;
+  for (int pidx = threadIdx.x; pidx < npairs; pidx += blockDim.x) {
+    float2 aq = make_float2(0.f, 0.f), ak = make_float2(0.f, 0.f);
+    const long long base = (long long)b * sb + (long long)start * st + 2 * pidx;
+#pragma unroll 4
+    for (int i = 0; i < len; ++i) {
+      const float2 vq = __bfloat1622float2(
+          *reinterpret_cast<const __nv_bfloat162*>(q + base + (long long)i * st));
+      const float2 vk = __bfloat1622float2(
+          *reinterpret_cast<const __nv_bfloat162*>(k + base + (long long)i * st));
+      aq.x += vq.x;
+      aq.y += vq.y;
+      ak.x += vk.x;
+      ak.y += vk.y;
+    }
+    const int h = pidx >> 6, d = (pidx & 63) * 2;
+    const long long o = (((long long)b * H + h) * nblk + blk) * 128 + d;
+    *reinterpret_cast<float2*>(qbar + o) = make_float2(aq.x * inv, aq.y * inv);
+    *reinterpret_cast<float2*>(kbar + o) = make_float2(ak.x * inv, ak.y * inv);
+  }
+}
+
+constexpr int kSelRows = 8;
+constexpr int kSelChunk = 64;
+
+__device__ __forceinline__ int warp_sum_i(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// number of probabilities with bit pattern >= tau
+__device__ __forceinline__ int count_ge(const uint32_t* pb, int n, uint32_t tau, int lane) {
+  int c = 0;
+  for (int j = lane; j < n; j += 32) c += pb[j] >= tau;
+  return warp_sum_i(c);
+}
+// sum (fp64) of probabilities with bit pattern >= tau
+__device__ __forceinline__ double mass_ge(const uint32_t* pb, int n, uint32_t tau, int lane) {
+  double m = 0.0;
+  for (int j = lane; j < n; j += 32) {
+    const uint32_t v = pb[j];
+    if (v >= tau) m += (double)__uint_as_float(v);
+  }
+  return warp_sum_d(m);
+}
+
+__global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ qbar,
+                                                     const float* __restrict__ kbar, int H,
+                                                     int nblk, int top_k, float top_p, float scale,
+                                                     int cap, int32_t* __restrict__ idx,
+                                                     int32_t* __restrict__ cnt) {
+  extern __shared__ float sm[];
+  float* q_s = sm;                                  // [8][128]
+  float* k_s = q_s + kSelRows * 128;                // [64][129]
+  float* sc = k_s + kSelChunk * 129;                // [8][nblk]
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int r0 = blockIdx.x * kSelRows;
+  const long long hb = ((long long)b * H + h) * nblk;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  for (int i = tid; i < kSelRows * 128; i += 256) {
+    const int r = i >> 7;
+    q_s[i] = (r0 + r < nblk) ? qbar[(hb + r0 + r) * 128 + (i & 127)] : 0.f;
+  }
+  // ---- scores: sc[r][j] = qbar_r . kbar_j * scale (fp32)
+  for (int c0 = 0; c0 < nblk; c0 += kSelChunk) {
+    __syncthreads();
+    for (int i = tid; i < kSelChunk * 128; i += 256) {
+      const int kr = i >> 7, c = i & 127;
+      k_s[kr * 129 + c] = (c0 + kr < nblk) ? kbar[(hb + c0 + kr) * 128 + c] : 0.f;
+    }
+    __syncthreads();
+    const int kk = tid & 63, ra = tid >> 6, rb = ra + 4;
+    float da = 0.f, db = 0.f;
+#pragma unroll 16
+    for (int c = 0; c < 128; ++c) {
+      const float kv = k_s[kk * 129 + c];
+      da = fmaf(q_s[ra * 128 + c], kv, da);
+      db = fmaf(q_s[rb * 128 + c], kv, db);
+    }
+    if (c0 + kk < nblk) {
+      sc[ra * nblk + c0 + kk] = da * scale;
+      sc[rb * nblk + c0 + kk] = db * scale;
+    }
+  }
+  __syncthreads();
+
+  // ---- per row selection: one warp per query block
+  const int row = r0 + warp;
+  if (row >= nblk) return;
+  float* s = sc + warp * nblk;
+  uint32_t* pb = reinterpret_cast<uint32_t*>(s);
+  const int n = nblk;
+  float mx = -INFINITY;
+  for (int j = lane; j < n; j += 32) mx = fmaxf(mx, s[j]);
+  mx = warp_max_f(mx);
+  double z = 0.0;
+  for (int j = lane; j < n; j += 32) {
+    const float p = expf(s[j] - mx);  // unnormalised probability in (0, 1]
+    s[j] = p;
+    z += (double)p;
+  }
+  z = warp_sum_d(z);
+  __syncwarp();
+
+  const uint32_t kOne = 0x3F800000u;  // bit pattern of 1.0f, the largest value
+  // top-k threshold: largest tau with count(P >= tau) >= k'
+  const int kq = min(max(top_k, 0), n);
+  uint32_t tau_k = kOne + 1;  // nothing selected by top-k when k' == 0
+  if (kq > 0) {
+    uint32_t lo = 0, hi = kOne + 1;
+    while (hi - lo > 1) {
+      const uint32_t mid = lo + ((hi - lo) >> 1);
+      if (count_ge(pb, n, mid, lane) >= kq) lo = mid; else hi = mid;
+    }
+    tau_k = lo;
+  }
+  // top-p threshold: largest tau with mass(P >= tau) >= p * Z
+  const double target = (double)top_p * z;
+  uint32_t tau_p;
+  int take_p;  // how many blocks top-p selects
+  if (target <= 0.0) {
+    tau_p = kOne;
+  } else if (mass_ge(pb, n, 0u, lane) < target) {
+    tau_p = 0u;  // the sum never reaches p (p >= 1 with rounding): all blocks
+  } else {
+    uint32_t lo = 0, hi = kOne + 1;
+    while (hi - lo > 1) {
+      const uint32_t mid = lo + ((hi - lo) >> 1);
+      if (mass_ge(pb, n, mid, lane) >= target) lo = mid; else hi = mid;
+    }
+    tau_p = lo;
+  }
+  {
+    const int c_gt = count_ge(pb, n, tau_p + 1, lane);
+    const int c_eq = count_ge(pb, n, tau_p, lane) - c_gt;
+    const double m_gt = mass_ge(pb, n, tau_p + 1, lane);
+    const double tv = (double)__uint_as_float(tau_p);
+    int m = 1;
+    if (tau_p == 0u && target > 0.0 && mass_ge(pb, n, 0u, lane) < target) {
+      m = c_eq;  // everything
+    } else if (target > m_gt && tv > 0.0) {
+      m = (int)ceil((target - m_gt) / tv);
+    }
+    m = max(1, min(m, c_eq));
+    take_p = c_gt + m;
+  }
+  // final threshold and number of tied blocks to take (lowest ids first)
+  uint32_t tau;
+  int take_eq;
+  if (take_p >= kq) {
+    tau = tau_p;
+    take_eq = take_p - count_ge(pb, n, tau_p + 1, lane);
+  } else {
+    tau = tau_k;
+    take_eq = kq - count_ge(pb, n, tau_k + 1, lane);
+  }
+  // ---- ascending compaction
+  int32_t* out = idx + (hb + row) * (long long)cap;
+  int pos = 0, ties = 0;
+  for (int j0 = 0; j0 < n; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t v = j < n ? pb[j] : 0u;
+    const bool eq = j < n && v == tau;
+    const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+    const int tie_rank = ties + __popc(eqm & ((1u << lane) - 1u));
+    const bool sel = j < n && (v > tau || (eq && tie_rank < take_eq));
+    const unsigned sm_ = __ballot_sync(0xffffffffu, sel);
+    if (sel) out[pos + __popc(sm_ & ((1u << lane) - 1u))] = j;
+    pos += __popc(sm_);
+    ties += __popc(eqm);
+  }
+  if (lane == 0) cnt[hb + row] = pos;
+}
+
+// Greedy partition of the query blocks into groups of <= 256 tokens and <= 16
+// blocks; must agree with the host-side count (see mmdit_api.cu).
+__global__ void groups_kernel(int T, int H, int W, int nblk, int4* groups) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  int g = 0, first = 0, nb = 0, tokens = 0, start = 0;
+  for (int b = 0; b < nblk; ++b) {
+    int st, len;
+    block_extent(T, H, W, b, st, len);
+    if (nb == 16 || tokens + len > 256) {
+      groups[g++] = make_int4(first, nb, start, tokens);
+      first = b;
+      nb = 0;
+      tokens = 0;
+      start = st;
+    }
+    if (nb == 0) start = st;
+    ++nb;
+    tokens += len;
+  }
+  if (nb > 0) groups[g++] = make_int4(first, nb, start, tokens);
+}
+
+__global__ void __launch_bounds__(256) union_kernel(const int32_t* __restrict__ idx,
+                                                    const int32_t* __restrict__ cnt, int cap,
+                                                    const int4* __restrict__ groups, int H,
+                                                    int nblk, int n_groups,
+                                                    uint32_t* __restrict__ ulist,
+                                                    int* __restrict__ ucnt) {
+  extern __shared__ uint32_t mask[];  // [nblk]
+  __shared__ int warp_tot[8];
+  const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int4 gr = groups[g];
+  for (int j = tid; j < nblk; j += 256) mask[j] = 0u;
+  __syncthreads();
+  const long long hb = ((long long)b * H + h) * nblk;
+  for (int i = 0; i < gr.y; ++i) {
+    const long long r = hb + gr.x + i;
+    const int c = min(max(cnt[r], 0), nblk);
+    for (int e = tid; e < c; e += 256) {
+      const int j = idx[r * cap + e];
+      if ((unsigned)j < (unsigned)nblk) atomicOr(&mask[j], 1u << i);
+    }
+  }
+  __syncthreads();
+  const long long lid = ((long long)b * H + h) * n_groups + g;
+  uint32_t* out = ulist + lid * nblk;
+  int running = 0;
+  for (int j0 = 0; j0 < nblk; j0 += 256) {
+    const int j = j0 + tid;
+    const uint32_t m = j < nblk ? mask[j] : 0u;
+    const unsigned bal = __ballot_sync(0xffffffffu, m != 0u);
+    if (lane == 0) warp_tot[warp] = __popc(bal);
+    __syncthreads();
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      before += (w < warp) ? warp_tot[w] : 0;
+      total += warp_tot[w];
+    }
+    if (m != 0u) out[running + before + __popc(bal & ((1u << lane) - 1u))] = (uint32_t)j | (m << 16);
+    running += total;
+    __syncthreads();
+  }
+  if (tid == 0) ucnt[lid] = running;
+}
+
+}  // namespace
+
+size_t select_smem_bytes(int nblk) {
+  return sizeof(float) * ((size_t)kSelRows * 128 + (size_t)kSelChunk * 129 + (size_t)kSelRows * nblk);
+}
+
+cudaError_t launch_pool(const __nv_bfloat16* q, const __nv_bfloat16* k, const mmdit_tensor_desc& d,
+                        int T, int H, int W, int nblk, float* qbar, float* kbar, cudaStream_t s) {
+  if (nblk == 0) return cudaSuccess;
+  pool_kernel<<<dim3(nblk, d.batch), 256, 0, s>>>(q, k, d.heads, d.stride_tok, d.stride_batch, T,
+                                                  H, W, nblk, qbar, kbar);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select(const float* qbar, const float* kbar, int B, int H, int nblk, int top_k,
+                          float top_p, float scale, int cap, int32_t* idx, int32_t* cnt,
+                          cudaStream_t s) {
+  if (nblk == 0) return cudaSuccess;
+  const size_t smem = select_smem_bytes(nblk);
+  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((nblk + kSelRows - 1) / kSelRows, H, B);
+  select_kernel<<<grid, 256, smem, s>>>(qbar, kbar, H, nblk, top_k, top_p, scale, cap, idx, cnt);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_groups(int T, int H, int W, int nblk, int4* groups, int*, cudaStream_t s) {
+  groups_kernel<<<1, 32, 0, s>>>(T, H, W, nblk, groups);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_union(const int32_t* idx, const int32_t* cnt, int cap, const int4* groups,
+                         int n_groups, const int*, int B, int H, int nblk, uint32_t* ulist,
+                         int* ucnt, cudaStream_t s) {
+  if (n_groups == 0) return cudaSuccess;
+  const size_t smem = sizeof(uint32_t) * (size_t)nblk;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  union_kernel<<<dim3(n_groups, H, B), 256, smem, s>>>(idx, cnt, cap, groups, H, nblk, n_groups,
+                                                       ulist, ucnt);
+  return cudaGetLastError();
+}
+
+}  // namespace mmdit

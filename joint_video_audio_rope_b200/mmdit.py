@@ -1,0 +1,224 @@
+"""Thin ctypes binding of libmmdit.so (the C ABI in include/mmdit.h).
+
+Argument marshalling only: every step of the hot path runs in the library's
+sm_100a kernels.  Functions carry the C names without the ``mmdit_`` prefix.
+Tensors are torch tensors (PyTorch supplies device memory and streams) or raw
+integer device addresses.  A non-zero status raises ``MmditError`` with the
+library's thread-local message.  If the shared library is missing this module
+raises ImportError: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import re
+from typing import Iterable, Optional, Sequence
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmmdit.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "mmdit.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing; build it with "
+                      "`python -m joint_video_audio_rope_b200.build`")
+_lib = C.CDLL(LIB_PATH)
+
+OK, EINVAL, EUNSUPPORTED, EWORKSPACE, ECUDA, ETIMEOUT = range(6)
+BF16, F32 = 0, 1
+SEG_VIDEO, SEG_AUDIO, SEG_TEXT = 0, 1, 2
+ORDER_RASTER, ORDER_BLOCK444 = 0, 1
+MAX_SEGMENTS = 8
+
+
+class Segment(C.Structure):
+    _fields_ = [(n, C.c_int32) for n in
+                ("kind", "n_tokens", "T", "H", "W", "t0", "t_num", "t_den", "order")]
+
+
+class Layout(C.Structure):
+    _fields_ = [("n_seg", C.c_int32), ("seg", Segment * MAX_SEGMENTS)]
+
+
+class TensorDesc(C.Structure):
+    _fields_ = [("batch", C.c_int32), ("n_tokens", C.c_int32), ("heads", C.c_int32),
+                ("head_dim", C.c_int32), ("dtype", C.c_int32),
+                ("stride_tok", C.c_int64), ("stride_batch", C.c_int64)]
+
+
+class RopeParams(C.Structure):
+    _fields_ = [("theta", C.c_float), ("dim_t", C.c_int32), ("dim_h", C.c_int32),
+                ("dim_w", C.c_int32)]
+
+
+_P = C.c_void_p
+_D = C.POINTER(TensorDesc)
+_L = C.POINTER(Layout)
+_R = C.POINTER(RopeParams)
+_SIGS = {
+    "mmdit_rope_apply": (C.c_int, [_P, _P, _D, _L, _R, _P]),
+    "mmdit_joint_attn": (C.c_int, [_P, _P, _P, _P, _P, _D, _L, C.c_float, _R, _P, C.c_int64,
+                                   _P, C.c_size_t, _P]),
+    "mmdit_joint_attn_workspace_size": (C.c_size_t, [_D]),
+    "mmdit_av_cross_attn": (C.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _D, _D, C.c_float, _P,
+                                      C.c_size_t, _P]),
+    "mmdit_av_cross_attn_workspace_size": (C.c_size_t, [_D, _D]),
+    "mmdit_block_select": (C.c_int, [_P, _P, _D, _L, C.c_int, C.c_float, C.c_float, C.c_int,
+                                     _P, _P, _P, C.c_size_t, _P]),
+    "mmdit_block_select_workspace_size": (C.c_size_t, [_D, _L]),
+    "mmdit_sparse_attn": (C.c_int, [_P, _P, _P, _P, _D, _L, _P, _P, C.c_int, C.c_float, _P,
+                                    C.c_size_t, _P]),
+    "mmdit_sparse_attn_workspace_size": (C.c_size_t, [_D, _L, C.c_int]),
+    "mmdit_num_blocks": (C.c_int, [_L]),
+    "mmdit_device_status": (C.c_int, [_P]),
+    "mmdit_last_error": (C.c_char_p, []),
+    "mmdit_version": (C.c_char_p, []),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+class MmditError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"mmdit status {status}: {msg}")
+        self.status = status
+
+
+def header_functions() -> list:
+    """Names of the functions include/mmdit.h declares."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"\b(mmdit_[a-z0-9_]+)\s*\(", text)))
+
+
+def last_error() -> str:
+    return _lib.mmdit_last_error().decode()
+
+
+def version() -> str:
+    return _lib.mmdit_version().decode()
+
+
+def _check(rc: int) -> int:
+    if rc != OK:
+        raise MmditError(rc, last_error())
+    return rc
+
+
+# ---------------------------------------------------------------- marshalling
+
+def make_layout(segments: Sequence[dict]) -> Layout:
+    lay = Layout()
+    lay.n_seg = len(segments)
+    for i, s in enumerate(segments):
+        seg = lay.seg[i]
+        for k in ("kind", "n_tokens", "T", "H", "W", "t0", "t_num", "t_den", "order"):
+            setattr(seg, k, int(s.get(k, 1 if k in ("t_num", "t_den") else 0)))
+    return lay
+
+
+def make_desc(batch, n_tokens, heads, head_dim, dtype, stride_tok=None, stride_batch=None):
+    st = heads * head_dim if stride_tok is None else stride_tok
+    sb = st * n_tokens if stride_batch is None else stride_batch
+    return TensorDesc(batch, n_tokens, heads, head_dim, dtype, st, sb)
+
+
+def desc_of(t) -> TensorDesc:
+    """Descriptor of a torch tensor viewed as [B, N, heads, head_dim]."""
+    import torch
+    if t.dim() != 4 or t.stride(3) != 1 or t.stride(2) != t.shape[3]:
+        raise ValueError("expected [B, N, heads, head_dim] with packed heads and channels")
+    dt = {torch.bfloat16: BF16, torch.float32: F32}[t.dtype]
+    return TensorDesc(t.shape[0], t.shape[1], t.shape[2], t.shape[3], dt, t.stride(1), t.stride(0))
+
+
+def rope_params(theta: float, dim_t: int, dim_h: int, dim_w: int) -> RopeParams:
+    return RopeParams(theta, dim_t, dim_h, dim_w)
+
+
+def _ptr(x) -> Optional[int]:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _ref(x):
+    return None if x is None else C.byref(x)
+
+
+# ---------------------------------------------------------------- entry points
+
+def rope_apply(q, k, desc: TensorDesc, layout: Layout, rope: RopeParams, stream=None) -> None:
+    _check(_lib.mmdit_rope_apply(_ptr(q), _ptr(k), C.byref(desc), C.byref(layout), C.byref(rope),
+                                 _stream(stream)))
+
+
+def joint_attn(q, k, v, o, desc: TensorDesc, layout: Layout, scale: float, lse=None,
+               rope_q: Optional[RopeParams] = None, cond_mask=None, mask_elems: int = 0,
+               workspace=None, ws_bytes: int = 0, stream=None) -> None:
+    _check(_lib.mmdit_joint_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), C.byref(desc),
+                                 C.byref(layout), scale, _ref(rope_q), _ptr(cond_mask),
+                                 mask_elems, _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def joint_attn_workspace_size(desc: TensorDesc) -> int:
+    return _lib.mmdit_joint_attn_workspace_size(C.byref(desc))
+
+
+def av_cross_attn(qv, kv, vv, qa, ka, va, o_video, o_audio, video: TensorDesc,
+                  audio: TensorDesc, scale: float, workspace=None, ws_bytes: int = 0,
+                  stream=None) -> None:
+    _check(_lib.mmdit_av_cross_attn(_ptr(qv), _ptr(kv), _ptr(vv), _ptr(qa), _ptr(ka), _ptr(va),
+                                    _ptr(o_video), _ptr(o_audio), C.byref(video), C.byref(audio),
+                                    scale, _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def av_cross_attn_workspace_size(video: TensorDesc, audio: TensorDesc) -> int:
+    return _lib.mmdit_av_cross_attn_workspace_size(C.byref(video), C.byref(audio))
+
+
+def block_select(q, k, desc: TensorDesc, layout: Layout, top_k: int, top_p: float, scale: float,
+                 cap: int, block_idx, block_cnt, workspace=None, ws_bytes: int = 0,
+                 stream=None) -> None:
+    _check(_lib.mmdit_block_select(_ptr(q), _ptr(k), C.byref(desc), C.byref(layout), top_k, top_p,
+                                   scale, cap, _ptr(block_idx), _ptr(block_cnt), _ptr(workspace),
+                                   ws_bytes, _stream(stream)))
+
+
+def block_select_workspace_size(desc: TensorDesc, layout: Layout) -> int:
+    return _lib.mmdit_block_select_workspace_size(C.byref(desc), C.byref(layout))
+
+
+def sparse_attn(q, k, v, o, desc: TensorDesc, layout: Layout, block_idx, block_cnt, cap: int,
+                scale: float, workspace=None, ws_bytes: int = 0, stream=None) -> None:
+    _check(_lib.mmdit_sparse_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), C.byref(desc),
+                                  C.byref(layout), _ptr(block_idx), _ptr(block_cnt), cap, scale,
+                                  _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def sparse_attn_workspace_size(desc: TensorDesc, layout: Layout, cap: int) -> int:
+    return _lib.mmdit_sparse_attn_workspace_size(C.byref(desc), C.byref(layout), cap)
+
+
+def num_blocks(layout: Layout) -> int:
+    return _lib.mmdit_num_blocks(C.byref(layout))
+
+
+def device_status(stream=None) -> int:
+    return _lib.mmdit_device_status(_stream(stream))
+
+
+def raw(name: str):
+    """The raw ctypes function of C symbol `name` (for boundary tests)."""
+    return getattr(_lib, name)

@@ -1,0 +1,156 @@
+"""Boundary tests that need no GPU: the library loads, exports every function
+include/mmdit.h declares, and rejects bad arguments with the documented
+status before launching anything (no CUDA call is reached)."""
+import ctypes as C
+import subprocess
+
+import pytest
+
+from joint_video_audio_rope_b200 import build as B
+
+B.build()
+from joint_video_audio_rope_b200 import mmdit as M  # noqa: E402
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def test_exports_every_declared_symbol():
+    names = M.header_functions()
+    assert "mmdit_joint_attn" in names and len(names) >= 12
+    out = subprocess.run(["nm", "-D", "--defined-only", M.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if l.strip()}
+    for n in names:
+        assert n in exported, n
+        assert M.raw(n) is not None
+    # nothing but the C ABI is exported
+    extra = {e for e in exported if e.startswith("mmdit")} - set(names)
+    assert not extra, extra
+
+
+def test_version_and_error_string():
+    assert "sm_100a" in M.version()
+    assert isinstance(M.last_error(), str)
+
+
+def _desc(**kw):
+    d = dict(batch=1, n_tokens=112, heads=2, head_dim=128, dtype=M.BF16)
+    d.update(kw)
+    return M.make_desc(**d)
+
+
+def _layout(n=112):
+    return M.make_layout([dict(kind=M.SEG_VIDEO, n_tokens=n, T=n // 16, H=4, W=4)])
+
+
+def _rope():
+    return M.rope_params(10000.0, 44, 42, 42)
+
+
+def _rc(fn, *args):
+    # stream 0 explicitly: no torch CUDA context is needed on a CPU machine
+    import inspect
+    nparams = len(inspect.signature(fn).parameters)
+    kw = {} if len(args) >= nparams else {"stream": 0}
+    with pytest.raises(M.MmditError) as e:
+        fn(*args, **kw)
+    return e.value.status
+
+
+def test_rope_rejects_bad_arguments():
+    assert _rc(M.rope_apply, None, None, _desc(), _layout(), _rope()) == M.EINVAL
+    assert _rc(M.rope_apply, FAKE, FAKE, _desc(dtype=7), _layout(), _rope()) == M.EUNSUPPORTED
+    assert _rc(M.rope_apply, FAKE, FAKE, _desc(head_dim=64), _layout(), _rope()) == M.EUNSUPPORTED
+    assert _rc(M.rope_apply, FAKE, FAKE, _desc(), _layout(96), _rope()) == M.EINVAL
+    assert _rc(M.rope_apply, FAKE, FAKE, _desc(), _layout(), M.rope_params(1e4, 44, 42, 40), 0) == M.EINVAL
+    assert _rc(M.rope_apply, FAKE, FAKE, _desc(), _layout(), M.rope_params(1e4, 43, 43, 42), 0) == M.EINVAL
+    assert _rc(M.rope_apply, FAKE + 8, FAKE, _desc(), _layout(), _rope()) == M.EINVAL
+    assert "NULL" in M.last_error() or "align" in M.last_error()
+
+
+def test_layout_validation():
+    bad_kind = M.make_layout([dict(kind=9, n_tokens=112)])
+    assert _rc(M.rope_apply, FAKE, None, _desc(), bad_kind, _rope()) == M.EINVAL
+    bad_grid = M.make_layout([dict(kind=M.SEG_VIDEO, n_tokens=112, T=7, H=4, W=5)])
+    assert _rc(M.rope_apply, FAKE, None, _desc(), bad_grid, _rope()) == M.EINVAL
+    bad_audio = M.make_layout([dict(kind=M.SEG_AUDIO, n_tokens=112, t_num=21, t_den=0)])
+    assert _rc(M.rope_apply, FAKE, None, _desc(), bad_audio, _rope()) == M.EINVAL
+    lay = M.Layout()
+    lay.n_seg = 9
+    assert _rc(M.rope_apply, FAKE, None, _desc(), lay, _rope()) == M.EINVAL
+    assert "n_seg" in M.last_error()
+
+
+def test_strides_validation():
+    d = _desc(stride_tok=100)  # < heads * head_dim
+    assert _rc(M.rope_apply, FAKE, None, d, _layout(), _rope()) == M.EINVAL
+    d = _desc(stride_tok=260)  # 520 bytes: not a multiple of 16
+    assert _rc(M.rope_apply, FAKE, None, d, _layout(), _rope()) == M.EINVAL
+    d = _desc(batch=2, stride_batch=256)  # batch items overlap
+    assert _rc(M.rope_apply, FAKE, None, d, _layout(), _rope()) == M.EINVAL
+
+
+def test_joint_attn_validation():
+    d = _desc()
+    L = _layout()
+    assert _rc(M.joint_attn, FAKE, FAKE, FAKE, None, d, L, 0.1) == M.EINVAL
+    assert _rc(M.joint_attn, FAKE, FAKE, FAKE, FAKE, d, L, 0.1) == M.EINVAL  # o aliases q
+    assert _rc(M.joint_attn, FAKE, FAKE, FAKE, FAKE + 4096, d, L, -1.0) == M.EINVAL
+    # the channel-concat mask is shape-checked: B * frames * H * W = 1 * 7 * 4 * 4
+    assert _rc(M.joint_attn, FAKE, FAKE, FAKE, FAKE + 4096, d, L, 0.1, None, None,
+               FAKE, 111) == M.EINVAL
+    assert "mask" in M.last_error()
+    f32 = _desc(dtype=M.F32)
+    assert _rc(M.joint_attn, FAKE, FAKE, FAKE, FAKE + 4096, f32, L, 0.1, None, _rope(),
+               None, 0) == M.EUNSUPPORTED
+    assert M.joint_attn_workspace_size(d) == 0
+
+
+def test_cross_attn_validation_and_workspace():
+    v = _desc(n_tokens=1000, heads=24)
+    a = _desc(n_tokens=218, heads=24)
+    ws = M.av_cross_attn_workspace_size(v, a)
+    assert ws > 0 and ws % 256 == 0
+    args = [FAKE + 4096 * i for i in range(8)]
+    assert _rc(M.av_cross_attn, *args, v, _desc(n_tokens=218, heads=12), 0.1) == M.EINVAL
+    assert _rc(M.av_cross_attn, *args, v, a, 0.1, None, 0) == M.EWORKSPACE
+    assert _rc(M.av_cross_attn, *args, v, a, 0.1, FAKE, ws - 1) == M.EWORKSPACE
+    assert _rc(M.av_cross_attn, *args, v, _desc(n_tokens=0, heads=24), 0.1, FAKE, ws) == M.EINVAL
+
+
+def _sparse_layout(T=21, H=68, W=120):
+    return M.make_layout([dict(kind=M.SEG_VIDEO, n_tokens=T * H * W, T=T, H=H, W=W,
+                               order=M.ORDER_BLOCK444)])
+
+
+def test_block_counts_and_select_validation():
+    L = _sparse_layout()
+    assert M.num_blocks(L) == 6 * 17 * 30 == 3060
+    assert M.num_blocks(_layout()) == 0  # raster: not a block-sparse layout
+    d = _desc(n_tokens=171360, heads=24)
+    ws = M.block_select_workspace_size(d, L)
+    assert ws == 2 * ((24 * 3060 * 128 * 4 + 255) // 256 * 256)
+    assert _rc(M.block_select, FAKE, FAKE, d, L, 32, 0.9, 0.088, 3059, FAKE, FAKE, FAKE, ws) == M.EINVAL
+    assert "cap" in M.last_error()
+    assert _rc(M.block_select, FAKE, FAKE, d, L, 32, 1.5, 0.088, 3060, FAKE, FAKE, FAKE, ws) == M.EINVAL
+    assert _rc(M.block_select, FAKE, FAKE, d, L, -1, 0.9, 0.088, 3060, FAKE, FAKE, FAKE, ws) == M.EINVAL
+    assert _rc(M.block_select, FAKE, FAKE, d, L, 32, 0.9, 0.088, 3060, FAKE, FAKE, FAKE, ws - 256) == M.EWORKSPACE
+    assert _rc(M.block_select, FAKE, FAKE, d, _layout(171360 // 16 * 16), 32, 0.9, 0.088, 3060,
+               FAKE, FAKE, FAKE, ws) == M.EINVAL
+    huge = _sparse_layout(T=40, H=80, W=80)  # 10*20*20 = 4000 blocks: fine
+    assert M.num_blocks(huge) == 4000
+    too_many = _sparse_layout(T=40, H=128, W=128)  # 16384 blocks
+    dd = _desc(n_tokens=40 * 128 * 128, heads=2)
+    assert _rc(M.block_select, FAKE, FAKE, dd, too_many, 32, 0.9, 0.088, 16384, FAKE, FAKE, FAKE,
+               1 << 30) == M.EUNSUPPORTED
+
+
+def test_sparse_attn_validation():
+    L = _sparse_layout()
+    d = _desc(n_tokens=171360, heads=24)
+    ws = M.sparse_attn_workspace_size(d, L, 3060)
+    assert ws > 0
+    args = [FAKE, FAKE + 4096, FAKE + 8192, FAKE + 12288]
+    assert _rc(M.sparse_attn, *args, d, L, FAKE, FAKE, 3000, 0.088, FAKE, ws) == M.EINVAL
+    assert _rc(M.sparse_attn, *args, d, L, FAKE, FAKE, 3060, 0.088, FAKE, ws - 1) == M.EWORKSPACE
+    assert _rc(M.sparse_attn, *args, d, L, FAKE, FAKE, 3060, 0.088, FAKE + 8, ws) == M.EINVAL

@@ -1,0 +1,391 @@
+"""GPU parity: the sm_100a kernels, called through the C ABI, against the fp64
+oracle on the same seeded inputs.  Sizes span several tiles with ragged tails
+and stay small enough for the oracle to finish in seconds.  Tolerances:
+bf16 max-abs 2e-2 and relative-L2 5e-3; fp32 max-abs 1e-5."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle as O
+from joint_video_audio_rope_b200 import workloads as WL
+
+from _util import (assert_close, errors, oracle_layout, rope_bands, selection_matches, to_device,
+                   to_host_f64)
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def M():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from joint_video_audio_rope_b200 import build
+    build.build()
+    from joint_video_audio_rope_b200 import mmdit
+    return mmdit
+
+
+def _make(w: WL.Workload):
+    x = WL.generate(w)
+    host = {n: WL.as_f64(x[n], w.dtype) for n in ("q", "k", "v")}
+    dev = {n: to_device(x[n], w.dtype) for n in ("q", "k", "v")}
+    return x, host, dev
+
+
+def _rope_oracle(host, w):
+    pos = O.positions(oracle_layout(w.segments))
+    return (np.stack([O.rope(host["q"][b], pos, w.theta) for b in range(w.batch)]),
+            np.stack([O.rope(host["k"][b], pos, w.theta) for b in range(w.batch)]))
+
+
+def _rope_dev(M, dev, w, q=True, k=True):
+    d = M.desc_of(dev["q"])
+    M.rope_apply(dev["q"] if q else None, dev["k"] if k else None, d, M.make_layout(w.segments),
+                 M.rope_params(w.theta, *rope_bands(w.head_dim)))
+
+
+def _custom(name, segs, heads=2, batch=1, dtype="bf16", seed=11, qk=None, v=None, **kw):
+    base = WL.WORKLOADS[name]
+    return WL.Workload(f"{name}_custom", segs, batch, heads, 128 if dtype == "bf16" else base.head_dim,
+                       dtype, seed, base.qk_std if qk is None else qk,
+                       base.v_std if v is None else v, base.planted_regions, base.planted_amp,
+                       False, base.sparse, kw.get("top_k", base.top_k), kw.get("top_p", base.top_p))
+
+
+# ------------------------------------------------------------------- RoPE
+
+def test_rope_f32_tiny(M):
+    w = WL.WORKLOADS["tiny_f32"]
+    _, host, dev = _make(w)
+    rq, rk = _rope_oracle(host, w)
+    _rope_dev(M, dev, w)
+    assert_close(to_host_f64(dev["q"]), rq, "f32", "rope q")
+    assert_close(to_host_f64(dev["k"]), rk, "f32", "rope k")
+
+
+@pytest.mark.parametrize("which", ["cond_b2", "block444"])
+def test_rope_bf16(M, which):
+    if which == "cond_b2":
+        w = WL.reduced("720p_cond_b2", 5, 6, 10, n_audio=218, n_text=40, heads=3)
+    else:
+        w = WL.reduced("1080p_sparse", 9, 8, 12, n_audio=30, heads=3)
+    _, host, dev = _make(w)
+    rq, rk = _rope_oracle(host, w)
+    _rope_dev(M, dev, w, q=True, k=False)
+    assert_close(to_host_f64(dev["q"]), rq, "bf16", "rope q")
+    assert np.array_equal(to_host_f64(dev["k"]), host["k"]), "k must be untouched"
+    _rope_dev(M, dev, w, q=False, k=True)
+    assert_close(to_host_f64(dev["k"]), rk, "bf16", "rope k")
+
+
+def test_rope_bf16_odd_strides(M):
+    # tokens padded to 3 heads + 1 spare head: stride_tok = 512 elements
+    w = WL.reduced("480p", 3, 4, 6, n_audio=20, n_text=8, heads=3)
+    _, host, dev = _make(w)
+    pad = torch.zeros((w.batch, w.n_tokens, 4, 128), dtype=torch.bfloat16, device="cuda")
+    pad[:, :, :3] = dev["q"]
+    view = pad[:, :, :3]
+    M.rope_apply(view, None, M.desc_of(view), M.make_layout(w.segments),
+                 M.rope_params(w.theta, 44, 42, 42))
+    rq, _ = _rope_oracle(host, w)
+    assert_close(to_host_f64(view), rq, "bf16", "rope strided")
+    assert torch.count_nonzero(pad[:, :, 3]) == 0
+
+
+# ------------------------------------------------------------ joint attention
+
+def _joint_oracle(host, w):
+    scale = 1.0 / math.sqrt(w.head_dim)
+    return O.joint_attn(host["q"], host["k"], host["v"], scale)
+
+
+def test_joint_f32_tiny(M):
+    w = WL.WORKLOADS["tiny_f32"]
+    _, host, dev = _make(w)
+    rq, rk = _rope_oracle(host, w)
+    _rope_dev(M, dev, w)
+    o = torch.empty_like(dev["q"])
+    lse = torch.empty((w.batch, w.heads, w.n_tokens), dtype=torch.float32, device="cuda")
+    M.joint_attn(dev["q"], dev["k"], dev["v"], o, M.desc_of(dev["q"]), M.make_layout(w.segments),
+                 1 / math.sqrt(w.head_dim), lse=lse)
+    ro, rl = O.joint_attn(rq, rk, host["v"], 1 / math.sqrt(w.head_dim))
+    assert_close(to_host_f64(o), ro, "f32", "joint f32")
+    assert_close(lse.cpu().numpy().transpose(0, 2, 1), rl, "f32", "lse f32")
+
+
+JOINT_CASES = {
+    # name: (workload, q/k std override)
+    "ragged_373": (lambda: _custom("480p", [WL.video(5, 6, 10), WL.audio(40), WL.text(33)]), None),
+    "cond_b2_1030": (lambda: _custom("720p_cond_b2", [WL.video(2, 6, 10, t0=-2), WL.video(12, 6, 10),
+                                                      WL.audio(218), WL.text(12)], batch=2), None),
+    "peaky_700": (lambda: _custom("480p", [WL.video(7, 8, 12), WL.audio(18), WL.text(10)]), 1.0),
+    "huge_logits_300": (lambda: _custom("480p", [WL.video(3, 10, 10)]), 4.0),
+    "one_token": (lambda: _custom("480p", [WL.text(1)]), None),
+    "exact_512": (lambda: _custom("480p", [WL.video(8, 8, 8)]), None),
+}
+
+
+@pytest.mark.parametrize("case", list(JOINT_CASES))
+def test_joint_bf16(M, case):
+    make, qk = JOINT_CASES[case]
+    w = make()
+    if qk is not None:
+        w.qk_std = qk
+    _, host, dev = _make(w)
+    o = torch.full_like(dev["q"], float("nan"))
+    lse = torch.empty((w.batch, w.heads, w.n_tokens), dtype=torch.float32, device="cuda")
+    scale = 1 / math.sqrt(128)
+    M.joint_attn(dev["q"], dev["k"], dev["v"], o, M.desc_of(dev["q"]), M.make_layout(w.segments),
+                 scale, lse=lse)
+    torch.cuda.synchronize()
+    assert M.device_status() == 0
+    ro, rl = O.joint_attn(host["q"], host["k"], host["v"], scale)
+    assert_close(to_host_f64(o), ro, "bf16", f"joint {case}")
+    got_lse = lse.cpu().numpy().transpose(0, 2, 1)
+    assert np.max(np.abs(got_lse - rl)) < 1e-2, "lse"
+
+
+def test_joint_bf16_fused_rope(M):
+    w = _custom("720p_cond_b2", [WL.video(1, 6, 10, t0=-1), WL.video(6, 6, 10), WL.audio(50),
+                                 WL.text(20)])
+    _, host, dev = _make(w)
+    rq, rk = _rope_oracle(host, w)
+    _rope_dev(M, dev, w, q=False, k=True)  # K rotated once, Q rotated on load
+    o = torch.empty_like(dev["q"])
+    M.joint_attn(dev["q"], dev["k"], dev["v"], o, M.desc_of(dev["q"]), M.make_layout(w.segments),
+                 1 / math.sqrt(128), rope_q=M.rope_params(w.theta, 44, 42, 42))
+    ro, _ = O.joint_attn(rq, rk, host["v"], 1 / math.sqrt(128))
+    assert_close(to_host_f64(o), ro, "bf16", "joint fused rope")
+    # the caller's Q is not modified by the fused rotation
+    assert np.array_equal(to_host_f64(dev["q"]), host["q"])
+
+
+def test_joint_mask_is_not_applied(M):
+    w = _custom("720p_cond_b2", [WL.video(2, 4, 8, t0=-2), WL.video(5, 4, 8), WL.audio(20),
+                                 WL.text(8)], batch=2)
+    w.mask = True
+    x, host, dev = _make(w)
+    mask = torch.from_numpy(x["mask"]).cuda()
+    outs = []
+    for m in (None, mask, 1 - mask):
+        o = torch.empty_like(dev["q"])
+        M.joint_attn(dev["q"], dev["k"], dev["v"], o, M.desc_of(dev["q"]),
+                     M.make_layout(w.segments), 1 / math.sqrt(128), cond_mask=m,
+                     mask_elems=0 if m is None else m.numel())
+        outs.append(o)
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+
+
+def test_joint_empty_sequence_is_noop(M):
+    d = M.make_desc(1, 0, 2, 128, M.BF16)
+    lay = M.make_layout([dict(kind=M.SEG_TEXT, n_tokens=0)])
+    q = torch.zeros(8, dtype=torch.bfloat16, device="cuda")
+    o = torch.zeros(8, dtype=torch.bfloat16, device="cuda")
+    M.joint_attn(q, q, q, o, d, lay, 0.1)
+    torch.cuda.synchronize()
+
+
+# ------------------------------------------------------------ cross attention
+
+def _cross(M, w, dev):
+    v0, v1 = w.video_range()
+    a0, a1 = w.audio_range()
+    qv, kv, vv = (dev[n][:, v0:v1] for n in ("q", "k", "v"))
+    qa, ka, va = (dev[n][:, a0:a1] for n in ("q", "k", "v"))
+    dv, da = M.desc_of(qv), M.desc_of(qa)
+    # outputs share the inputs' strides: slices of one [B, N, H, d] buffer
+    o_full = torch.full_like(dev["q"], float("nan"))
+    ov, oa = o_full[:, v0:v1], o_full[:, a0:a1]
+    ws_n = M.av_cross_attn_workspace_size(dv, da)
+    ws = torch.empty(max(ws_n, 256), dtype=torch.uint8, device="cuda")
+    M.av_cross_attn(qv, kv, vv, qa, ka, va, ov, oa, dv, da, 1 / math.sqrt(w.head_dim), ws, ws_n)
+    torch.cuda.synchronize()
+    return ov, oa
+
+
+def _cross_oracle(host, w):
+    v0, v1 = w.video_range()
+    a0, a1 = w.audio_range()
+    s = 1 / math.sqrt(w.head_dim)
+    return O.av_cross_attn(host["q"][:, v0:v1], host["k"][:, v0:v1], host["v"][:, v0:v1],
+                           host["q"][:, a0:a1], host["k"][:, a0:a1], host["v"][:, a0:a1], s)
+
+
+def test_cross_f32_tiny(M):
+    w = WL.WORKLOADS["tiny_f32"]
+    _, host, dev = _make(w)
+    ov, oa = _cross(M, w, dev)
+    rv, ra = _cross_oracle(host, w)
+    assert_close(to_host_f64(ov), rv, "f32", "cross v<-a")
+    assert_close(to_host_f64(oa), ra, "f32", "cross a<-v")
+
+
+CROSS_CASES = {
+    "small_b2": lambda: _custom("720p_cond_b2", [WL.video(1, 6, 10, t0=-1), WL.video(5, 6, 10),
+                                                 WL.audio(218), WL.text(16)], batch=2),
+    "split_kv": lambda: _custom("480p", [WL.video(21, 14, 16), WL.audio(218), WL.text(8)]),
+    "short_audio": lambda: _custom("480p", [WL.video(4, 5, 7), WL.audio(3)]),
+}
+
+
+@pytest.mark.parametrize("case", list(CROSS_CASES))
+def test_cross_bf16(M, case):
+    w = CROSS_CASES[case]()
+    _, host, dev = _make(w)
+    ov, oa = _cross(M, w, dev)
+    assert M.device_status() == 0
+    rv, ra = _cross_oracle(host, w)
+    assert_close(to_host_f64(ov), rv, "bf16", "cross v<-a")
+    assert_close(to_host_f64(oa), ra, "bf16", "cross a<-v")
+
+
+# ------------------------------------------------------------ block-sparse mode
+
+SPARSE_CASES = {
+    "t9_16x20": dict(T=9, H=16, W=20, top_k=4, top_p=0.9),
+    "t21_24x32": dict(T=21, H=24, W=32, top_k=32, top_p=0.9),
+    "odd_edges": dict(T=6, H=10, W=14, top_k=3, top_p=0.5),
+}
+
+
+def _sparse_workload(c, heads=2, seed=21):
+    base = WL.WORKLOADS["1080p_sparse"]
+    return WL.Workload("sparse_case", [WL.video(c["T"], c["H"], c["W"], order=WL.ORDER_BLOCK444)],
+                       1, heads, 128, "bf16", seed, base.qk_std, base.v_std, base.planted_regions,
+                       base.planted_amp, False, True, c["top_k"], c["top_p"])
+
+
+def _select_dev(M, w, dev):
+    lay = M.make_layout(w.segments)
+    d = M.desc_of(dev["q"])
+    nb = M.num_blocks(lay)
+    idx = torch.full((w.batch, w.heads, nb, nb), -1, dtype=torch.int32, device="cuda")
+    cnt = torch.full((w.batch, w.heads, nb), -1, dtype=torch.int32, device="cuda")
+    ws_n = M.block_select_workspace_size(d, lay)
+    ws = torch.empty(ws_n, dtype=torch.uint8, device="cuda")
+    M.block_select(dev["q"], dev["k"], d, lay, w.top_k, w.top_p, 1 / math.sqrt(128), nb, idx, cnt,
+                   ws, ws_n)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), cnt.cpu().numpy()
+
+
+def _oracle_select(host, w):
+    T, H, W = w.segments[0]["T"], w.segments[0]["H"], w.segments[0]["W"]
+    blocks = O.video_blocks(T, H, W)
+    qb, kb = O.pool(host["q"], blocks), O.pool(host["k"], blocks)
+    return blocks, qb, kb
+
+
+@pytest.mark.parametrize("case", list(SPARSE_CASES))
+def test_block_select(M, case):
+    w = _sparse_workload(SPARSE_CASES[case])
+    _, host, dev = _make(w)
+    idx, cnt = _select_dev(M, w, dev)
+    blocks, qb, kb = _oracle_select(host, w)
+    scale = 1 / math.sqrt(128)
+    p32 = float(np.float32(w.top_p))
+    bad = 0
+    for b in range(w.batch):
+        for h in range(w.heads):
+            for i in range(len(blocks)):
+                ref = O.select_row(qb[b, h, i], kb[b, h], w.top_k, p32, scale)
+                got = idx[b, h, i, :cnt[b, h, i]]
+                assert np.all(np.diff(got) > 0), "ascending, unique"
+                P = O.block_probs(qb[b, h, i], kb[b, h], scale)
+                if not selection_matches(got, ref, P, w.top_k, p32):
+                    bad += 1
+    assert bad == 0, f"{bad} rows differ beyond fp32 ties"
+
+
+def _upload_lists(sel, nb, w):
+    idx = np.full((w.batch, w.heads, nb, nb), -1, np.int32)
+    cnt = np.zeros((w.batch, w.heads, nb), np.int32)
+    for b in range(w.batch):
+        for h in range(w.heads):
+            for i in range(nb):
+                s = np.asarray(sel[b][h][i], np.int32)
+                idx[b, h, i, :len(s)] = s
+                cnt[b, h, i] = len(s)
+    return torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda()
+
+
+def _sparse_dev(M, w, dev, idx_t, cnt_t, nb):
+    lay = M.make_layout(w.segments)
+    d = M.desc_of(dev["q"])
+    o = torch.full_like(dev["q"], float("nan"))
+    ws_n = M.sparse_attn_workspace_size(d, lay, nb)
+    ws = torch.empty(ws_n, dtype=torch.uint8, device="cuda")
+    M.sparse_attn(dev["q"], dev["k"], dev["v"], o, d, lay, idx_t, cnt_t, nb, 1 / math.sqrt(128),
+                  ws, ws_n)
+    torch.cuda.synchronize()
+    assert M.device_status() == 0
+    return o
+
+
+@pytest.mark.parametrize("case", list(SPARSE_CASES))
+def test_sparse_attn_given_lists(M, case):
+    """GPU sparse attention on the oracle's selection vs the oracle."""
+    w = _sparse_workload(SPARSE_CASES[case])
+    _, host, dev = _make(w)
+    blocks, qb, kb = _oracle_select(host, w)
+    sel = O.block_select(qb, kb, w.top_k, float(np.float32(w.top_p)), 1 / math.sqrt(128))
+    idx_t, cnt_t = _upload_lists(sel, len(blocks), w)
+    o = _sparse_dev(M, w, dev, idx_t, cnt_t, len(blocks))
+    ref = O.sparse_attn(host["q"], host["k"], host["v"], blocks, sel, 1 / math.sqrt(128))
+    assert_close(to_host_f64(o), ref, "bf16", f"sparse {case}")
+
+
+def test_sparse_all_blocks_equals_dense(M):
+    w = _sparse_workload(SPARSE_CASES["odd_edges"])
+    _, host, dev = _make(w)
+    nb = len(O.video_blocks(6, 10, 14))
+    sel = [[[np.arange(nb) for _ in range(nb)] for _ in range(w.heads)]]
+    idx_t, cnt_t = _upload_lists(sel, nb, w)
+    o = _sparse_dev(M, w, dev, idx_t, cnt_t, nb)
+    ref, _ = O.joint_attn(host["q"], host["k"], host["v"], 1 / math.sqrt(128))
+    assert_close(to_host_f64(o), ref, "bf16", "sparse all = dense")
+
+
+def test_sparse_empty_and_single_lists(M):
+    w = _sparse_workload(SPARSE_CASES["t9_16x20"])
+    _, host, dev = _make(w)
+    blocks = O.video_blocks(9, 16, 20)
+    nb = len(blocks)
+    sel = [[[np.array([], np.int64) if i % 3 == 0 else np.array([(i * 7 + h) % nb])
+             for i in range(nb)] for h in range(w.heads)]]
+    idx_t, cnt_t = _upload_lists(sel, nb, w)
+    o = _sparse_dev(M, w, dev, idx_t, cnt_t, nb)
+    got = to_host_f64(o)
+    for h in range(w.heads):
+        for i, (s, n) in enumerate(blocks):
+            if i % 3 == 0:
+                assert np.all(got[0, s:s + n, h] == 0), "empty list -> zero rows"
+            else:
+                ref, _ = O.sparse_attn_rows(host["q"], host["k"], host["v"], blocks, sel[0][h][i],
+                                            1 / math.sqrt(128), 0, h, i)
+                assert_close(got[0, s:s + n, h], ref, "bf16", "single block")
+
+
+def test_select_then_sparse_end_to_end(M):
+    w = _sparse_workload(SPARSE_CASES["t21_24x32"])
+    _, host, dev = _make(w)
+    idx, cnt = _select_dev(M, w, dev)
+    nb = idx.shape[2]
+    o = _sparse_dev(M, w, dev, torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda(), nb)
+    blocks, qb, kb = _oracle_select(host, w)
+    got = to_host_f64(o)
+    scale = 1 / math.sqrt(128)
+    checked = 0
+    for h in range(w.heads):
+        for i, (s, n) in enumerate(blocks):
+            ref_sel = O.select_row(qb[0, h, i], kb[0, h], w.top_k, float(np.float32(w.top_p)), scale)
+            gsel = idx[0, h, i, :cnt[0, h, i]]
+            if not np.array_equal(gsel, ref_sel):
+                continue  # tie rows are covered by test_block_select
+            ref, _ = O.sparse_attn_rows(host["q"], host["k"], host["v"], blocks, ref_sel, scale, 0,
+                                        h, i)
+            assert_close(got[0, s:s + n, h], ref, "bf16", f"e2e h{h} blk{i}")
+            checked += 1
+    assert checked >= 0.95 * w.heads * len(blocks)
