@@ -113,14 +113,15 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.lines = []
+        self.lines = []      # (host arrival time, csv line)
         self.thread = None
+        self.window = None   # host-time window of the timed region
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -130,9 +131,9 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
 
-    def stop(self) -> dict:
+    def stop(self, window=None) -> dict:
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -144,7 +145,15 @@ class ClockSampler:
             self.thread.join(timeout=2)
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        lines = self.lines
+        if window is not None:
+            inside = [l for l in lines if window[0] <= l[0] <= window[1] + 0.1]
+            if inside:
+                lines = inside
+            else:  # timed region shorter than the sampling period: nearest sample
+                mid = 0.5 * (window[0] + window[1])
+                lines = sorted(lines, key=lambda l: abs(l[0] - mid))[:1]
+        for _, line in lines:
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
                 continue
@@ -225,9 +234,11 @@ def oracle_sample(w: WL.Workload, host: dict, rows: int, seed: int = 0):
 
 def cpu_baseline(w: WL.Workload, host: dict, target_s: float = 15.0) -> dict:
     """Time the oracle as it stands on a bounded sample (about `target_s`)."""
-    probe_rows = 16
-    dt, _ = oracle_sample(w, host, probe_rows, seed=1)
-    rows = int(max(8, min(w.n_tokens, probe_rows * target_s / max(dt, 1e-3))))
+    # two probes separate the fixed cost (RoPE of every key) from the per-row cost
+    d1, _ = oracle_sample(w, host, 8, seed=1)
+    d2, _ = oracle_sample(w, host, 32, seed=1)
+    per_row = max((d2 - d1) / 24.0, 1e-4)
+    rows = int(max(8, min(w.n_tokens, (target_s - d1) / per_row)))
     dt, flops = oracle_sample(w, host, rows, seed=2)
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": f"{rows} sampled query rows x {w.heads} heads (+ all audio rows for the "
@@ -341,12 +352,15 @@ def run_gpu(args) -> int:
     time.sleep(0.3)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    host_t0 = time.time()
     t_start.record(stream)
     for i in range(args.steps):
         step(evs[i])
     t_end.record(stream)
     torch.cuda.synchronize(dev)
-    clocks = sampler.stop()
+    host_t1 = time.time()
+    time.sleep(0.15)
+    clocks = sampler.stop((host_t0, host_t1))
     barrier(world, dev)
     if M.device_status(stream) != 0:
         raise RuntimeError("device status after timing: " + M.last_error())
