@@ -183,6 +183,32 @@ MMDIT_API size_t mmdit_av_cross_attn_workspace_size(const mmdit_tensor_desc* vid
                                           const mmdit_tensor_desc* audio);
 
 /*
+ * mmdit_av_cross_attn_noalloc -- the same cross-attention as
+ *   mmdit_av_cross_attn, for callers that cannot allocate device memory or
+ *   size a workspace (a plugin inside a runtime that owns every device
+ *   allocation, a serving loop that forbids allocation after start-up).  The
+ *   source pages have no counterpart: this is an interface convenience.
+ *   Scratch is a fixed file-scope device array of MMDIT_NOALLOC_SCRATCH_BYTES
+ *   that every GPU loading the library holds until exit; the call performs no
+ *   cudaMalloc/cudaFree and no allocating library routine.  Arguments and
+ *   outputs are those of mmdit_av_cross_attn minus the workspace; bf16 only.
+ *   The first call on each device (with that device current) looks up the
+ *   array's device address and caches it, so make that first call before any
+ *   stream capture.  All calls share the array: calls that overlap on the GPU
+ *   race.  The split of the video keys is reduced until the partial results
+ *   fit; problems whose batch*heads*ceil(Na/256)*256 rows need more than the
+ *   array even unsplit (130 floats per row) are rejected with MMDIT_EINVAL.
+ *   Errors : EINVAL, EUNSUPPORTED, ECUDA.
+ */
+#define MMDIT_NOALLOC_SCRATCH_BYTES (16 * 1024 * 1024)
+MMDIT_API int mmdit_av_cross_attn_noalloc(const void* qv, const void* kv, const void* vv,
+                                          const void* qa, const void* ka, const void* va,
+                                          void* o_video, void* o_audio,
+                                          const mmdit_tensor_desc* video,
+                                          const mmdit_tensor_desc* audio, float scale,
+                                          mmdit_stream_t stream);
+
+/*
  * mmdit_block_select -- hybrid top-k / top-p key-block selection of the
  *   block-sparse mode (Prism guide, Method section 3).
  *   Q and K of one block-major video segment are mean-pooled per 4x4x4 block

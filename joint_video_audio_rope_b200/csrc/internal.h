@@ -80,5 +80,13 @@ cudaError_t launch_union(const int32_t* idx, const int32_t* cnt, int cap, const 
 
 // helpers (mmdit_api.cu)
 int* device_error_flag();  // device address of this device's error word
+int fail(int code, const char* fmt, ...);  // sets the thread-local message
+int cuda_fail(cudaError_t e, const char* what);
+bool aligned16(const void* p);
+int check_desc(const mmdit_tensor_desc* d, const char* name);
+int make_map(CUtensorMap* m, const void* base, const mmdit_tensor_desc& d, int n_tokens,
+             const char* name);
+int check_sm100();
+size_t align256(size_t x);
 
 }  // namespace mmdit

@@ -16,8 +16,11 @@ namespace mmdit {
 __device__ int g_device_error_word = 0;
 
 namespace {
-
 thread_local std::string t_last_error;
+}  // namespace
+
+// Helpers below are shared with the other entry-point file (noalloc.cu)
+// through internal.h.
 
 int fail(int code, const char* fmt, ...) {
   char buf[512];
@@ -219,8 +222,6 @@ CrossPlan plan_cross(const mmdit_tensor_desc* v, const mmdit_tensor_desc* a) {
   p.part_ml_bytes = align256(rows * 2 * sizeof(float));
   return p;
 }
-
-}  // namespace
 
 int* device_error_flag() {
   static int* cache[64] = {};

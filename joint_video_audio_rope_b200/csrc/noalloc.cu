@@ -1,0 +1,151 @@
+// Allocation-free variant of the audio<->video cross-attention.
+//
+// The regular mmdit_av_cross_attn needs a caller-sized workspace for the
+// split-KV partial results of the audio-query direction.  Some callers cannot
+// provide one: a plugin hosted by an inference runtime that owns every device
+// allocation of the process, or a serving loop that forbids allocation after
+// start-up so that its memory footprint stays fixed, has no way to call
+// cudaMalloc or to grow a workspace on demand.  mmdit_av_cross_attn_noalloc
+// serves them: its scratch is a fixed file-scope device array of
+// MMDIT_NOALLOC_SCRATCH_BYTES, so the call allocates nothing.  Every GPU that
+// loads this library holds that array until the process exits.
+//
+// The array is a device symbol.  Host code cannot use its name as an address
+// (a kernel handed the host-side stand-in would fault or, where the GPU can
+// reach host memory, silently use the wrong memory), so the first call on each
+// device, with that device current, looks the address up once with
+// cudaGetSymbolAddress and caches it; that first call should therefore come
+// before any stream capture.  Every call shares the array and finds the
+// previous call's contents in it; nothing here needs it zeroed (every partial
+// row is written before it is read).  Calls that overlap on the GPU (two
+// streams, or two host threads on one device) race on the array.
+#include <mutex>
+
+#include "internal.h"
+
+namespace mmdit {
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MMDIT_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device (looked up once
+// per device).
+int scratch_address(void** out) {
+  static void* cache[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(MMDIT_EUNSUPPORTED, "device index %d >= 64", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(noalloc scratch)");
+    cache[dev] = p;
+  }
+  *out = cache[dev];
+  return MMDIT_OK;
+}
+
+}  // namespace
+
+}  // namespace mmdit
+
+using namespace mmdit;
+
+extern "C" int mmdit_av_cross_attn_noalloc(const void* qv, const void* kv, const void* vv,
+                                           const void* qa, const void* ka, const void* va,
+                                           void* o_video, void* o_audio,
+                                           const mmdit_tensor_desc* video,
+                                           const mmdit_tensor_desc* audio, float scale,
+                                           mmdit_stream_t stream) {
+  int rc;
+  if ((rc = check_desc(video, "video")) || (rc = check_desc(audio, "audio"))) return rc;
+  if (video->batch != audio->batch || video->heads != audio->heads ||
+      video->head_dim != audio->head_dim || video->dtype != audio->dtype)
+    return fail(MMDIT_EINVAL, "av_cross_noalloc: video and audio descriptors disagree");
+  if (video->dtype != MMDIT_BF16)
+    return fail(MMDIT_EUNSUPPORTED, "av_cross_noalloc: bf16 only");
+  const void* ptrs[8] = {qv, kv, vv, qa, ka, va, o_video, o_audio};
+  for (const void* p : ptrs) {
+    if (p == nullptr) return fail(MMDIT_EINVAL, "av_cross_noalloc: every tensor must be non-NULL");
+    if (!aligned16(p)) return fail(MMDIT_EINVAL, "av_cross_noalloc: 16-byte alignment");
+  }
+  if (video->n_tokens < 1 || audio->n_tokens < 1)
+    return fail(MMDIT_EINVAL, "av_cross_noalloc: both streams need at least one token");
+  if (!(scale > 0.f) || !isfinite(scale))
+    return fail(MMDIT_EINVAL, "av_cross_noalloc: scale must be > 0");
+
+  // Split the video keys of the audio-query direction as the regular call
+  // does (<= 32 key tiles per split), then lower the split count until the
+  // partial results fit the fixed scratch array.
+  const int n_qtiles = (audio->n_tokens + 255) / 256;
+  const int nq_pad = n_qtiles * 256;
+  const int tiles = (video->n_tokens + 127) / 128;
+  const size_t rows_per_split = (size_t)audio->batch * audio->heads * nq_pad;
+  auto bytes_for = [&](int splits) {
+    return align256((size_t)splits * rows_per_split * 128 * sizeof(float)) +
+           align256((size_t)splits * rows_per_split * 2 * sizeof(float));
+  };
+  int splits = std::max(1, (tiles + 31) / 32);
+  while (splits > 1 && bytes_for(splits) > (size_t)MMDIT_NOALLOC_SCRATCH_BYTES) --splits;
+  if (bytes_for(splits) > (size_t)MMDIT_NOALLOC_SCRATCH_BYTES)
+    return fail(MMDIT_EINVAL,
+                "av_cross_noalloc: batch*heads*audio rows need %zu bytes of scratch; the "
+                "fixed maximum is %d bytes (use mmdit_av_cross_attn with a workspace)",
+                bytes_for(1), MMDIT_NOALLOC_SCRATCH_BYTES);
+  const int kv_per_split = ((tiles + splits - 1) / splits) * 128;
+  splits = (video->n_tokens + kv_per_split - 1) / kv_per_split;
+  if ((rc = check_sm100())) return rc;
+  void* scratch = nullptr;
+  if ((rc = scratch_address(&scratch))) return rc;
+
+  AttnParams p{};
+  AttnProblem& a2v = p.prob[0];
+  if ((rc = make_map(&a2v.tmQ, qa, *audio, audio->n_tokens, "qa")) ||
+      (rc = make_map(&a2v.tmK, kv, *video, video->n_tokens, "kv")) ||
+      (rc = make_map(&a2v.tmV, vv, *video, video->n_tokens, "vv")))
+    return rc;
+  a2v.part_o = static_cast<float*>(scratch);
+  a2v.part_ml = reinterpret_cast<float*>(
+      static_cast<char*>(scratch) + align256((size_t)splits * rows_per_split * 128 * sizeof(float)));
+  a2v.Nq = audio->n_tokens;
+  a2v.Nkv = video->n_tokens;
+  a2v.H = audio->heads;
+  a2v.B = audio->batch;
+  a2v.n_qtiles = n_qtiles;
+  a2v.n_splits = splits;
+  a2v.kv_per_split = kv_per_split;
+  a2v.ctas = n_qtiles * splits * a2v.H * a2v.B;
+  a2v.mode = kModeDense;
+  AttnProblem& v2a = p.prob[1];
+  if ((rc = make_map(&v2a.tmQ, qv, *video, video->n_tokens, "qv")) ||
+      (rc = make_map(&v2a.tmK, ka, *audio, audio->n_tokens, "ka")) ||
+      (rc = make_map(&v2a.tmV, va, *audio, audio->n_tokens, "va")))
+    return rc;
+  v2a.o = (__nv_bfloat16*)o_video;
+  v2a.o_st = video->stride_tok;
+  v2a.o_sb = video->stride_batch;
+  v2a.Nq = video->n_tokens;
+  v2a.Nkv = audio->n_tokens;
+  v2a.H = video->heads;
+  v2a.B = video->batch;
+  v2a.n_qtiles = (video->n_tokens + 255) / 256;
+  v2a.n_splits = 1;
+  v2a.kv_per_split = ((audio->n_tokens + 127) / 128) * 128;
+  v2a.ctas = v2a.n_qtiles * v2a.H * v2a.B;
+  v2a.mode = kModeDense;
+  p.n_prob = 2;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.err = device_error_flag();
+  if (p.err == nullptr) return fail(MMDIT_ECUDA, "device error flag unavailable");
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = launch_attn_tc(p, s);
+  if (e == cudaSuccess)
+    e = launch_split_combine(a2v.part_o, a2v.part_ml, (__nv_bfloat16*)o_audio, audio->stride_tok,
+                             audio->stride_batch, splits, audio->batch, audio->heads,
+                             audio->n_tokens, nq_pad, s);
+  return e == cudaSuccess ? MMDIT_OK : cuda_fail(e, "av_cross_noalloc launch");
+}

@@ -62,6 +62,8 @@ _SIGS = {
     "mmdit_av_cross_attn": (C.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _D, _D, C.c_float, _P,
                                       C.c_size_t, _P]),
     "mmdit_av_cross_attn_workspace_size": (C.c_size_t, [_D, _D]),
+    "mmdit_av_cross_attn_noalloc": (C.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _D, _D, C.c_float,
+                                              _P]),
     "mmdit_block_select": (C.c_int, [_P, _P, _D, _L, C.c_int, C.c_float, C.c_float, C.c_int,
                                      _P, _P, _P, C.c_size_t, _P]),
     "mmdit_block_select_workspace_size": (C.c_size_t, [_D, _L]),
@@ -186,6 +188,19 @@ def av_cross_attn(qv, kv, vv, qa, ka, va, o_video, o_audio, video: TensorDesc,
 
 def av_cross_attn_workspace_size(video: TensorDesc, audio: TensorDesc) -> int:
     return _lib.mmdit_av_cross_attn_workspace_size(C.byref(video), C.byref(audio))
+
+
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024  # MMDIT_NOALLOC_SCRATCH_BYTES
+
+
+def av_cross_attn_noalloc(qv, kv, vv, qa, ka, va, o_video, o_audio, video: TensorDesc,
+                          audio: TensorDesc, scale: float, stream=None) -> None:
+    """av_cross_attn without a workspace: the library's fixed device scratch
+    array is used instead (for callers that cannot allocate device memory)."""
+    _check(_lib.mmdit_av_cross_attn_noalloc(_ptr(qv), _ptr(kv), _ptr(vv), _ptr(qa), _ptr(ka),
+                                            _ptr(va), _ptr(o_video), _ptr(o_audio),
+                                            C.byref(video), C.byref(audio), scale,
+                                            _stream(stream)))
 
 
 def block_select(q, k, desc: TensorDesc, layout: Layout, top_k: int, top_p: float, scale: float,
