@@ -92,6 +92,30 @@ def dense_step_flops(w: WL.Workload) -> dict:
             "cross": attn_flops(nv, na, d, H, B) + attn_flops(na, nv, d, H, B)}
 
 
+# DRAM bytes per launch of the dominant kernel from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), valid only while the kernel
+# source is the one that was captured (sha1 of attn_tc.cu + common.cuh).
+NCU_TRAFFIC = {
+    "480p": {"src": "cdceda44044c6879", "bytes": 832812032},  # profiles/attn_tc_joint_480p.md
+}
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha1()
+    for f in ("attn_tc.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "joint_video_audio_rope_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str):
+    t = NCU_TRAFFIC.get(workload)
+    if t is None or t["src"] != kernel_source_hash():
+        return None
+    return t["bytes"]
+
+
 def read_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -232,13 +256,22 @@ def oracle_sample(w: WL.Workload, host: dict, rows: int, seed: int = 0):
     return time.perf_counter() - t0, flops
 
 
+def calibrate_rows(w: WL.Workload, host: dict, target_s: float) -> int:
+    """Number of sampled query rows whose oracle sample takes about target_s
+    (grown geometrically from a small probe; the fixed cost of rotating every
+    key is part of each probe)."""
+    rows = 8
+    for _ in range(6):
+        dt, _ = oracle_sample(w, host, rows, seed=1)
+        if dt >= 0.5 * target_s or rows >= w.n_tokens:
+            break
+        rows = int(min(w.n_tokens, rows * min(8.0, max(2.0, 0.8 * target_s / max(dt, 1e-3)))))
+    return max(8, rows)
+
+
 def cpu_baseline(w: WL.Workload, host: dict, target_s: float = 15.0) -> dict:
     """Time the oracle as it stands on a bounded sample (about `target_s`)."""
-    # two probes separate the fixed cost (RoPE of every key) from the per-row cost
-    d1, _ = oracle_sample(w, host, 8, seed=1)
-    d2, _ = oracle_sample(w, host, 32, seed=1)
-    per_row = max((d2 - d1) / 24.0, 1e-4)
-    rows = int(max(8, min(w.n_tokens, (target_s - d1) / per_row)))
+    rows = calibrate_rows(w, host, target_s)
     dt, flops = oracle_sample(w, host, rows, seed=2)
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": f"{rows} sampled query rows x {w.heads} heads (+ all audio rows for the "
@@ -432,7 +465,8 @@ def run_gpu(args) -> int:
         "gpu_launches": launches_per_step * args.steps,
         "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (" + dom + ")",
                      "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4), "traffic": ncu_traffic(w.name),
+                     "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "peak_source": f"bf16_tflops_sustained of {peak_src}"},
         "clocks": clocks,
     }
@@ -461,8 +495,7 @@ def run_reference(args) -> int:
     x = WL.generate(w)
     cores = blas_threads()
     # calibrate one step to about args.ref_step_seconds of oracle work
-    dt, _ = oracle_sample(w, x, 16, seed=1)
-    rows = int(max(8, min(w.n_tokens, 16 * args.ref_step_seconds / max(dt, 1e-3))))
+    rows = calibrate_rows(w, x, args.ref_step_seconds)
     for i in range(args.warmup):
         oracle_sample(w, x, rows, seed=100 + i)
     tot_s, tot_f = 0.0, 0.0
