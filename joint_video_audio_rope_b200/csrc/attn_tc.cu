@@ -48,6 +48,16 @@ constexpr int kKVOff = 2 * kTileBytes;
 constexpr int kBarOff = kKVOff + kStages * kTileBytes;
 constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + barriers + alignment slack
 constexpr float kRescaleLog2 = 8.0f;      // move the max only beyond a factor 2^8
+// 32-column chunks of S whose exponentials run on the FMA pipe (polynomial)
+// instead of the MUFU, on tiles without masked columns: bit c = chunk c.
+// Measured on B200 (480p joint attention): 0 chunks 1113 TFLOP/s, 1 chunk
+// 961, 2 chunks 849 -- the softmax is bound by the latency of its per-tile
+// handoffs, not by MUFU throughput, so the default keeps every exponential on
+// the MUFU.
+#ifndef MMDIT_POLY_CHUNKS
+#define MMDIT_POLY_CHUNKS 0x0
+#endif
+constexpr int kPolyChunks = MMDIT_POLY_CHUNKS;
 
 // barrier indices (8 bytes each)
 enum {
@@ -116,22 +126,14 @@ __device__ __forceinline__ Work decode_work(const AttnParams& P) {
 
 // Token start of the two 64-row halves of key tile j, and (sparse) the
 // merged-list entries they come from.
-__device__ __forceinline__ void kv_tile(const AttnProblem& pr, const Work& w, int j, int& s0,
-                                        int& s1, uint32_t& e0, uint32_t& e1) {
+__device__ __forceinline__ void kv_tile(const AttnProblem& pr, const Work& w, int j, int ucount,
+                                        int& s0, int& s1) {
   if (pr.mode == kModeDense) {
     s0 = w.kv_lo + j * 128;
     s1 = s0 + 64;
-    e0 = e1 = 0;
   } else {
-    const int cnt = pr.ucnt[((long long)w.b * pr.H + w.h) * pr.n_qtiles + w.qtile];
-    e0 = pr.ulist[w.ubase + 2 * j];
-    e1 = (2 * j + 1 < cnt) ? pr.ulist[w.ubase + 2 * j + 1] : 0u;
-    int len;
-    block_extent(pr.vT, pr.vH, pr.vW, (int)(e0 & 0xFFFFu), s0, len);
-    if (2 * j + 1 < cnt)
-      block_extent(pr.vT, pr.vH, pr.vW, (int)(e1 & 0xFFFFu), s1, len);
-    else
-      s1 = s0;  // loaded but fully masked
+    s0 = (int)pr.ulist[w.ubase + 2 * j].x;
+    s1 = (2 * j + 1 < ucount) ? (int)pr.ulist[w.ubase + 2 * j + 1].x : s0;  // else fully masked
   }
 }
 
@@ -251,10 +253,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int last[kStages] = {-1, -1, -1, -1};
       bool ok = true;
+      const int ucount = pr.mode == kModeSparse
+                             ? pr.ucnt[((long long)w.b * pr.H + w.h) * pr.n_qtiles + w.qtile]
+                             : 0;
       for (int j = 0; j < nkv && ok; ++j) {
         int s0, s1;
-        uint32_t e0, e1;
-        kv_tile(pr, w, j, s0, s1, e0, e1);
+        kv_tile(pr, w, j, ucount, s0, s1);
         for (int kind = 0; kind < 2; ++kind) {
           const int i = 2 * j + kind;
           const int slot = i % kStages;
@@ -363,7 +367,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     float m_used = -INFINITY, l = 0.f;
+    const uint64_t sl2x2 = pack_f32x2(sl2, sl2);
+    int ucount = 0;
+    if (pr.mode == kModeSparse)
+      ucount = pr.ucnt[((long long)w.b * pr.H + w.h) * pr.n_qtiles + w.qtile];
     for (int j = 0; j < nkv; ++j) {
+      // valid key columns of each 64-row half of this tile for this row
+      // (independent of S, so computed before waiting for it)
+      int len0, len1;
+      if (pr.mode == kModeDense) {
+        const int s0 = w.kv_lo + j * 128;
+        len0 = max(0, min(64, w.kv_hi - s0));
+        len1 = max(0, min(64, w.kv_hi - s0 - 64));
+      } else {
+        const uint2 e0 = pr.ulist[w.ubase + 2 * j];
+        const uint2 e1 = (2 * j + 1 < ucount) ? pr.ulist[w.ubase + 2 * j + 1] : make_uint2(0u, 0u);
+        len0 = ((e0.y >> 16) >> qb) & 1u ? (int)(e0.y & 0xFFu) : 0;
+        len1 = ((e1.y >> 16) >> qb) & 1u ? (int)(e1.y & 0xFFu) : 0;
+      }
       ok = ok && mbar_wait(bar(B_SFULL + t), j & 1, err);
       if (__any_sync(0xffffffffu, !ok)) {
         ok = false;
@@ -372,44 +393,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       tc_fence_after();
       float s[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(s_addr + c * 32, v);
+      {
+        uint32_t v0[32], v1[32], v2[32], v3[32];
+        tmem_ld32(s_addr, v0);
+        tmem_ld32(s_addr + 32, v1);
+        tmem_ld32(s_addr + 64, v2);
+        tmem_ld32(s_addr + 96, v3);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(v[i]);
-      }
-      // valid key columns of each 64-row half for this row
-      int len0, len1;
-      if (pr.mode == kModeDense) {
-        const int s0 = w.kv_lo + j * 128;
-        len0 = max(0, min(64, w.kv_hi - s0));
-        len1 = max(0, min(64, w.kv_hi - s0 - 64));
-      } else {
-        const int cnt = pr.ucnt[((long long)w.b * pr.H + w.h) * pr.n_qtiles + w.qtile];
-        const uint32_t e0 = pr.ulist[w.ubase + 2 * j];
-        const uint32_t e1 = (2 * j + 1 < cnt) ? pr.ulist[w.ubase + 2 * j + 1] : 0u;
-        int st;
-        block_extent(pr.vT, pr.vH, pr.vW, (int)(e0 & 0xFFFFu), st, len0);
-        len0 = ((e0 >> 16) >> qb) & 1u ? len0 : 0;
-        if (2 * j + 1 < cnt) {
-          block_extent(pr.vT, pr.vH, pr.vW, (int)(e1 & 0xFFFFu), st, len1);
-          len1 = ((e1 >> 16) >> qb) & 1u ? len1 : 0;
-        } else {
-          len1 = 0;
+        for (int i = 0; i < 32; ++i) {
+          s[i] = __uint_as_float(v0[i]);
+          s[32 + i] = __uint_as_float(v1[i]);
+          s[64 + i] = __uint_as_float(v2[i]);
+          s[96 + i] = __uint_as_float(v3[i]);
         }
       }
-      if (len0 < 64 || len1 < 64) {
+      const bool masked = len0 < 64 || len1 < 64;
+      if (masked) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           if (c >= len0) s[c] = -INFINITY;
           if (c >= len1) s[64 + c] = -INFINITY;
         }
       }
-      float mt = s[0];
-#pragma unroll
-      for (int c = 1; c < 128; ++c) mt = fmaxf(mt, s[c]);
+      const float mt = row_max128(s);
       const bool grow = mt > m_used + thresh || (m_used == -INFINITY && mt > -INFINITY);
       float alpha = 1.f;
       if (grow) {
@@ -432,21 +439,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
       }
       const float mref = (m_used == -INFINITY) ? 0.f : m_used * sl2;
-      float sum = 0.f;
+      const uint64_t nm2 = pack_f32x2(-mref, -mref);
+      // Exponentials: MUFU ex2 for most columns; on tiles without masked
+      // columns, the columns of kPolyChunks go to the FMA pipe instead.
+      const bool poly_ok = !__any_sync(0xffffffffu, masked);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t v[32];
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+        const bool poly = poly_ok && ((kPolyChunks >> c) & 1);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2_approx(fmaf(s[c * 64 + 2 * i], sl2, -mref));
-          const float p1 = ex2_approx(fmaf(s[c * 64 + 2 * i + 1], sl2, -mref));
-          v[i] = pack_bf16x2(p0, p1);
-          sum += p0 + p1;
+        for (int i = 0; i < 16; ++i) {
+          const uint64_t x2 = ffma_f32x2(pack_f32x2(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]),
+                                         sl2x2, nm2);
+          float p0, p1;
+          if (poly) {
+            exp2_poly_f32x2(x2, p0, p1);
+          } else {
+            float x0, x1;
+            unpack_f32x2(x2, x0, x1);
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          pk[i] = pack_bf16x2(p0, p1);
+          acc[i & 3] = add_f32x2(acc[i & 3], pack_f32x2(p0, p1));
         }
-        tmem_st32(s_addr + c * 32, v);
+        tmem_st16(s_addr + c * 16, pk);  // P: 2 bf16 per column
       }
       tmem_wait_st();
-      l += sum;
+      {
+        float a0, a1, b0, b1, c0, c1, d0, d1;
+        unpack_f32x2(add_f32x2(acc[0], acc[1]), a0, a1);
+        unpack_f32x2(add_f32x2(acc[2], acc[3]), b0, b1);
+        (void)c0; (void)c1; (void)d0; (void)d1;
+        l += (a0 + a1) + (b0 + b1);
+      }
       tc_fence_before();
       mbar_arrive(bar(B_PFULL + t));
     }

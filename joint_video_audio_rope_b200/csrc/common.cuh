@@ -275,6 +275,87 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
          | ((uint32_t)(M >> 4) << 24);   // M / 16
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15])
+      : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// packed fp32x2 arithmetic (sm_100: one instruction for two lanes of fp32)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack_f32x2(uint64_t r, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t ffma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Maximum of 128 values as eight independent 3-input-max chains and a small
+// tree (depth 11 instead of a 127-long dependency chain).
+__device__ __forceinline__ float row_max128(const float (&s)[128]) {
+  float a[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = s[k];
+#pragma unroll
+  for (int i = 8; i + 16 <= 128; i += 16) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = max3f(a[k], s[i + k], s[i + 8 + k]);
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = fmaxf(a[k], s[120 + k]);
+  return max3f(max3f(a[0], a[1], a[2]), max3f(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+}
+
+// 2^x on the FMA pipe for two lanes, x <= 8 (used on part of the softmax
+// columns to unload the MUFU).  Range reduction after Cody and Waite: j =
+// round(x) by the 1.5*2^23 shift, f = x - j in [-1/2, 1/2] exactly; 2^f by a
+// degree-3 polynomial fitted for relative error (coefficients from
+// csrc/fit_exp2_poly.py, max relative error 7.5e-5 in fp32); 2^j is added to
+// the exponent field: bits(t) << 23 equals j << 23 modulo 2^32 because the
+// shift constant's low nine bits are zero.  x is clamped at -125 so the result
+// stays a normal number (values that small vanish against the row sum >= 1).
+__device__ __forceinline__ void exp2_poly_f32x2(uint64_t x2, float& p0, float& p1) {
+  float x0, x1;
+  unpack_f32x2(x2, x0, x1);
+  const uint64_t x = pack_f32x2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t magic = pack_f32x2(12582912.f, 12582912.f);
+  const uint64_t nmagic = pack_f32x2(-12582912.f, -12582912.f);
+  const uint64_t t = add_f32x2(x, magic);
+  const uint64_t jf = add_f32x2(t, nmagic);
+  const uint64_t f = ffma_f32x2(jf, pack_f32x2(-1.f, -1.f), x);
+  uint64_t p = ffma_f32x2(pack_f32x2(0.05517132207751274f, 0.05517132207751274f), f,
+                          pack_f32x2(0.24261054396629333f, 0.24261054396629333f));
+  p = ffma_f32x2(p, f, pack_f32x2(0.6932609677314758f, 0.6932609677314758f));
+  p = ffma_f32x2(p, f, pack_f32x2(0.9999281167984009f, 0.9999281167984009f));
+  float pa, pb, ta, tb;
+  unpack_f32x2(p, pa, pb);
+  unpack_f32x2(t, ta, tb);
+  p0 = __int_as_float(__float_as_int(pa) + (__float_as_int(ta) << 23));
+  p1 = __int_as_float(__float_as_int(pb) + (__float_as_int(tb) << 23));
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

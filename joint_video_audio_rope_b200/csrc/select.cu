@@ -18,9 +18,10 @@
 //   groups_kernel  partitions the query blocks into CTA groups of <= 256
 //                  tokens and <= 16 blocks (greedy, in block order).
 //   union_kernel   per (group, head, batch): merges the groups' selected
-//                  lists into one ascending list whose entries carry a
-//                  16-bit membership mask (which query blocks of the group
-//                  selected the key block).  The attention kernel walks it.
+//                  lists into one ascending list; each entry holds the key
+//                  block's start token, its length and a 16-bit membership
+//                  mask (which query blocks of the group selected it).  The
+//                  attention kernel walks it.
 #include <math.h>
 
 #include "internal.h"
@@ -193,7 +194,7 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ q
     } else if (target > m_gt && tv > 0.0) {
       m = (int)ceil((target - m_gt) / tv);
     }
-    m = max(1, min(m, c_eq));
+    m = c_eq > 0 ? max(1, min(m, c_eq)) : 0;
     take_p = c_gt + m;
   }
   // final threshold and number of tied blocks to take (lowest ids first)
@@ -249,8 +250,8 @@ __global__ void groups_kernel(int T, int H, int W, int nblk, int4* groups) {
 __global__ void __launch_bounds__(256) union_kernel(const int32_t* __restrict__ idx,
                                                     const int32_t* __restrict__ cnt, int cap,
                                                     const int4* __restrict__ groups, int H,
-                                                    int nblk, int n_groups,
-                                                    uint32_t* __restrict__ ulist,
+                                                    int nblk, int n_groups, int T, int Hg, int Wg,
+                                                    uint2* __restrict__ ulist,
                                                     int* __restrict__ ucnt) {
   extern __shared__ uint32_t mask[];  // [nblk]
   __shared__ int warp_tot[8];
@@ -270,7 +271,7 @@ __global__ void __launch_bounds__(256) union_kernel(const int32_t* __restrict__ 
   }
   __syncthreads();
   const long long lid = ((long long)b * H + h) * n_groups + g;
-  uint32_t* out = ulist + lid * nblk;
+  uint2* out = ulist + lid * nblk;
   int running = 0;
   for (int j0 = 0; j0 < nblk; j0 += 256) {
     const int j = j0 + tid;
@@ -284,7 +285,12 @@ __global__ void __launch_bounds__(256) union_kernel(const int32_t* __restrict__ 
       before += (w < warp) ? warp_tot[w] : 0;
       total += warp_tot[w];
     }
-    if (m != 0u) out[running + before + __popc(bal & ((1u << lane) - 1u))] = (uint32_t)j | (m << 16);
+    if (m != 0u) {
+      int st, len;
+      block_extent(T, Hg, Wg, j, st, len);
+      out[running + before + __popc(bal & ((1u << lane) - 1u))] =
+          make_uint2((uint32_t)st, (uint32_t)len | (m << 16));
+    }
     running += total;
     __syncthreads();
   }
@@ -324,8 +330,8 @@ cudaError_t launch_groups(int T, int H, int W, int nblk, int4* groups, int*, cud
 }
 
 cudaError_t launch_union(const int32_t* idx, const int32_t* cnt, int cap, const int4* groups,
-                         int n_groups, const int*, int B, int H, int nblk, uint32_t* ulist,
-                         int* ucnt, cudaStream_t s) {
+                         int n_groups, const int*, int B, int H, int nblk, int T, int Hg,
+                         int Wg, uint2* ulist, int* ucnt, cudaStream_t s) {
   if (n_groups == 0) return cudaSuccess;
   const size_t smem = sizeof(uint32_t) * (size_t)nblk;
   if (smem > 48 * 1024) {
@@ -334,7 +340,7 @@ cudaError_t launch_union(const int32_t* idx, const int32_t* cnt, int cap, const 
     if (e != cudaSuccess) return e;
   }
   union_kernel<<<dim3(n_groups, H, B), 256, smem, s>>>(idx, cnt, cap, groups, H, nblk, n_groups,
-                                                       ulist, ucnt);
+                                                       T, Hg, Wg, ulist, ucnt);
   return cudaGetLastError();
 }
 

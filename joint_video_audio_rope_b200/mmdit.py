@@ -15,7 +15,8 @@ import re
 from typing import Iterable, Optional, Sequence
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmmdit.so")
+# MMDIT_LIB may point at another build of the same library (e.g. a variant).
+LIB_PATH = os.environ.get("MMDIT_LIB") or os.path.join(_PKG, "libmmdit.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "mmdit.h")
 
 if not os.path.exists(LIB_PATH):
