@@ -25,6 +25,15 @@ def rope_bands(head_dim):
     return head_dim - 2 * dh, dh, dh
 
 
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """Values rounded to bfloat16 (via float32, nearest even), as float64.
+
+    Models the bf16 storage of an intermediate tensor between two steps of
+    the path (e.g. the RoPE output that the attention step reads); the
+    rounding is done by the test on the oracle's own values."""
+    return WL.bf16_bits_to_f32(WL.f32_to_bf16_bits(np.asarray(x, np.float32))).astype(np.float64)
+
+
 def to_device(x: np.ndarray, dtype: str):
     import torch
     if dtype == "bf16":

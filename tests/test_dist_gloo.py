@@ -1,0 +1,68 @@
+"""Multi-process host logic of bench.py on CPU (gloo, world size 2): rank
+discovery from the torchrun environment, the barrier around the timed region
+and the max-over-ranks reduction of the per-rank device time.  The data path
+itself has no collective (replicas, weak scaling)."""
+import os
+import socket
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch.distributed as dist
+
+    import bench
+    r, w, lr = bench.dist_env()
+    dist.init_process_group("gloo", rank=r, world_size=w, timeout=datetime.timedelta(seconds=60))
+    bench.barrier(w)
+    # each rank "measured" a different time; every rank must see the max
+    got = bench.reduce_max(10.0 + 5.0 * r, w)
+    bench.barrier(w)
+    dist.destroy_process_group()
+    out.put((r, w, lr, got))
+
+
+def test_rank_logic_two_processes():
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res == [(0, 2, 0, 15.0), (1, 2, 1, 15.0)]
+
+
+def test_single_rank_is_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.reduce_max(3.5, 1) == 3.5
+    bench.barrier(1)  # no process group needed
+
+
+def test_reference_arm_other_ranks_exit_without_work(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    assert bench.main(["--impl", "reference", "--workload", "tiny_f32"]) == 0

@@ -1,0 +1,196 @@
+"""Full-size parity: the benchmark workloads at their full sizes, run through
+the same C-ABI calls and launch configuration that bench.py times, checked
+against the fp64 oracle on sampled outputs it can compute one by one.
+
+Sampled rows per (batch, head): seeded random query rows, the first and last
+rows of the sequence and of every segment (the edge tiles, conditioning
+frames, audio and text), and every audio row for the audio-query direction
+of the cross-attention.  Tolerances: bf16 max-abs 2e-2, relative-L2 5e-3.
+The block-sparse workload additionally checks selected block sets exactly
+(outside fp32 ties) on sampled query blocks of four heads, and the sparse
+output of every sampled block whose selection agrees with the oracle.
+
+Between steps the path stores Q and K in bf16 (the RoPE step writes them in
+place), so the oracle's own RoPE output is rounded to bf16 before it feeds the
+oracle's attention and selection; the RoPE step itself is compared unrounded."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle as O
+from joint_video_audio_rope_b200 import workloads as WL
+
+from _util import assert_close, bf16_round, oracle_layout, selection_matches
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+ROWS = 48  # random query rows per (batch, head)
+
+
+@pytest.fixture(scope="module")
+def M():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from joint_video_audio_rope_b200 import build
+    build.build()
+    from joint_video_audio_rope_b200 import mmdit
+    return mmdit
+
+
+def _up(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def _f64(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def _sample_rows(w, rng):
+    n = w.n_tokens
+    rows = set(rng.choice(n, size=min(ROWS, n), replace=False).tolist())
+    start = 0
+    for s in w.segments:
+        e = start + s["n_tokens"]
+        rows.update(range(start, min(start + 3, e)))
+        rows.update(range(max(start, e - 3), e))
+        start = e
+    rows.update(range(0, 2))
+    rows.update(range(n - 2, n))
+    return np.array(sorted(rows))
+
+
+def _run_dense_step(M, w, x):
+    q, k, v = _up(x["q"]), _up(x["k"]), _up(x["v"])
+    desc = M.desc_of(q)
+    lay = M.make_layout(w.segments)
+    M.rope_apply(q, k, desc, lay, M.rope_params(w.theta, 44, 42, 42))
+    o = torch.empty_like(q)
+    scale = 1 / math.sqrt(128)
+    M.joint_attn(q, k, v, o, desc, lay, scale)
+    v0, v1 = w.video_range()
+    a0, a1 = w.audio_range()
+    oc = torch.empty_like(q)
+    dv, da = M.desc_of(q[:, v0:v1]), M.desc_of(q[:, a0:a1])
+    n = M.av_cross_attn_workspace_size(dv, da)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    M.av_cross_attn(q[:, v0:v1], k[:, v0:v1], v[:, v0:v1], q[:, a0:a1], k[:, a0:a1], v[:, a0:a1],
+                    oc[:, v0:v1], oc[:, a0:a1], dv, da, scale, ws, n)
+    torch.cuda.synchronize()
+    assert M.device_status() == M.OK
+    return q, k, o, oc
+
+
+@pytest.mark.parametrize("name", ["480p", "720p", "720p_cond_b2"])
+def test_dense_workload_full_size(M, name):
+    w = WL.WORKLOADS[name]
+    x = WL.generate(w)
+    q, k, o, oc = _run_dense_step(M, w, x)
+    rng = np.random.default_rng(1234)
+    pos = O.positions(oracle_layout(w.segments))
+    scale = 1 / math.sqrt(128)
+    v0, v1 = w.video_range()
+    a0, a1 = w.audio_range()
+    for b in range(w.batch):
+        kk = O.rope(WL.as_f64(x["k"][b], "bf16"), pos, w.theta)        # every key
+        vv = WL.as_f64(x["v"][b], "bf16")
+        rows = _sample_rows(w, rng)
+        qr = O.rope(WL.as_f64(x["q"][b, rows], "bf16"), pos[rows], w.theta)
+        # RoPE outputs of the sampled tokens (all heads)
+        assert_close(_f64(q[b, rows]), qr, "bf16", f"{name} rope q")
+        assert_close(_f64(k[b, rows]), kk[rows], "bf16", f"{name} rope k")
+        kk, qr = bf16_round(kk), bf16_round(qr)
+        got_o = _f64(o[b, rows])
+        got_v = _f64(oc[b, rows])
+        ref_o = np.zeros_like(got_o)
+        for h in range(w.heads):
+            ref_o[:, h], _ = O.attn(qr[:, h], kk[:, h], vv[:, h], scale)
+        assert_close(got_o, ref_o, "bf16", f"{name} joint b{b}")
+        # cross: sampled video rows over the audio keys
+        vr = rows[(rows >= v0) & (rows < v1)]
+        sel = np.isin(rows, vr)
+        ref_v = np.zeros((len(vr), w.heads, 128))
+        for h in range(w.heads):
+            ref_v[:, h], _ = O.attn(qr[sel, h], kk[a0:a1, h], vv[a0:a1, h], scale)
+        assert_close(got_v[sel], ref_v, "bf16", f"{name} cross v<-a b{b}")
+        # cross: every audio row over the video keys
+        qa = bf16_round(O.rope(WL.as_f64(x["q"][b, a0:a1], "bf16"), pos[a0:a1], w.theta))
+        ref_a = np.zeros((a1 - a0, w.heads, 128))
+        for h in range(w.heads):
+            ref_a[:, h], _ = O.attn(qa[:, h], kk[v0:v1, h], vv[v0:v1, h], scale)
+        assert_close(_f64(oc[b, a0:a1]), ref_a, "bf16", f"{name} cross a<-v b{b}")
+
+
+def test_sparse_workload_full_size(M):
+    w = WL.WORKLOADS["1080p_sparse"]
+    x = WL.generate(w)
+    q, k, v = _up(x["q"]), _up(x["k"]), _up(x["v"])
+    v0, v1 = w.video_range()
+    a0, a1 = w.audio_range()
+    desc = M.desc_of(q)
+    lay = M.make_layout(w.segments)
+    M.rope_apply(q, k, desc, lay, M.rope_params(w.theta, 44, 42, 42))
+    vlay = M.make_layout([s for s in w.segments if s["kind"] == WL.SEG_VIDEO])
+    vd = M.desc_of(q[:, v0:v1])
+    nb = M.num_blocks(vlay)
+    scale = 1 / math.sqrt(128)
+    idx = torch.empty((1, w.heads, nb, nb), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((1, w.heads, nb), dtype=torch.int32, device="cuda")
+    n = max(M.block_select_workspace_size(vd, vlay), M.sparse_attn_workspace_size(vd, vlay, nb))
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    M.block_select(q[:, v0:v1], k[:, v0:v1], vd, vlay, w.top_k, w.top_p, scale, nb, idx, cnt, ws, n)
+    o = torch.empty_like(q)
+    M.sparse_attn(q[:, v0:v1], k[:, v0:v1], v[:, v0:v1], o[:, v0:v1], vd, vlay, idx, cnt, nb, scale,
+                  ws, n)
+    oc = torch.empty_like(q)
+    dv, da = M.desc_of(q[:, v0:v1]), M.desc_of(q[:, a0:a1])
+    nc = M.av_cross_attn_workspace_size(dv, da)
+    wc = torch.empty(nc, dtype=torch.uint8, device="cuda")
+    M.av_cross_attn(q[:, v0:v1], k[:, v0:v1], v[:, v0:v1], q[:, a0:a1], k[:, a0:a1], v[:, a0:a1],
+                    oc[:, v0:v1], oc[:, a0:a1], dv, da, scale, wc, nc)
+    torch.cuda.synchronize()
+    assert M.device_status() == M.OK
+
+    seg = w.segments[0]
+    blocks = O.video_blocks(seg["T"], seg["H"], seg["W"])
+    pos = O.positions(oracle_layout(w.segments))
+    rng = np.random.default_rng(99)
+    heads = [0, 7, 13, 23]
+    idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
+    got_o = o[0, v0:v1]
+    p32 = float(np.float32(w.top_p))
+    blk_sample = np.unique(np.concatenate([rng.choice(nb, 24, replace=False),
+                                           [0, 1, nb - 2, nb - 1]]))  # incl. short t-slab
+    for h in heads:
+        qh = O.rope(WL.as_f64(x["q"][0, v0:v1, h:h + 1], "bf16"), pos[v0:v1], w.theta)
+        kh = O.rope(WL.as_f64(x["k"][0, v0:v1, h:h + 1], "bf16"), pos[v0:v1], w.theta)
+        vh = WL.as_f64(x["v"][0, v0:v1, h:h + 1], "bf16")
+        assert_close(_f64(q[0, v0:v1, h]), qh[:, 0], "bf16", f"rope h{h}")
+        qh, kh = bf16_round(qh), bf16_round(kh)
+        qb, kb = O.pool(qh[None], blocks), O.pool(kh[None], blocks)
+        agree = 0
+        for i in blk_sample:
+            ref_sel = O.select_row(qb[0, 0, i], kb[0, 0], w.top_k, p32, scale)
+            got_sel = idx_h[0, h, i, :cnt_h[0, h, i]]
+            P = O.block_probs(qb[0, 0, i], kb[0, 0], scale)
+            assert selection_matches(got_sel, ref_sel, P, w.top_k, p32), f"select h{h} blk{i}"
+            if not np.array_equal(got_sel, ref_sel):
+                continue
+            agree += 1
+            s0, nn = blocks[i]
+            ref, _ = O.sparse_attn_rows(qh[None], kh[None], vh[None], blocks, ref_sel, scale, 0,
+                                        0, i)
+            assert_close(_f64(got_o[s0:s0 + nn, h]), ref, "bf16", f"sparse h{h} blk{i}")
+        assert agree >= 0.9 * len(blk_sample)
+    # dense cross-attention on sampled video rows and every audio row (2 heads)
+    kk = bf16_round(O.rope(WL.as_f64(x["k"][0], "bf16"), pos, w.theta))
+    vv = WL.as_f64(x["v"][0], "bf16")
+    rows = np.sort(rng.choice(v1, 32, replace=False))
+    qr = bf16_round(O.rope(WL.as_f64(x["q"][0, rows], "bf16"), pos[rows], w.theta))
+    qa = bf16_round(O.rope(WL.as_f64(x["q"][0, a0:a1], "bf16"), pos[a0:a1], w.theta))
+    for h in (3, 17):
+        rv, _ = O.attn(qr[:, h], kk[a0:a1, h], vv[a0:a1, h], scale)
+        assert_close(_f64(oc[0, rows, h]), rv, "bf16", f"cross v<-a h{h}")
+        ra, _ = O.attn(qa[:, h], kk[v0:v1, h], vv[v0:v1, h], scale)
+        assert_close(_f64(oc[0, a0:a1, h]), ra, "bf16", f"cross a<-v h{h}")

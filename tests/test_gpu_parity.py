@@ -10,8 +10,8 @@ import pytest
 import oracle as O
 from joint_video_audio_rope_b200 import workloads as WL
 
-from _util import (assert_close, errors, oracle_layout, rope_bands, selection_matches, to_device,
-                   to_host_f64)
+from _util import (assert_close, bf16_round, errors, oracle_layout, rope_bands, selection_matches,
+                   to_device, to_host_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -156,7 +156,8 @@ def test_joint_bf16_fused_rope(M):
     o = torch.empty_like(dev["q"])
     M.joint_attn(dev["q"], dev["k"], dev["v"], o, M.desc_of(dev["q"]), M.make_layout(w.segments),
                  1 / math.sqrt(128), rope_q=M.rope_params(w.theta, 44, 42, 42))
-    ro, _ = O.joint_attn(rq, rk, host["v"], 1 / math.sqrt(128))
+    # Q is rotated in fp32 and held in bf16 shared memory; K is stored in bf16
+    ro, _ = O.joint_attn(bf16_round(rq), bf16_round(rk), host["v"], 1 / math.sqrt(128))
     assert_close(to_host_f64(o), ro, "bf16", "joint fused rope")
     # the caller's Q is not modified by the fused rotation
     assert np.array_equal(to_host_f64(dev["q"]), host["q"])
