@@ -325,8 +325,16 @@ def run_gpu(args) -> int:
         ws_sel = ws_sp = 0
     ws = torch.empty(max(ws_cross, ws_sel, ws_sp, 256), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    # RoPE works in place.  On the block-sparse workload the selected blocks (so
+    # the work) depend on the values, so every step starts from the generated
+    # Q and K (a device copy counted in the step); dense work does not depend
+    # on the values and the step rotates the previous step's tensors again.
+    q0k0 = (q.clone(), k.clone()) if sparse else None
 
     def step(ev=None):
+        if q0k0 is not None:
+            q.copy_(q0k0[0])
+            k.copy_(q0k0[1])
         if ev is not None:
             ev[0].record(stream)
         M.rope_apply(q, k, desc, lay, rope, stream)
@@ -352,7 +360,7 @@ def run_gpu(args) -> int:
             ev[4].record(stream)
 
     # launches of this library's kernels per step
-    launches_per_step = 1 + (2 + 3 if sparse else 1) + 2
+    launches_per_step = 1 + (2 + 3 if sparse else 1) + 3
 
     for _ in range(args.warmup):
         step()
@@ -414,6 +422,9 @@ def run_gpu(args) -> int:
         q.copy_(hq, non_blocking=True)
         k.copy_(hk, non_blocking=True)
         v.copy_(hv, non_blocking=True)
+        if q0k0 is not None:  # the fresh host inputs are the step's inputs
+            q0k0[0].copy_(q)
+            q0k0[1].copy_(k)
         step()
         ho.copy_(o, non_blocking=True)
         hoc.copy_(o_cross, non_blocking=True)

@@ -38,15 +38,29 @@ namespace mmdit {
 
 namespace {
 
-constexpr int kThreads = 320;
-constexpr int kStages = 4;                // K/V ring slots (one 128 x 128 tile each)
-constexpr int kTileBytes = 128 * 128 * 2; // 32 KB
+constexpr int kTileBytes = 128 * 128 * 2; // 32 KB: one 128 x 128 bf16 tile
 constexpr int kHalfCol = 128 * 128;       // bytes of one 64-channel column half
 constexpr int kBoxBytes = 64 * 128;       // one TMA box: 64 rows x 64 channels
-constexpr int kQOff = 0;
-constexpr int kKVOff = 2 * kTileBytes;
-constexpr int kBarOff = kKVOff + kStages * kTileBytes;
-constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + barriers + alignment slack
+
+// Kernel shape: QT Q tiles of 128 rows per CTA (one softmax warpgroup each)
+// and an ST-slot K/V ring.  QT = 2 fills the SM (198 KB smem, 512 TMEM
+// columns) and lets the two tiles ping-pong on the tensor core; QT = 1 with a
+// 2-slot ring needs 97 KB and 256 columns, so two CTAs share an SM and hide
+// each other's load and epilogue latency (used for short key sequences).
+template <int QT, int ST>
+struct Cfg {
+  static constexpr int kThreads = 32 * (4 * QT + 2);
+  static constexpr int kProducerWarp = 4 * QT;
+  static constexpr int kMmaWarp = 4 * QT + 1;
+  static constexpr int kStages = ST;
+  static constexpr int kRows = 128 * QT;  // query rows per CTA
+  static constexpr int kQOff = 0;
+  static constexpr int kKVOff = QT * kTileBytes;
+  static constexpr int kBarOff = kKVOff + ST * kTileBytes;
+  static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + barriers + alignment slack
+  static constexpr int kTmemCols = 256 * QT;               // S_t and O_t per tile
+  static constexpr int kMinBlocks = QT == 1 ? 2 : 1;
+};
 constexpr float kRescaleLog2 = 8.0f;      // move the max only beyond a factor 2^8
 // 32-column chunks of S whose exponentials run on the FMA pipe (polynomial)
 // instead of the MUFU, on tiles without masked columns: bit c = chunk c.
@@ -78,14 +92,14 @@ constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 0, 1);  // P (TMEM), V: M
 struct Work {
   int prob, b, h, split, qtile;
   int q0;       // first query token of the CTA (row 0 of Q tile 0)
-  int q_valid;  // valid query rows of the CTA (<= 256)
+  int q_valid;  // valid query rows of the CTA (<= rows per CTA)
   int kv_lo, kv_hi;  // dense: key range
   int nkv;      // number of 128-row key tiles
   long long ubase;   // sparse: offset of the merged list
   int g_first, g_nblk;
 };
 
-__device__ __forceinline__ Work decode_work(const AttnParams& P) {
+__device__ __forceinline__ Work decode_work(const AttnParams& P, int rows) {
   Work w;
   int idx = blockIdx.x;
   w.prob = 0;
@@ -101,8 +115,8 @@ __device__ __forceinline__ Work decode_work(const AttnParams& P) {
   w.h = idx % pr.H;
   w.b = idx / pr.H;
   if (pr.mode == kModeDense) {
-    w.q0 = w.qtile * 256;
-    w.q_valid = min(256, pr.Nq - w.q0);
+    w.q0 = w.qtile * rows;
+    w.q_valid = min(rows, pr.Nq - w.q0);
     w.kv_lo = w.split * pr.kv_per_split;
     w.kv_hi = min(pr.Nkv, w.kv_lo + pr.kv_per_split);
     w.nkv = w.kv_hi > w.kv_lo ? (w.kv_hi - w.kv_lo + 127) / 128 : 0;
@@ -198,8 +212,14 @@ __device__ void rope_row_smem(uint8_t* q_tile, int r, int tok, const DevLayout& 
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+template <int QT, int ST>
+__global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks)
     attn_tc_kernel(const __grid_constant__ AttnParams P) {
+  using C = Cfg<QT, ST>;
+  constexpr int kStages = C::kStages;
+  constexpr int kQOff = C::kQOff;
+  constexpr int kKVOff = C::kKVOff;
+  constexpr int kBarOff = C::kBarOff;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -209,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + 8 * B_COUNT);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const Work w = decode_work(P);
+  const Work w = decode_work(P, C::kRows);
   const AttnProblem& pr = P.prob[w.prob];
   int* err = P.err;
   const bool skip = *(volatile int*)err != 0;  // an earlier kernel timed out
@@ -229,8 +249,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(B_MMADONE), 1);
     fence_mbar_init();
   }
-  if (warp == 9) {
-    tmem_alloc(smem_u32(tmem_slot), 512);
+  if (warp == C::kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -239,19 +259,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const int nkv = skip ? 0 : w.nkv;
 
-  if (warp == 8) {
+  if (warp == C::kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && !skip) {
       tma_prefetch_desc(&pr.tmQ);
       tma_prefetch_desc(&pr.tmK);
       tma_prefetch_desc(&pr.tmV);
-      for (int t = 0; t < 2; ++t) {
+      for (int t = 0; t < QT; ++t) {
         mbar_expect_tx(bar(B_QFULL + t), kTileBytes);
         const int s0 = w.q0 + t * 128;
         tma_tile(sbase + kQOff + t * kTileBytes, &pr.tmQ, bar(B_QFULL + t), w.h, w.b, s0,
                  s0 + 64);
       }
-      int last[kStages] = {-1, -1, -1, -1};
+      int last[kStages];
+#pragma unroll
+      for (int i = 0; i < kStages; ++i) last[i] = -1;
       bool ok = true;
       const int ucount = pr.mode == kModeSparse
                              ? pr.ucnt[((long long)w.b * pr.H + w.h) * pr.n_qtiles + w.qtile]
@@ -273,28 +295,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // every copy issued must land before the CTA's shared memory goes away
-      for (int t = 0; t < 2; ++t) mbar_wait(bar(B_QFULL + t), 0, err);
+      for (int t = 0; t < QT; ++t) mbar_wait(bar(B_QFULL + t), 0, err);
       for (int s = 0; s < kStages; ++s)
         if (last[s] >= 0) mbar_wait(bar(B_KVFULL + s), (last[s] / kStages) & 1, err);
     }
-  } else if (warp == 9) {
+  } else if (warp == C::kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
+    // Issue order per key tile j (t = Q tiles of the CTA):
+    //   PV_t(j) then QK_t(j+1), tile after tile, so that P_t (which aliases S_t
+    //   in TMEM) is consumed by PV_t before QK_t(j+1) overwrites S_t, and the
+    //   completion of QK_t(j+1) also implies PV_t(j) is done.
     if (lane == 0 && !skip) {
       bool ok = true;
-      const uint32_t q_s[2] = {sbase + kQOff, sbase + kQOff + kTileBytes};
-      const uint32_t s_t[2] = {tmem, tmem + 128};
-      const uint32_t o_t[2] = {tmem + 256, tmem + 384};
       const int qbar = pr.rope_q ? B_QREADY : B_QFULL;
-      for (int t = 0; t < 2 && ok; ++t) ok = mbar_wait(bar(qbar + t), 0, err);
+      for (int t = 0; t < QT && ok; ++t) ok = mbar_wait(bar(qbar + t), 0, err);
       if (ok && nkv > 0) {
-        // prologue: S_t = Q_t K_0^T for both tiles
+        // prologue: S_t = Q_t K_0^T for every tile
         ok = mbar_wait(bar(B_KVFULL + 0), 0, err);
         if (ok) {
           tc_fence_after();
-          mma_qk(s_t[0], q_s[0], sbase + kKVOff);
-          tc_commit(bar(B_SFULL + 0));
-          mma_qk(s_t[1], q_s[1], sbase + kKVOff);
-          tc_commit(bar(B_SFULL + 1));
+#pragma unroll
+          for (int t = 0; t < QT; ++t) {
+            mma_qk(tmem + t * 128, sbase + kQOff + t * kTileBytes, sbase + kKVOff);
+            tc_commit(bar(B_SFULL + t));
+          }
           tc_commit(bar(B_KVEMPTY + 0));
         }
         for (int j = 0; j < nkv && ok; ++j) {
@@ -304,28 +328,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t k_smem = sbase + kKVOff + sk * kTileBytes;
           const bool more = j + 1 < nkv;
           if (!(ok = mbar_wait(bar(B_KVFULL + sv), (iv / kStages) & 1, err))) break;
-          if (!(ok = mbar_wait(bar(B_PFULL + 0), j & 1, err))) break;
-          tc_fence_after();
-          mma_pv(o_t[0], s_t[0], v_smem, j > 0);
-          if (more) {
-            if (!(ok = mbar_wait(bar(B_KVFULL + sk), (ik / kStages) & 1, err))) break;
+#pragma unroll
+          for (int t = 0; t < QT; ++t) {
+            if (!(ok = mbar_wait(bar(B_PFULL + t), j & 1, err))) break;
             tc_fence_after();
-            mma_qk(s_t[0], q_s[0], k_smem);
-            tc_commit(bar(B_SFULL + 0));
-          }
-          if (!(ok = mbar_wait(bar(B_PFULL + 1), j & 1, err))) break;
-          tc_fence_after();
-          mma_pv(o_t[1], s_t[1], v_smem, j > 0);
-          tc_commit(bar(B_KVEMPTY + sv));
-          if (more) {
-            mma_qk(s_t[1], q_s[1], k_smem);
-            tc_commit(bar(B_SFULL + 1));
-            tc_commit(bar(B_KVEMPTY + sk));
+            mma_pv(tmem + QT * 128 + t * 128, tmem + t * 128, v_smem, j > 0);
+            if (t == QT - 1) tc_commit(bar(B_KVEMPTY + sv));
+            if (more) {
+              if (t == 0) {
+                if (!(ok = mbar_wait(bar(B_KVFULL + sk), (ik / kStages) & 1, err))) break;
+                tc_fence_after();
+              }
+              mma_qk(tmem + t * 128, sbase + kQOff + t * kTileBytes, k_smem);
+              tc_commit(bar(B_SFULL + t));
+              if (t == QT - 1) tc_commit(bar(B_KVEMPTY + sk));
+            }
           }
         }
       }
-      tc_commit(bar(B_OFULL + 0));
-      tc_commit(bar(B_OFULL + 1));
+      for (int t = 0; t < QT; ++t) tc_commit(bar(B_OFULL + t));
       tc_commit(bar(B_MMADONE));
       mbar_wait(bar(B_MMADONE), 0, err);
     }
@@ -336,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = t * 128 + r;              // row inside the CTA
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t s_addr = tmem + lane_off + t * 128;
-    const uint32_t o_addr = tmem + lane_off + 256 + t * 128;
+    const uint32_t o_addr = tmem + lane_off + QT * 128 + t * 128;
     const float sl2 = P.scale_log2;
     const float thresh = kRescaleLog2 / sl2;  // in raw score units
     bool ok = !skip;
@@ -490,8 +511,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (pr.part_o != nullptr) {
         // split-KV partial: unnormalised O, running max (log2 units) and sum
         const long long prow =
-            (((long long)w.split * pr.B + w.b) * pr.H + w.h) * (long long)(pr.n_qtiles * 256) +
-            (long long)w.qtile * 256 + row;
+            (((long long)w.split * pr.B + w.b) * pr.H + w.h) * (long long)(pr.n_qtiles * C::kRows) +
+            (long long)w.qtile * C::kRows + row;
         float* dst = pr.part_o + prow * 128;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -552,10 +573,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == C::kMmaWarp) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
@@ -587,20 +608,29 @@ __global__ void split_combine_kernel(const float* __restrict__ part_o,
       __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
 }
 
-}  // namespace
-
-cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
+template <int QT, int ST>
+cudaError_t launch_shape(const AttnParams& p, cudaStream_t s) {
+  using C = Cfg<QT, ST>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<QT, ST>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const int ctas = p.prob[0].ctas + (p.n_prob > 1 ? p.prob[1].ctas : 0);
   if (ctas == 0) return cudaSuccess;
-  attn_tc_kernel<<<ctas, kThreads, kSmemBytes, s>>>(p);
+  attn_tc_kernel<QT, ST><<<ctas, C::kThreads, C::kSmemBytes, s>>>(p);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+int attn_rows_per_cta(int q_tiles) { return 128 * q_tiles; }
+
+cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
+  if (p.q_tiles == 1) return launch_shape<1, 2>(p, s);
+  return launch_shape<2, 4>(p, s);
 }
 
 cudaError_t launch_split_combine(const float* part_o, const float* part_ml, __nv_bfloat16* o,

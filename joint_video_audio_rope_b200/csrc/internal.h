@@ -54,6 +54,7 @@ struct AttnProblem {
 struct AttnParams {
   AttnProblem prob[2];
   int n_prob;
+  int q_tiles;                // 128-row Q tiles per CTA: 2 (default) or 1
   float scale_log2;           // softmax scale * log2(e)
   DevLayout layout;           // for fused Q RoPE
   RopeTab rope;
@@ -61,6 +62,7 @@ struct AttnParams {
 };
 
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s);
+int attn_rows_per_cta(int q_tiles);  // query rows one CTA covers
 cudaError_t launch_split_combine(const float* part_o, const float* part_ml, __nv_bfloat16* o,
                                  long long o_st, long long o_sb, int n_splits, int B, int H,
                                  int Nq, int Nq_pad, cudaStream_t s);

@@ -209,11 +209,17 @@ struct CrossPlan {
   size_t part_o_bytes, part_ml_bytes;
 };
 
+// Split of the video keys for the audio-query direction: enough splits that
+// the (few) audio query tiles x heads x batch fill two waves of the B200's 148
+// SMs, each split a whole number of 128-key tiles.
+constexpr int kCrossTargetCtas = 2 * 148;
+
 CrossPlan plan_cross(const mmdit_tensor_desc* v, const mmdit_tensor_desc* a) {
   CrossPlan p{};
   p.n_qtiles_a = (a->n_tokens + 255) / 256;
   const int tiles = (v->n_tokens + 127) / 128;
-  p.splits = std::max(1, (tiles + 31) / 32);
+  const int base = p.n_qtiles_a * a->heads * a->batch;
+  p.splits = std::max(1, std::min(tiles, (kCrossTargetCtas + base / 2) / base));
   p.kv_per_split = ((tiles + p.splits - 1) / p.splits) * 128;
   p.splits = std::max(1, (v->n_tokens + p.kv_per_split - 1) / p.kv_per_split);
   p.nq_pad = p.n_qtiles_a * 256;
@@ -406,9 +412,10 @@ int mmdit_av_cross_attn(const void* qv, const void* kv, const void* vv, const vo
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(MMDIT_EINVAL, "av_cross: workspace must be 256-byte aligned");
   if ((rc = check_sm100())) return rc;
-  AttnParams p{};
-  // problem 0: audio queries over the video keys, split across CTAs
-  AttnProblem& a2v = p.prob[0];
+  // audio queries over the video keys: 2 Q tiles per CTA, keys split across
+  // CTAs, unnormalised partials merged by the combine kernel
+  AttnParams pa{};
+  AttnProblem& a2v = pa.prob[0];
   if ((rc = make_map(&a2v.tmQ, qa, *audio, audio->n_tokens, "qa")) ||
       (rc = make_map(&a2v.tmK, kv, *video, video->n_tokens, "kv")) ||
       (rc = make_map(&a2v.tmV, vv, *video, video->n_tokens, "vv")))
@@ -425,8 +432,15 @@ int mmdit_av_cross_attn(const void* qv, const void* kv, const void* vv, const vo
   a2v.kv_per_split = c.kv_per_split;
   a2v.ctas = a2v.n_qtiles * a2v.n_splits * a2v.H * a2v.B;
   a2v.mode = kModeDense;
-  // problem 1: video queries over the audio keys
-  AttnProblem& v2a = p.prob[1];
+  pa.n_prob = 1;
+  pa.q_tiles = 2;
+  pa.scale_log2 = scale * 1.4426950408889634f;
+  pa.err = device_error_flag();
+  if (pa.err == nullptr) return fail(MMDIT_ECUDA, "device error flag unavailable");
+  // video queries over the (short) audio keys: 1 Q tile per CTA, two CTAs per
+  // SM hide each other's load and epilogue latency
+  AttnParams pv{};
+  AttnProblem& v2a = pv.prob[0];
   if ((rc = make_map(&v2a.tmQ, qv, *video, video->n_tokens, "qv")) ||
       (rc = make_map(&v2a.tmK, ka, *audio, audio->n_tokens, "ka")) ||
       (rc = make_map(&v2a.tmV, va, *audio, audio->n_tokens, "va")))
@@ -438,16 +452,17 @@ int mmdit_av_cross_attn(const void* qv, const void* kv, const void* vv, const vo
   v2a.Nkv = audio->n_tokens;
   v2a.H = video->heads;
   v2a.B = video->batch;
-  v2a.n_qtiles = (video->n_tokens + 255) / 256;
+  v2a.n_qtiles = (video->n_tokens + 127) / 128;
   v2a.n_splits = 1;
   v2a.kv_per_split = ((audio->n_tokens + 127) / 128) * 128;
   v2a.ctas = v2a.n_qtiles * v2a.H * v2a.B;
   v2a.mode = kModeDense;
-  p.n_prob = 2;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.err = device_error_flag();
-  if (p.err == nullptr) return fail(MMDIT_ECUDA, "device error flag unavailable");
-  cudaError_t e = launch_attn_tc(p, s);
+  pv.n_prob = 1;
+  pv.q_tiles = 1;
+  pv.scale_log2 = pa.scale_log2;
+  pv.err = pa.err;
+  cudaError_t e = launch_attn_tc(pa, s);
+  if (e == cudaSuccess) e = launch_attn_tc(pv, s);
   if (e == cudaSuccess)
     e = launch_split_combine(a2v.part_o, a2v.part_ml, (__nv_bfloat16*)o_audio, audio->stride_tok,
                              audio->stride_batch, c.splits, audio->batch, audio->heads,
