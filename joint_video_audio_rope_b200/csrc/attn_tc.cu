@@ -49,7 +49,11 @@ constexpr int kBoxBytes = 64 * 128;       // one TMA box: 64 rows x 64 channels
 // each other's load and epilogue latency (used for short key sequences).
 template <int QT, int ST>
 struct Cfg {
-  static constexpr int kThreads = 32 * (4 * QT + 2);
+  // QT softmax warpgroups + one warpgroup holding the TMA producer warp, the
+  // MMA warp and two idle warps: the register file is handed out per
+  // warpgroup, so the CTA is a whole number of them and setmaxnreg moves
+  // registers from the producer/MMA warpgroup to the softmax warpgroups.
+  static constexpr int kThreads = 128 * (QT + 1);
   static constexpr int kProducerWarp = 4 * QT;
   static constexpr int kMmaWarp = 4 * QT + 1;
   static constexpr int kStages = ST;
@@ -57,9 +61,22 @@ struct Cfg {
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = QT * kTileBytes;
   static constexpr int kBarOff = kKVOff + ST * kTileBytes;
-  static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + barriers + alignment slack
+  // epilogue staging: per softmax warp 32 rows x kStageCols bf16 channels,
+  // so O leaves as row-contiguous stores instead of one row per lane
+  static constexpr int kStageCols = QT == 2 ? 64 : 32;
+  static constexpr int kStageWarpBytes = 32 * kStageCols * 2;
+  static constexpr int kStageOff = kBarOff + 256;
+  static constexpr int kSmemBytes = kStageOff + 4 * QT * kStageWarpBytes + 1024;  // + align slack
   static constexpr int kTmemCols = 256 * QT;               // S_t and O_t per tile
   static constexpr int kMinBlocks = QT == 1 ? 2 : 1;
+  // Registers per thread: at launch 65,536 / (threads x CTAs per SM), rounded
+  // down to 8; then the producer/MMA warpgroup drops to kRegsLow and the
+  // softmax warpgroups rise to kRegsHigh, keeping
+  // 128 * (QT * kRegsHigh + kRegsLow) <= kThreads * kRegsLaunch.
+  static constexpr int kRegsLaunch = (65536 / (kThreads * kMinBlocks)) / 8 * 8;
+  static constexpr int kRegsLow = QT == 2 ? 104 : 56;
+  static constexpr int kRegsHigh = ((kThreads * kRegsLaunch / 128 - kRegsLow) / QT) / 8 * 8;
+  static_assert(128 * (QT * kRegsHigh + kRegsLow) <= kThreads * kRegsLaunch, "register split");
 };
 constexpr float kRescaleLog2 = 8.0f;      // move the max only beyond a factor 2^8
 // 32-column chunks of S whose exponentials run on the FMA pipe (polynomial)
@@ -74,6 +91,8 @@ constexpr float kRescaleLog2 = 8.0f;      // move the max only beyond a factor 2
 constexpr int kPolyChunks = MMDIT_POLY_CHUNKS;
 
 // barrier indices (8 bytes each)
+// Phases: Q, O and their "empty" barriers complete once per work item; S and
+// P once per key tile; the ring barriers once per load.
 enum {
   B_QFULL = 0,    // 2: Q tile landed (TMA)
   B_QREADY = 2,   // 2: Q tile rotated in place (fused RoPE), 128 arrivals
@@ -81,9 +100,11 @@ enum {
   B_KVEMPTY = 8,  // 4: ring slot consumed (tcgen05.commit)
   B_SFULL = 12,   // 2: S tile ready in TMEM
   B_PFULL = 14,   // 2: P tile written to TMEM (128 arrivals)
-  B_OFULL = 16,   // 2: last PV of the tile done
-  B_MMADONE = 18, // 1: every MMA of the CTA done (teardown)
-  B_COUNT = 19
+  B_OFULL = 16,   // 2: last PV of the item done (O ready for the epilogue)
+  B_QEMPTY = 18,  // 2: last QK of the item done (Q buffer reusable)
+  B_OEMPTY = 20,  // 2: epilogue has read O out of TMEM (128 arrivals)
+  B_MMADONE = 22, // 1: every MMA of the CTA done (teardown)
+  B_COUNT = 23
 };
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0, 0);  // Q, K: K-major
@@ -99,9 +120,21 @@ struct Work {
   int g_first, g_nblk;
 };
 
-__device__ __forceinline__ Work decode_work(const AttnParams& P, int rows) {
+__device__ __forceinline__ int total_items(const AttnParams& P) {
+  return P.prob[0].ctas + (P.n_prob > 1 ? P.prob[1].ctas : 0);
+}
+
+// k-th work item of this CTA: the CTA's own item, or (persistent launches)
+// items blockIdx.x + k * gridDim.x.
+template <bool PERSIST>
+__device__ __forceinline__ int item_of(const AttnParams&, int k, int n_items) {
+  if (!PERSIST) return k == 0 ? (int)blockIdx.x : n_items;
+  return (int)blockIdx.x + k * (int)gridDim.x;
+}
+
+__device__ __forceinline__ Work decode_work(const AttnParams& P, int item, int rows) {
   Work w;
-  int idx = blockIdx.x;
+  int idx = item;
   w.prob = 0;
   if (P.n_prob > 1 && idx >= P.prob[0].ctas) {
     idx -= P.prob[0].ctas;
@@ -212,7 +245,11 @@ __device__ void rope_row_smem(uint8_t* q_tile, int r, int tok, const DevLayout& 
   }
 }
 
-template <int QT, int ST>
+// PERSIST = false: one work item per CTA (grid = items; the loops below run
+// once, so no cross-item state is live).  PERSIST = true: each CTA walks items
+// blockIdx.x, blockIdx.x + gridDim.x, ... keeping TMEM and barriers alive, and
+// the next item's Q load and QK overlap the current item's epilogue.
+template <int QT, int ST, bool PERSIST>
 __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks)
     attn_tc_kernel(const __grid_constant__ AttnParams P) {
   using C = Cfg<QT, ST>;
@@ -229,8 +266,7 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + 8 * B_COUNT);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const Work w = decode_work(P, C::kRows);
-  const AttnProblem& pr = P.prob[w.prob];
+  const int n_items = PERSIST ? total_items(P) : (int)blockIdx.x + 1;
   int* err = P.err;
   const bool skip = *(volatile int*)err != 0;  // an earlier kernel timed out
 
@@ -241,6 +277,8 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
       mbar_init(bar(B_SFULL + t), 1);
       mbar_init(bar(B_PFULL + t), 128);
       mbar_init(bar(B_OFULL + t), 1);
+      mbar_init(bar(B_QEMPTY + t), 1);
+      mbar_init(bar(B_OEMPTY + t), 128);
     }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar(B_KVFULL + s), 1);
@@ -257,45 +295,54 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int nkv = skip ? 0 : w.nkv;
 
+  if (warp >= 4 * QT) {
+    // producer / MMA warpgroup: give registers to the softmax warpgroups
+    setmaxnreg_dec<C::kRegsLow>();
   if (warp == C::kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && !skip) {
-      tma_prefetch_desc(&pr.tmQ);
-      tma_prefetch_desc(&pr.tmK);
-      tma_prefetch_desc(&pr.tmV);
-      for (int t = 0; t < QT; ++t) {
-        mbar_expect_tx(bar(B_QFULL + t), kTileBytes);
-        const int s0 = w.q0 + t * 128;
-        tma_tile(sbase + kQOff + t * kTileBytes, &pr.tmQ, bar(B_QFULL + t), w.h, w.b, s0,
-                 s0 + 64);
-      }
       int last[kStages];
 #pragma unroll
       for (int i = 0; i < kStages; ++i) last[i] = -1;
       bool ok = true;
-      const int ucount = pr.mode == kModeSparse
-                             ? pr.ucnt[((long long)w.b * pr.H + w.h) * pr.n_qtiles + w.qtile]
-                             : 0;
-      for (int j = 0; j < nkv && ok; ++j) {
-        int s0, s1;
-        kv_tile(pr, w, j, ucount, s0, s1);
-        for (int kind = 0; kind < 2; ++kind) {
-          const int i = 2 * j + kind;
-          const int slot = i % kStages;
-          if (!mbar_wait(bar(B_KVEMPTY + slot), ((i / kStages) & 1) ^ 1, err)) {
-            ok = false;
-            break;
+      int ld = 0;  // ring loads issued so far (all items)
+      int it = 0;  // items of this CTA so far
+      for (int item = item_of<PERSIST>(P, 0, n_items); item < n_items && ok;
+           item = item_of<PERSIST>(P, ++it, n_items)) {
+        const Work w = decode_work(P, item, C::kRows);
+        const AttnProblem& pr = P.prob[w.prob];
+        if (it == 0) {
+          tma_prefetch_desc(&pr.tmQ);
+          tma_prefetch_desc(&pr.tmK);
+          tma_prefetch_desc(&pr.tmV);
+        }
+        for (int t = 0; t < QT && ok; ++t) {
+          if (it > 0 && !(ok = mbar_wait(bar(B_QEMPTY + t), (it - 1) & 1, err))) break;
+          mbar_expect_tx(bar(B_QFULL + t), kTileBytes);
+          const int s0 = w.q0 + t * 128;
+          tma_tile(sbase + kQOff + t * kTileBytes, &pr.tmQ, bar(B_QFULL + t), w.h, w.b, s0,
+                   s0 + 64);
+        }
+        const int ucount = pr.mode == kModeSparse
+                               ? pr.ucnt[((long long)w.b * pr.H + w.h) * pr.n_qtiles + w.qtile]
+                               : 0;
+        for (int j = 0; j < w.nkv && ok; ++j) {
+          int s0, s1;
+          kv_tile(pr, w, j, ucount, s0, s1);
+          for (int kind = 0; kind < 2; ++kind, ++ld) {
+            const int slot = ld % kStages;
+            if (!(ok = mbar_wait(bar(B_KVEMPTY + slot), ((ld / kStages) & 1) ^ 1, err))) break;
+            mbar_expect_tx(bar(B_KVFULL + slot), kTileBytes);
+            tma_tile(sbase + kKVOff + slot * kTileBytes, kind ? &pr.tmV : &pr.tmK,
+                     bar(B_KVFULL + slot), w.h, w.b, s0, s1);
+            last[slot] = ld;
           }
-          mbar_expect_tx(bar(B_KVFULL + slot), kTileBytes);
-          tma_tile(sbase + kKVOff + slot * kTileBytes, kind ? &pr.tmV : &pr.tmK,
-                   bar(B_KVFULL + slot), w.h, w.b, s0, s1);
-          last[slot] = i;
         }
       }
       // every copy issued must land before the CTA's shared memory goes away
-      for (int t = 0; t < QT; ++t) mbar_wait(bar(B_QFULL + t), 0, err);
+      if (it > 0)
+        for (int t = 0; t < QT; ++t) mbar_wait(bar(B_QFULL + t), (it - 1) & 1, err);
       for (int s = 0; s < kStages; ++s)
         if (last[s] >= 0) mbar_wait(bar(B_KVFULL + s), (last[s] / kStages) & 1, err);
     }
@@ -304,206 +351,238 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
     // Issue order per key tile j (t = Q tiles of the CTA):
     //   PV_t(j) then QK_t(j+1), tile after tile, so that P_t (which aliases S_t
     //   in TMEM) is consumed by PV_t before QK_t(j+1) overwrites S_t, and the
-    //   completion of QK_t(j+1) also implies PV_t(j) is done.
+    //   completion of QK_t(j+1) also implies PV_t(j) is done.  Across items the
+    //   first PV_t of an item waits until the epilogue has read O_t out.
     if (lane == 0 && !skip) {
       bool ok = true;
-      const int qbar = pr.rope_q ? B_QREADY : B_QFULL;
-      for (int t = 0; t < QT && ok; ++t) ok = mbar_wait(bar(qbar + t), 0, err);
-      if (ok && nkv > 0) {
-        // prologue: S_t = Q_t K_0^T for every tile
-        ok = mbar_wait(bar(B_KVFULL + 0), 0, err);
-        if (ok) {
+      int cs = 0;   // ring loads consumed so far (all items)
+      int pt = 0;   // key tiles processed so far (P barrier phases)
+      int it = 0;
+      for (int item = item_of<PERSIST>(P, 0, n_items); item < n_items && ok;
+           item = item_of<PERSIST>(P, ++it, n_items)) {
+        const Work w = decode_work(P, item, C::kRows);
+        const AttnProblem& pr = P.prob[w.prob];
+        const int nkv = w.nkv;
+        const int qbar = pr.rope_q ? B_QREADY : B_QFULL;
+        for (int t = 0; t < QT && ok; ++t) ok = mbar_wait(bar(qbar + t), it & 1, err);
+        if (!ok) break;
+        auto k_slot = [&](int j) { return (cs + 2 * j) % kStages; };
+        auto v_slot = [&](int j) { return (cs + 2 * j + 1) % kStages; };
+        auto ring_parity = [&](int i) { return ((cs + i) / kStages) & 1; };
+        if (nkv > 0) {
+          // prologue: S_t = Q_t K_0^T for every tile
+          const int s_k0 = k_slot(0);
+          if (!(ok = mbar_wait(bar(B_KVFULL + s_k0), ring_parity(0), err))) break;
           tc_fence_after();
 #pragma unroll
           for (int t = 0; t < QT; ++t) {
-            mma_qk(tmem + t * 128, sbase + kQOff + t * kTileBytes, sbase + kKVOff);
+            mma_qk(tmem + t * 128, sbase + kQOff + t * kTileBytes, sbase + kKVOff + s_k0 * kTileBytes);
             tc_commit(bar(B_SFULL + t));
+            if (nkv == 1) tc_commit(bar(B_QEMPTY + t));
           }
-          tc_commit(bar(B_KVEMPTY + 0));
-        }
-        for (int j = 0; j < nkv && ok; ++j) {
-          const int iv = 2 * j + 1, ik = 2 * j + 2;
-          const int sv = iv % kStages, sk = ik % kStages;
-          const uint32_t v_smem = sbase + kKVOff + sv * kTileBytes;
-          const uint32_t k_smem = sbase + kKVOff + sk * kTileBytes;
-          const bool more = j + 1 < nkv;
-          if (!(ok = mbar_wait(bar(B_KVFULL + sv), (iv / kStages) & 1, err))) break;
+          tc_commit(bar(B_KVEMPTY + s_k0));
+          for (int j = 0; j < nkv && ok; ++j) {
+            const int sv = v_slot(j), sk = k_slot(j + 1);
+            const uint32_t v_smem = sbase + kKVOff + sv * kTileBytes;
+            const uint32_t k_smem = sbase + kKVOff + sk * kTileBytes;
+            const bool more = j + 1 < nkv;
+            if (!(ok = mbar_wait(bar(B_KVFULL + sv), ring_parity(2 * j + 1), err))) break;
 #pragma unroll
-          for (int t = 0; t < QT; ++t) {
-            if (!(ok = mbar_wait(bar(B_PFULL + t), j & 1, err))) break;
-            tc_fence_after();
-            mma_pv(tmem + QT * 128 + t * 128, tmem + t * 128, v_smem, j > 0);
-            if (t == QT - 1) tc_commit(bar(B_KVEMPTY + sv));
-            if (more) {
-              if (t == 0) {
-                if (!(ok = mbar_wait(bar(B_KVFULL + sk), (ik / kStages) & 1, err))) break;
-                tc_fence_after();
+            for (int t = 0; t < QT; ++t) {
+              if (!(ok = mbar_wait(bar(B_PFULL + t), (pt + j) & 1, err))) break;
+              if (j == 0 && it > 0 && !(ok = mbar_wait(bar(B_OEMPTY + t), (it - 1) & 1, err)))
+                break;
+              tc_fence_after();
+              mma_pv(tmem + QT * 128 + t * 128, tmem + t * 128, v_smem, j > 0);
+              if (t == QT - 1) tc_commit(bar(B_KVEMPTY + sv));
+              if (more) {
+                if (t == 0) {
+                  if (!(ok = mbar_wait(bar(B_KVFULL + sk), ring_parity(2 * j + 2), err))) break;
+                  tc_fence_after();
+                }
+                mma_qk(tmem + t * 128, sbase + kQOff + t * kTileBytes, k_smem);
+                tc_commit(bar(B_SFULL + t));
+                if (j + 2 == nkv) tc_commit(bar(B_QEMPTY + t));
+                if (t == QT - 1) tc_commit(bar(B_KVEMPTY + sk));
               }
-              mma_qk(tmem + t * 128, sbase + kQOff + t * kTileBytes, k_smem);
-              tc_commit(bar(B_SFULL + t));
-              if (t == QT - 1) tc_commit(bar(B_KVEMPTY + sk));
             }
           }
+          cs += 2 * nkv;
+          pt += nkv;
+        } else {
+          for (int t = 0; t < QT; ++t) {
+            if (it > 0 && !(ok = mbar_wait(bar(B_OEMPTY + t), (it - 1) & 1, err))) break;
+            tc_commit(bar(B_QEMPTY + t));
+          }
         }
+        for (int t = 0; t < QT; ++t) tc_commit(bar(B_OFULL + t));
       }
-      for (int t = 0; t < QT; ++t) tc_commit(bar(B_OFULL + t));
       tc_commit(bar(B_MMADONE));
       mbar_wait(bar(B_MMADONE), 0, err);
     }
+  }  // warps 4*QT+2 and 4*QT+3 have no role
   } else {
     // ------------------------------------------------------------ softmax
+    setmaxnreg_inc<C::kRegsHigh>();
     const int t = warp >> 2;                  // Q tile of this warpgroup
     const int r = (warp & 3) * 32 + lane;     // row inside the tile == TMEM lane
-    const int row = t * 128 + r;              // row inside the CTA
+    const int row = t * 128 + r;              // row inside the CTA's rows
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t s_addr = tmem + lane_off + t * 128;
     const uint32_t o_addr = tmem + lane_off + QT * 128 + t * 128;
     const float sl2 = P.scale_log2;
     const float thresh = kRescaleLog2 / sl2;  // in raw score units
+    const uint64_t sl2x2 = pack_f32x2(sl2, sl2);
     bool ok = !skip;
+    int st = 0;  // S tiles consumed so far (all items)
+    int it = 0;
+    for (int item = item_of<PERSIST>(P, 0, n_items); item < n_items && ok;
+           item = item_of<PERSIST>(P, ++it, n_items)) {
+      const Work w = decode_work(P, item, C::kRows);
+      const AttnProblem& pr = P.prob[w.prob];
+      const int nkv = w.nkv;
 
-    if (ok && pr.rope_q) {
-      ok = mbar_wait(bar(B_QFULL + t), 0, err);
-      if (ok) {
-        rope_row_smem(smem + kQOff + t * kTileBytes, r, w.q0 + row, P.layout, P.rope);
-        fence_proxy_async_smem();
+      if (pr.rope_q) {
+        ok = mbar_wait(bar(B_QFULL + t), it & 1, err);
+        if (ok) {
+          rope_row_smem(smem + kQOff + t * kTileBytes, r, w.q0 + row, P.layout, P.rope);
+          fence_proxy_async_smem();
+        }
+        mbar_arrive(bar(B_QREADY + t));
       }
-      mbar_arrive(bar(B_QREADY + t));
-    }
 
-    // sparse mode: which query block of the group this row belongs to
-    int qb = 0;
-    if (pr.mode == kModeSparse) {
-      int acc = 0;
-      qb = 31;  // rows past the group: member of nothing
-      for (int i = 0; i < w.g_nblk; ++i) {
-        int st, len;
-        block_extent(pr.vT, pr.vH, pr.vW, w.g_first + i, st, len);
-        if (row < acc + len) {
-          qb = i;
+      // sparse mode: which query block of the group this row belongs to
+      int qb = 0;
+      int ucount = 0;
+      if (pr.mode == kModeSparse) {
+        int acc = 0;
+        qb = 31;  // rows past the group: member of nothing
+        for (int i = 0; i < w.g_nblk; ++i) {
+          int bst, blen;
+          block_extent(pr.vT, pr.vH, pr.vW, w.g_first + i, bst, blen);
+          if (row < acc + blen) {
+            qb = i;
+            break;
+          }
+          acc += blen;
+        }
+        ucount = pr.ucnt[((long long)w.b * pr.H + w.h) * pr.n_qtiles + w.qtile];
+      }
+
+      float m_used = -INFINITY, l = 0.f;
+      for (int j = 0; j < nkv; ++j, ++st) {
+        // valid key columns of each 64-row half of this tile for this row
+        // (independent of S, so computed before waiting for it)
+        int len0, len1;
+        if (pr.mode == kModeDense) {
+          const int s0 = w.kv_lo + j * 128;
+          len0 = max(0, min(64, w.kv_hi - s0));
+          len1 = max(0, min(64, w.kv_hi - s0 - 64));
+        } else {
+          const uint2 e0 = pr.ulist[w.ubase + 2 * j];
+          const uint2 e1 = (2 * j + 1 < ucount) ? pr.ulist[w.ubase + 2 * j + 1] : make_uint2(0u, 0u);
+          len0 = ((e0.y >> 16) >> qb) & 1u ? (int)(e0.y & 0xFFu) : 0;
+          len1 = ((e1.y >> 16) >> qb) & 1u ? (int)(e1.y & 0xFFu) : 0;
+        }
+        ok = ok && mbar_wait(bar(B_SFULL + t), st & 1, err);
+        if (__any_sync(0xffffffffu, !ok)) {
+          ok = false;
           break;
         }
-        acc += len;
+        __syncwarp();
+        tc_fence_after();
+        float s[128];
+        {
+          uint32_t v0[32], v1[32], v2[32], v3[32];
+          tmem_ld32(s_addr, v0);
+          tmem_ld32(s_addr + 32, v1);
+          tmem_ld32(s_addr + 64, v2);
+          tmem_ld32(s_addr + 96, v3);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            s[i] = __uint_as_float(v0[i]);
+            s[32 + i] = __uint_as_float(v1[i]);
+            s[64 + i] = __uint_as_float(v2[i]);
+            s[96 + i] = __uint_as_float(v3[i]);
+          }
+        }
+        const bool masked = len0 < 64 || len1 < 64;
+        if (masked) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            if (c >= len0) s[c] = -INFINITY;
+            if (c >= len1) s[64 + c] = -INFINITY;
+          }
+        }
+        const float mt = row_max128(s);
+        const bool grow = mt > m_used + thresh || (m_used == -INFINITY && mt > -INFINITY);
+        float alpha = 1.f;
+        if (grow) {
+          alpha = (m_used == -INFINITY) ? 0.f : ex2_approx((m_used - mt) * sl2);
+          m_used = mt;
+          l *= alpha;
+        }
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+          // rescale the running O of this row (previous PV is complete: it was
+          // issued before the QK whose completion released this S tile)
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t v[32];
+            tmem_ld32(o_addr + c * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+            tmem_st32(o_addr + c * 32, v);
+          }
+          tmem_wait_st();
+        }
+        const float mref = (m_used == -INFINITY) ? 0.f : m_used * sl2;
+        const uint64_t nm2 = pack_f32x2(-mref, -mref);
+        // Exponentials: MUFU ex2 for most columns; on tiles without masked
+        // columns, the columns of kPolyChunks go to the FMA pipe instead.
+        const bool poly_ok = !__any_sync(0xffffffffu, masked);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+          const bool poly = poly_ok && ((kPolyChunks >> c) & 1);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const uint64_t x2 = ffma_f32x2(pack_f32x2(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]),
+                                           sl2x2, nm2);
+            float p0, p1;
+            if (poly) {
+              exp2_poly_f32x2(x2, p0, p1);
+            } else {
+              float x0, x1;
+              unpack_f32x2(x2, x0, x1);
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+            pk[i] = pack_bf16x2(p0, p1);
+            acc[i & 3] = add_f32x2(acc[i & 3], pack_f32x2(p0, p1));
+          }
+          tmem_st16(s_addr + c * 16, pk);  // P: 2 bf16 per column
+        }
+        tmem_wait_st();
+        {
+          float a0, a1, b0, b1;
+          unpack_f32x2(add_f32x2(acc[0], acc[1]), a0, a1);
+          unpack_f32x2(add_f32x2(acc[2], acc[3]), b0, b1);
+          l += (a0 + a1) + (b0 + b1);
+        }
+        tc_fence_before();
+        mbar_arrive(bar(B_PFULL + t));
       }
-    }
 
-    float m_used = -INFINITY, l = 0.f;
-    const uint64_t sl2x2 = pack_f32x2(sl2, sl2);
-    int ucount = 0;
-    if (pr.mode == kModeSparse)
-      ucount = pr.ucnt[((long long)w.b * pr.H + w.h) * pr.n_qtiles + w.qtile];
-    for (int j = 0; j < nkv; ++j) {
-      // valid key columns of each 64-row half of this tile for this row
-      // (independent of S, so computed before waiting for it)
-      int len0, len1;
-      if (pr.mode == kModeDense) {
-        const int s0 = w.kv_lo + j * 128;
-        len0 = max(0, min(64, w.kv_hi - s0));
-        len1 = max(0, min(64, w.kv_hi - s0 - 64));
-      } else {
-        const uint2 e0 = pr.ulist[w.ubase + 2 * j];
-        const uint2 e1 = (2 * j + 1 < ucount) ? pr.ulist[w.ubase + 2 * j + 1] : make_uint2(0u, 0u);
-        len0 = ((e0.y >> 16) >> qb) & 1u ? (int)(e0.y & 0xFFu) : 0;
-        len1 = ((e1.y >> 16) >> qb) & 1u ? (int)(e1.y & 0xFFu) : 0;
-      }
-      ok = ok && mbar_wait(bar(B_SFULL + t), j & 1, err);
+      // ---------------------------------------------------------- epilogue
+      ok = ok && mbar_wait(bar(B_OFULL + t), it & 1, err);
       if (__any_sync(0xffffffffu, !ok)) {
         ok = false;
         break;
       }
       __syncwarp();
-      tc_fence_after();
-      float s[128];
-      {
-        uint32_t v0[32], v1[32], v2[32], v3[32];
-        tmem_ld32(s_addr, v0);
-        tmem_ld32(s_addr + 32, v1);
-        tmem_ld32(s_addr + 64, v2);
-        tmem_ld32(s_addr + 96, v3);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          s[i] = __uint_as_float(v0[i]);
-          s[32 + i] = __uint_as_float(v1[i]);
-          s[64 + i] = __uint_as_float(v2[i]);
-          s[96 + i] = __uint_as_float(v3[i]);
-        }
-      }
-      const bool masked = len0 < 64 || len1 < 64;
-      if (masked) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          if (c >= len0) s[c] = -INFINITY;
-          if (c >= len1) s[64 + c] = -INFINITY;
-        }
-      }
-      const float mt = row_max128(s);
-      const bool grow = mt > m_used + thresh || (m_used == -INFINITY && mt > -INFINITY);
-      float alpha = 1.f;
-      if (grow) {
-        alpha = (m_used == -INFINITY) ? 0.f : ex2_approx((m_used - mt) * sl2);
-        m_used = mt;
-        l *= alpha;
-      }
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        // rescale the running O of this row (previous PV is complete: it was
-        // issued before the QK whose completion released this S tile)
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          tmem_ld32(o_addr + c * 32, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-          tmem_st32(o_addr + c * 32, v);
-        }
-        tmem_wait_st();
-      }
-      const float mref = (m_used == -INFINITY) ? 0.f : m_used * sl2;
-      const uint64_t nm2 = pack_f32x2(-mref, -mref);
-      // Exponentials: MUFU ex2 for most columns; on tiles without masked
-      // columns, the columns of kPolyChunks go to the FMA pipe instead.
-      const bool poly_ok = !__any_sync(0xffffffffu, masked);
-      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
-        const bool poly = poly_ok && ((kPolyChunks >> c) & 1);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const uint64_t x2 = ffma_f32x2(pack_f32x2(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]),
-                                         sl2x2, nm2);
-          float p0, p1;
-          if (poly) {
-            exp2_poly_f32x2(x2, p0, p1);
-          } else {
-            float x0, x1;
-            unpack_f32x2(x2, x0, x1);
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
-          }
-          pk[i] = pack_bf16x2(p0, p1);
-          acc[i & 3] = add_f32x2(acc[i & 3], pack_f32x2(p0, p1));
-        }
-        tmem_st16(s_addr + c * 16, pk);  // P: 2 bf16 per column
-      }
-      tmem_wait_st();
-      {
-        float a0, a1, b0, b1, c0, c1, d0, d1;
-        unpack_f32x2(add_f32x2(acc[0], acc[1]), a0, a1);
-        unpack_f32x2(add_f32x2(acc[2], acc[3]), b0, b1);
-        (void)c0; (void)c1; (void)d0; (void)d1;
-        l += (a0 + a1) + (b0 + b1);
-      }
-      tc_fence_before();
-      mbar_arrive(bar(B_PFULL + t));
-    }
-
-    // ------------------------------------------------------------ epilogue
-    if (ok && nkv > 0) ok = mbar_wait(bar(B_OFULL + t), 0, err);
-    const bool all_ok = !__any_sync(0xffffffffu, !ok);
-    __syncwarp();
-    if (all_ok && !skip) {
       tc_fence_after();
       const bool valid_row = row < w.q_valid;
       const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -537,19 +616,26 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
           pr.part_ml[prow * 2 + 1] = l;
         }
       } else {
-        __nv_bfloat16* dst = pr.o + (long long)w.b * pr.o_sb + (long long)qrow * pr.o_st +
-                             (long long)w.h * 128;
+        // normalised bf16 O: each round stages kStageCols channels of the
+        // warp's 32 rows in shared memory (16-byte chunks XOR-swizzled by row,
+        // conflict-free both ways), then writes them back so that 8 lanes
+        // cover one row's contiguous bytes
+        constexpr int SC = C::kStageCols;
+        constexpr int CH = SC / 8;  // 16-byte chunks per staged row
+        uint8_t* stage = smem + C::kStageOff + warp * C::kStageWarpBytes;
+        const int wrow0 = (warp & 3) * 32;  // first row of this warp inside the tile
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          if (nkv > 0) {
-            tmem_ld32(o_addr + c * 32, v);
-            tmem_wait_ld();
-          } else {
+        for (int r = 0; r < 128 / SC; ++r) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0u;
-          }
-          if (valid_row) {
+          for (int c = 0; c < SC / 32; ++c) {
+            uint32_t v[32];
+            if (nkv > 0) {
+              tmem_ld32(o_addr + r * SC + c * 32, v);
+              tmem_wait_ld();
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] = 0u;
+            }
 #pragma unroll
             for (int i = 0; i < 32; i += 8) {
               uint4 pk;
@@ -557,9 +643,26 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
               pk.y = pack_bf16x2(__uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv);
               pk.z = pack_bf16x2(__uint_as_float(v[i + 4]) * inv, __uint_as_float(v[i + 5]) * inv);
               pk.w = pack_bf16x2(__uint_as_float(v[i + 6]) * inv, __uint_as_float(v[i + 7]) * inv);
-              *reinterpret_cast<uint4*>(dst + c * 32 + i) = pk;
+              const int chunk = c * 4 + i / 8;
+              *reinterpret_cast<uint4*>(stage + lane * (SC * 2) + ((chunk ^ (lane % CH)) << 4)) = pk;
             }
           }
+          __syncwarp();
+          constexpr int RPI = 32 / CH;  // rows per store instruction
+#pragma unroll
+          for (int i = 0; i < 32 / RPI; ++i) {
+            const int srow = i * RPI + lane / CH, chunk = lane % CH;
+            const uint4 pk = *reinterpret_cast<const uint4*>(stage + srow * (SC * 2) +
+                                                             ((chunk ^ (srow % CH)) << 4));
+            const int trow = t * 128 + wrow0 + srow;  // row inside the CTA
+            if (trow < w.q_valid) {
+              __nv_bfloat16* dst = pr.o + (long long)w.b * pr.o_sb +
+                                   (long long)(w.q0 + trow) * pr.o_st + (long long)w.h * 128 +
+                                   r * SC + chunk * 8;
+              *reinterpret_cast<uint4*>(dst) = pk;
+            }
+          }
+          __syncwarp();
         }
         if (pr.lse != nullptr && valid_row) {
           const float mref = (m_used == -INFINITY) ? 0.f : m_used * sl2;
@@ -567,6 +670,9 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
               l > 0.f ? (mref + log2f(l)) * 0.69314718055994531f : -INFINITY;
         }
       }
+      // O has been read out of TMEM: the next item's first PV may overwrite it
+      tc_fence_before();
+      mbar_arrive(bar(B_OEMPTY + t));
     }
   }
 
@@ -608,19 +714,28 @@ __global__ void split_combine_kernel(const float* __restrict__ part_o,
       __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
 }
 
-template <int QT, int ST>
+template <int QT, int ST, bool PERSIST>
 cudaError_t launch_shape(const AttnParams& p, cudaStream_t s) {
   using C = Cfg<QT, ST>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<QT, ST>,
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<QT, ST, PERSIST>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const int ctas = p.prob[0].ctas + (p.n_prob > 1 ? p.prob[1].ctas : 0);
-  if (ctas == 0) return cudaSuccess;
-  attn_tc_kernel<QT, ST><<<ctas, C::kThreads, C::kSmemBytes, s>>>(p);
+  const int items = p.prob[0].ctas + (p.n_prob > 1 ? p.prob[1].ctas : 0);
+  if (items == 0) return cudaSuccess;
+  int grid = items;
+  if (PERSIST) {
+    // one CTA per resident slot; each CTA walks items blockIdx.x + k*gridDim.x
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    grid = std::min(items, sms * C::kMinBlocks);
+  }
+  attn_tc_kernel<QT, ST, PERSIST><<<grid, C::kThreads, C::kSmemBytes, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -629,8 +744,9 @@ cudaError_t launch_shape(const AttnParams& p, cudaStream_t s) {
 int attn_rows_per_cta(int q_tiles) { return 128 * q_tiles; }
 
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
-  if (p.q_tiles == 1) return launch_shape<1, 2>(p, s);
-  return launch_shape<2, 4>(p, s);
+  if (p.q_tiles == 1)
+    return p.persistent ? launch_shape<1, 2, true>(p, s) : launch_shape<1, 2, false>(p, s);
+  return p.persistent ? launch_shape<2, 4, true>(p, s) : launch_shape<2, 4, false>(p, s);
 }
 
 cudaError_t launch_split_combine(const float* part_o, const float* part_ml, __nv_bfloat16* o,

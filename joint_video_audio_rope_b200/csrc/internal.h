@@ -40,7 +40,7 @@ struct AttnProblem {
   int n_qtiles;               // ceil(Nq / 256) (dense) or number of groups (sparse)
   int n_splits;               // KV splits per (q tile pair, head, batch)
   int kv_per_split;           // tokens per split, multiple of 128
-  int ctas;                   // n_qtiles * H * B * n_splits
+  int ctas;                   // work items: n_qtiles * H * B * n_splits
   int mode;                   // AttnMode
   // sparse mode: the query groups and the merged key-block lists
   const int4* groups;         // per group: {first block, n blocks, start token, n tokens}
@@ -55,6 +55,7 @@ struct AttnParams {
   AttnProblem prob[2];
   int n_prob;
   int q_tiles;                // 128-row Q tiles per CTA: 2 (default) or 1
+  int persistent;             // 0: one CTA per work item; 1: one CTA per SM slot, looping
   float scale_log2;           // softmax scale * log2(e)
   DevLayout layout;           // for fused Q RoPE
   RopeTab rope;

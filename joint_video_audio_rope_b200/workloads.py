@@ -118,6 +118,12 @@ WORKLOADS: Dict[str, Workload] = {
         "1080p_sparse", [video(21, 68, 120, order=ORDER_BLOCK444), audio(218)],
         batch=1, heads=24, head_dim=128, dtype="bf16", seed=4,
         qk_std=1.0, v_std=1.0, planted_regions=8, planted_amp=2.0, sparse=True),
+    # a quarter of the 1080p grid (17 x 30 -> 17 x 15 blocks per frame slab):
+    # the same structure at a size an ncu capture can hold (~2 GB on device)
+    "1080p_sparse_quarter": Workload(
+        "1080p_sparse_quarter", [video(21, 34, 60, order=ORDER_BLOCK444), audio(218)],
+        batch=1, heads=24, head_dim=128, dtype="bf16", seed=5,
+        qk_std=1.0, v_std=1.0, planted_regions=8, planted_amp=2.0, sparse=True),
 }
 
 
