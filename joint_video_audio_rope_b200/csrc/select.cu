@@ -5,16 +5,18 @@
 // S_i = TopK(P_i, k) U TopP(P_i, p).
 //
 // Kernels:
-//   pool_kernel    one CTA per (block, batch): coalesced 128-bit reads of the
-//                  block's <= 64 tokens of Q and K, fp32 sums, mean over the
-//                  block's real tokens.  HBM-bound: Q and K are read once.
+//   pool_kernel    one CTA per (block, batch): each thread sums 8 channels
+//                  (one 16-byte vector) of Q and K over the block's <= 64
+//                  tokens in fp32 and divides by the real token count.
+//                  HBM-bound: Q and K are read once.
 //   select_kernel  one CTA per (8 query blocks, head, batch): fp32 block
-//                  scores into shared memory, then one warp per row: fp32
-//                  probabilities, fp64 normaliser and prefix masses, value
-//                  thresholds of the k-th block (count search) and of the
-//                  top-p crossing block (mass search) by bisection on the
-//                  fp32 bit patterns, and an ascending-id compaction with
-//                  warp ballots.  Ranking is P descending, ties by lower id.
+//                  scores into shared memory, then one warp per row with the
+//                  row's probabilities in registers: fp32 probabilities,
+//                  fp64 normaliser and prefix masses, value thresholds of the
+//                  k-th block (count search) and of the top-p crossing block
+//                  (mass search) by bisection on the fp32 bit patterns, and an
+//                  ascending-id compaction with warp ballots.  Ranking is P
+//                  descending, ties by lower id.
 //   groups_kernel  partitions the query blocks into CTA groups of <= 256
 //                  tokens and <= 16 blocks (greedy, in block order).
 //   union_kernel   per (group, head, batch): merges the groups' selected
@@ -38,26 +40,34 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   const int blk = blockIdx.x, b = blockIdx.y;
   int start, len;
   block_extent(T, Hg, Wg, blk, start, len);
-  const int npairs = H * 64;  // bf16 pairs per token row (head_dim 128)
+  const int nvec = H * 16;  // 16-byte vectors (8 channels) per token row (head_dim 128)
   const float inv = 1.f / (float)len;
-  for (int pidx = threadIdx.x; pidx < npairs; pidx += blockDim.x) {
-    float2 aq = make_float2(0.f, 0.f), ak = make_float2(0.f, 0.f);
-    const long long base = (long long)b * sb + (long long)start * st + 2 * pidx;
-#pragma unroll 4
+  for (int vi = threadIdx.x; vi < nvec; vi += blockDim.x) {
+    float aq[8], ak[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) aq[c] = ak[c] = 0.f;
+    const long long base = (long long)b * sb + (long long)start * st + 8 * vi;
+#pragma unroll 8
     for (int i = 0; i < len; ++i) {
-      const float2 vq = __bfloat1622float2(
-          *reinterpret_cast<const __nv_bfloat162*>(q + base + (long long)i * st));
-      const float2 vk = __bfloat1622float2(
-          *reinterpret_cast<const __nv_bfloat162*>(k + base + (long long)i * st));
-      aq.x += vq.x;
-      aq.y += vq.y;
-      ak.x += vk.x;
-      ak.y += vk.y;
+      const uint4 rq = __ldg(reinterpret_cast<const uint4*>(q + base + (long long)i * st));
+      const uint4 rk = __ldg(reinterpret_cast<const uint4*>(k + base + (long long)i * st));
+      const __nv_bfloat162* pq = reinterpret_cast<const __nv_bfloat162*>(&rq);
+      const __nv_bfloat162* pk = reinterpret_cast<const __nv_bfloat162*>(&rk);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float2 fq = __bfloat1622float2(pq[c]), fk = __bfloat1622float2(pk[c]);
+        aq[2 * c] += fq.x;
+        aq[2 * c + 1] += fq.y;
+        ak[2 * c] += fk.x;
+        ak[2 * c + 1] += fk.y;
+      }
     }
-    const int h = pidx >> 6, d = (pidx & 63) * 2;
+    const int h = vi >> 4, d = (vi & 15) * 8;
     const long long o = (((long long)b * H + h) * nblk + blk) * 128 + d;
-    *reinterpret_cast<float2*>(qbar + o) = make_float2(aq.x * inv, aq.y * inv);
-    *reinterpret_cast<float2*>(kbar + o) = make_float2(ak.x * inv, ak.y * inv);
+    *reinterpret_cast<float4*>(qbar + o) = make_float4(aq[0] * inv, aq[1] * inv, aq[2] * inv, aq[3] * inv);
+    *reinterpret_cast<float4*>(qbar + o + 4) = make_float4(aq[4] * inv, aq[5] * inv, aq[6] * inv, aq[7] * inv);
+    *reinterpret_cast<float4*>(kbar + o) = make_float4(ak[0] * inv, ak[1] * inv, ak[2] * inv, ak[3] * inv);
+    *reinterpret_cast<float4*>(kbar + o + 4) = make_float4(ak[4] * inv, ak[5] * inv, ak[6] * inv, ak[7] * inv);
   }
 }
 
@@ -80,22 +90,38 @@ __device__ __forceinline__ float warp_max_f(float v) {
   return v;
 }
 
-// number of probabilities with bit pattern >= tau
-__device__ __forceinline__ int count_ge(const uint32_t* pb, int n, uint32_t tau, int lane) {
-  int c = 0;
-  for (int j = lane; j < n; j += 32) c += pb[j] >= tau;
-  return warp_sum_i(c);
-}
-// sum (fp64) of probabilities with bit pattern >= tau
-__device__ __forceinline__ double mass_ge(const uint32_t* pb, int n, uint32_t tau, int lane) {
-  double m = 0.0;
-  for (int j = lane; j < n; j += 32) {
-    const uint32_t v = pb[j];
-    if (v >= tau) m += (double)__uint_as_float(v);
-  }
-  return warp_sum_d(m);
-}
+// One warp holds one row of VPL * 32 probabilities in registers: lane l owns
+// blocks l, l + 32, ...; slots past the row hold -1 (a negative bit pattern,
+// below every threshold).  Probabilities are >= 0, so their fp32 bit patterns
+// order like their values and thresholds are searched on the bits.
+template <int VPL>
+struct Row {
+  float v[VPL];
 
+  // number of probabilities with bit pattern >= tau (tau >= 0)
+  __device__ __forceinline__ int count_ge(int tau) const {
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) c += __float_as_int(v[i]) >= tau;
+    return warp_sum_i(c);
+  }
+  // sum of the probabilities with bit pattern >= tau: fp32 over chunks of 8
+  // values (each <= 1, error ~1e-7 of the chunk), fp64 across chunks and lanes
+  __device__ __forceinline__ double mass_ge(int tau) const {
+    double m = 0.0;
+#pragma unroll
+    for (int i0 = 0; i0 < VPL; i0 += 8) {
+      float c = 0.f;
+#pragma unroll
+      for (int i = i0; i < i0 + 8 && i < VPL; ++i)
+        c += __float_as_int(v[i]) >= tau ? v[i] : 0.f;
+      m += (double)c;
+    }
+    return warp_sum_d(m);
+  }
+};
+
+template <int VPL>
 __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ qbar,
                                                      const float* __restrict__ kbar, int H,
                                                      int nblk, int top_k, float top_p, float scale,
@@ -137,59 +163,66 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ q
   }
   __syncthreads();
 
-  // ---- per row selection: one warp per query block
+  // ---- per row selection: one warp per query block, the row in registers
   const int row = r0 + warp;
   if (row >= nblk) return;
-  float* s = sc + warp * nblk;
-  uint32_t* pb = reinterpret_cast<uint32_t*>(s);
   const int n = nblk;
+  const float* srow = sc + warp * nblk;
+  Row<VPL> P;
   float mx = -INFINITY;
-  for (int j = lane; j < n; j += 32) mx = fmaxf(mx, s[j]);
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int j = lane + 32 * i;
+    P.v[i] = j < n ? srow[j] : -INFINITY;
+    mx = fmaxf(mx, P.v[i]);
+  }
   mx = warp_max_f(mx);
   double z = 0.0;
-  for (int j = lane; j < n; j += 32) {
-    const float p = expf(s[j] - mx);  // unnormalised probability in (0, 1]
-    s[j] = p;
-    z += (double)p;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int j = lane + 32 * i;
+    // unnormalised probability in (0, 1]; -1 marks the slots past the row
+    P.v[i] = j < n ? expf(P.v[i] - mx) : -1.f;
+    if (j < n) z += (double)P.v[i];
   }
   z = warp_sum_d(z);
-  __syncwarp();
 
-  const uint32_t kOne = 0x3F800000u;  // bit pattern of 1.0f, the largest value
+  const int kOne = 0x3F800000;  // bit pattern of 1.0f, the largest value
   // top-k threshold: largest tau with count(P >= tau) >= k'
   const int kq = min(max(top_k, 0), n);
-  uint32_t tau_k = kOne + 1;  // nothing selected by top-k when k' == 0
+  int tau_k = kOne + 1;  // nothing selected by top-k when k' == 0
   if (kq > 0) {
-    uint32_t lo = 0, hi = kOne + 1;
+    int lo = 0, hi = kOne + 1;
     while (hi - lo > 1) {
-      const uint32_t mid = lo + ((hi - lo) >> 1);
-      if (count_ge(pb, n, mid, lane) >= kq) lo = mid; else hi = mid;
+      const int mid = lo + ((hi - lo) >> 1);
+      if (P.count_ge(mid) >= kq) lo = mid; else hi = mid;
     }
     tau_k = lo;
   }
   // top-p threshold: largest tau with mass(P >= tau) >= p * Z
   const double target = (double)top_p * z;
-  uint32_t tau_p;
-  int take_p;  // how many blocks top-p selects
+  const double mass_all = P.mass_ge(0);
+  int tau_p;
   if (target <= 0.0) {
     tau_p = kOne;
-  } else if (mass_ge(pb, n, 0u, lane) < target) {
-    tau_p = 0u;  // the sum never reaches p (p >= 1 with rounding): all blocks
+  } else if (mass_all < target) {
+    tau_p = 0;  // the sum never reaches p (p >= 1 with rounding): all blocks
   } else {
-    uint32_t lo = 0, hi = kOne + 1;
+    int lo = 0, hi = kOne + 1;
     while (hi - lo > 1) {
-      const uint32_t mid = lo + ((hi - lo) >> 1);
-      if (mass_ge(pb, n, mid, lane) >= target) lo = mid; else hi = mid;
+      const int mid = lo + ((hi - lo) >> 1);
+      if (P.mass_ge(mid) >= target) lo = mid; else hi = mid;
     }
     tau_p = lo;
   }
+  int take_p;  // how many blocks top-p selects
   {
-    const int c_gt = count_ge(pb, n, tau_p + 1, lane);
-    const int c_eq = count_ge(pb, n, tau_p, lane) - c_gt;
-    const double m_gt = mass_ge(pb, n, tau_p + 1, lane);
-    const double tv = (double)__uint_as_float(tau_p);
+    const int c_gt = P.count_ge(tau_p + 1);
+    const int c_eq = P.count_ge(tau_p) - c_gt;
+    const double m_gt = P.mass_ge(tau_p + 1);
+    const double tv = (double)__int_as_float(tau_p);
     int m = 1;
-    if (tau_p == 0u && target > 0.0 && mass_ge(pb, n, 0u, lane) < target) {
+    if (tau_p == 0 && target > 0.0 && mass_all < target) {
       m = c_eq;  // everything
     } else if (target > m_gt && tv > 0.0) {
       m = (int)ceil((target - m_gt) / tv);
@@ -198,25 +231,25 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ q
     take_p = c_gt + m;
   }
   // final threshold and number of tied blocks to take (lowest ids first)
-  uint32_t tau;
-  int take_eq;
+  int tau, take_eq;
   if (take_p >= kq) {
     tau = tau_p;
-    take_eq = take_p - count_ge(pb, n, tau_p + 1, lane);
+    take_eq = take_p - P.count_ge(tau_p + 1);
   } else {
     tau = tau_k;
-    take_eq = kq - count_ge(pb, n, tau_k + 1, lane);
+    take_eq = kq - P.count_ge(tau_k + 1);
   }
   // ---- ascending compaction
   int32_t* out = idx + (hb + row) * (long long)cap;
   int pos = 0, ties = 0;
-  for (int j0 = 0; j0 < n; j0 += 32) {
-    const int j = j0 + lane;
-    const uint32_t v = j < n ? pb[j] : 0u;
-    const bool eq = j < n && v == tau;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int j = lane + 32 * i;
+    const int vb = __float_as_int(P.v[i]);
+    const bool eq = vb == tau;  // padding (-1) never equals tau >= 0
     const unsigned eqm = __ballot_sync(0xffffffffu, eq);
     const int tie_rank = ties + __popc(eqm & ((1u << lane) - 1u));
-    const bool sel = j < n && (v > tau || (eq && tie_rank < take_eq));
+    const bool sel = vb > tau || (eq && tie_rank < take_eq);
     const unsigned sm_ = __ballot_sync(0xffffffffu, sel);
     if (sel) out[pos + __popc(sm_ & ((1u << lane) - 1u))] = j;
     pos += __popc(sm_);
@@ -311,17 +344,36 @@ cudaError_t launch_pool(const __nv_bfloat16* q, const __nv_bfloat16* k, const mm
   return cudaGetLastError();
 }
 
+template <int VPL>
+cudaError_t launch_select_vpl(const float* qbar, const float* kbar, int B, int H, int nblk,
+                              int top_k, float top_p, float scale, int cap, int32_t* idx,
+                              int32_t* cnt, cudaStream_t s) {
+  const size_t smem = select_smem_bytes(nblk);
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<VPL>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((nblk + kSelRows - 1) / kSelRows, H, B);
+  select_kernel<VPL><<<grid, 256, smem, s>>>(qbar, kbar, H, nblk, top_k, top_p, scale, cap, idx,
+                                             cnt);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_select(const float* qbar, const float* kbar, int B, int H, int nblk, int top_k,
                           float top_p, float scale, int cap, int32_t* idx, int32_t* cnt,
                           cudaStream_t s) {
   if (nblk == 0) return cudaSuccess;
-  const size_t smem = select_smem_bytes(nblk);
-  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
-  if (e != cudaSuccess) return e;
-  dim3 grid((nblk + kSelRows - 1) / kSelRows, H, B);
-  select_kernel<<<grid, 256, smem, s>>>(qbar, kbar, H, nblk, top_k, top_p, scale, cap, idx, cnt);
-  return cudaGetLastError();
+  // registers per lane: the row rounded up to a multiple of 32 x {8, 32, 64, 96, 128, 192}
+  const int vpl = (nblk + 31) / 32;
+#define MMDIT_SEL(V) \
+  if (vpl <= V) return launch_select_vpl<V>(qbar, kbar, B, H, nblk, top_k, top_p, scale, cap, idx, cnt, s)
+  MMDIT_SEL(8);
+  MMDIT_SEL(32);
+  MMDIT_SEL(64);
+  MMDIT_SEL(96);
+  MMDIT_SEL(128);
+  MMDIT_SEL(192);
+#undef MMDIT_SEL
+  return cudaErrorInvalidValue;  // more blocks than the library supports (checked earlier)
 }
 
 cudaError_t launch_groups(int T, int H, int W, int nblk, int4* groups, int*, cudaStream_t s) {
