@@ -456,7 +456,7 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
       int ucount = 0;
       if (pr.mode == kModeSparse) {
         int acc = 0;
-        qb = 31;  // rows past the group: member of nothing
+        qb = -1;  // rows past the group: member of nothing
         for (int i = 0; i < w.g_nblk; ++i) {
           int bst, blen;
           block_extent(pr.vT, pr.vH, pr.vW, w.g_first + i, bst, blen);
@@ -474,15 +474,27 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
         // valid key columns of each 64-row half of this tile for this row
         // (independent of S, so computed before waiting for it)
         int len0, len1;
+        uint32_t seg0 = 0xFu, seg1 = 0xFu;  // valid 16-row segments of each half
         if (pr.mode == kModeDense) {
           const int s0 = w.kv_lo + j * 128;
           len0 = max(0, min(64, w.kv_hi - s0));
           len1 = max(0, min(64, w.kv_hi - s0 - 64));
         } else {
-          const uint2 e0 = pr.ulist[w.ubase + 2 * j];
-          const uint2 e1 = (2 * j + 1 < ucount) ? pr.ulist[w.ubase + 2 * j + 1] : make_uint2(0u, 0u);
-          len0 = ((e0.y >> 16) >> qb) & 1u ? (int)(e0.y & 0xFFu) : 0;
-          len1 = ((e1.y >> 16) >> qb) & 1u ? (int)(e1.y & 0xFFu) : 0;
+          const uint4 e0 = pr.ulist[w.ubase + 2 * j];
+          const uint4 e1 = (2 * j + 1 < ucount) ? pr.ulist[w.ubase + 2 * j + 1]
+                                                : make_uint4(0u, 0u, 0u, 0u);
+          len0 = (int)e0.y;
+          len1 = (int)e1.y;
+          // this row's query block (0..15) in each segment's membership mask;
+          // rows past the group (qb < 0) are members of nothing
+          if (qb >= 0) {
+            seg0 = ((e0.z >> qb) & 1u) | (((e0.z >> (16 + qb)) & 1u) << 1) |
+                   (((e0.w >> qb) & 1u) << 2) | (((e0.w >> (16 + qb)) & 1u) << 3);
+            seg1 = ((e1.z >> qb) & 1u) | (((e1.z >> (16 + qb)) & 1u) << 1) |
+                   (((e1.w >> qb) & 1u) << 2) | (((e1.w >> (16 + qb)) & 1u) << 3);
+          } else {
+            seg0 = seg1 = 0u;
+          }
         }
         ok = ok && mbar_wait(bar(B_SFULL + t), st & 1, err);
         if (__any_sync(0xffffffffu, !ok)) {
@@ -507,12 +519,12 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
             s[96 + i] = __uint_as_float(v3[i]);
           }
         }
-        const bool masked = len0 < 64 || len1 < 64;
+        const bool masked = len0 < 64 || len1 < 64 || seg0 != 0xFu || seg1 != 0xFu;
         if (masked) {
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
-            if (c >= len0) s[c] = -INFINITY;
-            if (c >= len1) s[64 + c] = -INFINITY;
+            if (c >= len0 || !((seg0 >> (c >> 4)) & 1u)) s[c] = -INFINITY;
+            if (c >= len1 || !((seg1 >> (c >> 4)) & 1u)) s[64 + c] = -INFINITY;
           }
         }
         const float mt = row_max128(s);

@@ -44,7 +44,7 @@ struct AttnProblem {
   int mode;                   // AttnMode
   // sparse mode: the query groups and the merged key-block lists
   const int4* groups;         // per group: {first block, n blocks, start token, n tokens}
-  const uint2* ulist;         // [B][H][n_groups][ucap]: {start token, len | member mask << 16}
+  const uint4* ulist;         // [B][H][n_groups][ucap]: {start, len, seg masks 0|1, seg masks 2|3}
   const int* ucnt;            // [B][H][n_groups]
   int ucap;
   int vT, vH, vW;             // block-major video grid (sparse mode)
@@ -79,7 +79,7 @@ cudaError_t launch_groups(int T, int H, int W, int nblk, int4* groups, int* n_gr
                           cudaStream_t s);
 cudaError_t launch_union(const int32_t* idx, const int32_t* cnt, int cap, const int4* groups,
                          int n_groups_max, const int* n_groups, int B, int H, int nblk, int T,
-                         int Hg, int Wg, uint2* ulist, int* ucnt, cudaStream_t s);
+                         int Hg, int Wg, uint4* ulist, int* ucnt, cudaStream_t s);
 
 // helpers (mmdit_api.cu)
 int* device_error_flag();  // device address of this device's error word

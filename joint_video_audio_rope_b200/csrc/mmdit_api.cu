@@ -525,7 +525,7 @@ size_t mmdit_sparse_attn_workspace_size(const mmdit_tensor_desc* desc, const mmd
   if (check_desc(desc, "sparse_attn") || sparse_layout(layout, desc, T, H, W, nblk)) return 0;
   const int ng = host_group_count(T, H, W, nblk);
   const size_t lists = (size_t)desc->batch * desc->heads * ng;
-  return align256(sizeof(int4) * ng) + align256(lists * nblk * sizeof(uint2)) +
+  return align256(sizeof(int4) * ng) + align256(lists * nblk * sizeof(uint4)) +
          align256(lists * sizeof(int));
 }
 
@@ -548,7 +548,7 @@ int mmdit_sparse_attn(const void* q, const void* k, const void* v, void* o,
   const int ng = host_group_count(T, H, W, nblk);
   const size_t lists = (size_t)desc->batch * desc->heads * ng;
   const size_t g_bytes = align256(sizeof(int4) * ng);
-  const size_t l_bytes = align256(lists * nblk * sizeof(uint2));
+  const size_t l_bytes = align256(lists * nblk * sizeof(uint4));
   const size_t c_bytes = align256(lists * sizeof(int));
   if (workspace == nullptr || ws_bytes < g_bytes + l_bytes + c_bytes)
     return fail(MMDIT_EWORKSPACE, "sparse_attn: workspace needs %zu bytes", g_bytes + l_bytes + c_bytes);
@@ -557,7 +557,7 @@ int mmdit_sparse_attn(const void* q, const void* k, const void* v, void* o,
   if ((rc = check_sm100())) return rc;
   char* ws = static_cast<char*>(workspace);
   int4* groups = reinterpret_cast<int4*>(ws);
-  uint2* ulist = reinterpret_cast<uint2*>(ws + g_bytes);
+  uint4* ulist = reinterpret_cast<uint4*>(ws + g_bytes);
   int* ucnt = reinterpret_cast<int*>(ws + g_bytes + l_bytes);
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = launch_groups(T, H, W, nblk, groups, nullptr, s);

@@ -19,11 +19,13 @@
 //                  descending, ties by lower id.
 //   groups_kernel  partitions the query blocks into CTA groups of <= 256
 //                  tokens and <= 16 blocks (greedy, in block order).
-//   union_kernel   per (group, head, batch): merges the groups' selected
-//                  lists into one ascending list; each entry holds the key
-//                  block's start token, its length and a 16-bit membership
-//                  mask (which query blocks of the group selected it).  The
-//                  attention kernel walks it.
+//   union_kernel   per (group, head, batch): merges the group's selected
+//                  lists into one ascending list of 64-row key half-tiles;
+//                  an entry holds a start token, a length and a 16-bit
+//                  membership mask per 16-token segment (which query blocks
+//                  of the group selected that key block).  Consecutive
+//                  16-token blocks share an entry.  The attention kernel
+//                  walks the list two entries per key tile.
 #include <math.h>
 
 #include "internal.h"
@@ -280,14 +282,54 @@ __global__ void groups_kernel(int T, int H, int W, int nblk, int4* groups) {
   if (nb > 0) groups[g++] = make_int4(first, nb, start, tokens);
 }
 
+// Block-wide inclusive scans over one value per thread (256 threads).
+__device__ __forceinline__ int block_scan_sum(int v, int* wsum, int lane, int warp, int& total) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) wsum[warp] = v;
+  __syncthreads();
+  int before = 0;
+  total = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    before += (w < warp) ? wsum[w] : 0;
+    total += wsum[w];
+  }
+  __syncthreads();
+  return v + before;
+}
+__device__ __forceinline__ int block_scan_max(int v, int* wmax, int lane, int warp) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v = max(v, n);
+  }
+  if (lane == 31) wmax[warp] = v;
+  __syncthreads();
+  int before = -1;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) before = (w < warp) ? max(before, wmax[w]) : before;
+  __syncthreads();
+  return max(v, before);
+}
+
+// Merged key-block list of one query group.  Entry = one 64-row half of an
+// attention key tile: {start token, length, membership masks of its four
+// 16-token segments (16 bits each: which query blocks of the group selected
+// the key block the segment belongs to)}.  A 64-token block is one entry;
+// runs of consecutive 16-token blocks (the short last t-slab), which are
+// contiguous in block-major storage, are packed four to an entry.
 __global__ void __launch_bounds__(256) union_kernel(const int32_t* __restrict__ idx,
                                                     const int32_t* __restrict__ cnt, int cap,
                                                     const int4* __restrict__ groups, int H,
                                                     int nblk, int n_groups, int T, int Hg, int Wg,
-                                                    uint2* __restrict__ ulist,
+                                                    uint4* __restrict__ ulist,
                                                     int* __restrict__ ucnt) {
   extern __shared__ uint32_t mask[];  // [nblk]
-  __shared__ int warp_tot[8];
+  __shared__ int wtmp[8];
   const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int4 gr = groups[g];
@@ -304,27 +346,49 @@ __global__ void __launch_bounds__(256) union_kernel(const int32_t* __restrict__ 
   }
   __syncthreads();
   const long long lid = ((long long)b * H + h) * n_groups + g;
-  uint2* out = ulist + lid * nblk;
-  int running = 0;
+  uint4* out = ulist + lid * nblk;
+  auto packable = [&](int j) {
+    if (j < 0 || j >= nblk || mask[j] == 0u) return false;
+    int st, len;
+    block_extent(T, Hg, Wg, j, st, len);
+    return len == 16;
+  };
+  int running = 0, run_carry = -1;
   for (int j0 = 0; j0 < nblk; j0 += 256) {
     const int j = j0 + tid;
-    const uint32_t m = j < nblk ? mask[j] : 0u;
-    const unsigned bal = __ballot_sync(0xffffffffu, m != 0u);
-    if (lane == 0) warp_tot[warp] = __popc(bal);
-    __syncthreads();
-    int before = 0, total = 0;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      before += (w < warp) ? warp_tot[w] : 0;
-      total += warp_tot[w];
-    }
-    if (m != 0u) {
+    const bool in = j < nblk && mask[j] != 0u;
+    const bool pk = in && packable(j);
+    // start of a run of consecutive packable blocks
+    const bool run_start = pk && !packable(j - 1);
+    int last_start = block_scan_max(run_start ? j : -1, wtmp, lane, warp);
+    last_start = max(last_start, run_carry);
+    const int rank = pk ? j - last_start : 0;
+    const bool leader = in && (!pk || (rank & 3) == 0);
+    int total;
+    const int pos = block_scan_sum(leader ? 1 : 0, wtmp, lane, warp, total) - (leader ? 1 : 0);
+    if (leader) {
       int st, len;
       block_extent(T, Hg, Wg, j, st, len);
-      out[running + before + __popc(bal & ((1u << lane) - 1u))] =
-          make_uint2((uint32_t)st, (uint32_t)len | (m << 16));
+      uint32_t m[4];
+      if (!pk) {
+        m[0] = m[1] = m[2] = m[3] = mask[j];
+      } else {
+        m[0] = mask[j];
+        len = 16;
+        m[1] = m[2] = m[3] = 0u;
+        for (int q = 1; q < 4 && packable(j + q); ++q) {
+          m[q] = mask[j + q];
+          len += 16;
+        }
+      }
+      out[running + pos] = make_uint4((uint32_t)st, (uint32_t)len, m[0] | (m[1] << 16),
+                                      m[2] | (m[3] << 16));
     }
     running += total;
+    // the last thread's run start carries into the next chunk
+    if (tid == 255) wtmp[0] = last_start;
+    __syncthreads();
+    run_carry = wtmp[0];
     __syncthreads();
   }
   if (tid == 0) ucnt[lid] = running;
@@ -383,7 +447,7 @@ cudaError_t launch_groups(int T, int H, int W, int nblk, int4* groups, int*, cud
 
 cudaError_t launch_union(const int32_t* idx, const int32_t* cnt, int cap, const int4* groups,
                          int n_groups, const int*, int B, int H, int nblk, int T, int Hg,
-                         int Wg, uint2* ulist, int* ucnt, cudaStream_t s) {
+                         int Wg, uint4* ulist, int* ucnt, cudaStream_t s) {
   if (n_groups == 0) return cudaSuccess;
   const size_t smem = sizeof(uint32_t) * (size_t)nblk;
   if (smem > 48 * 1024) {
