@@ -68,6 +68,16 @@ cudaError_t launch_split_combine(const float* part_o, const float* part_ml, __nv
                                  long long o_st, long long o_sb, int n_splits, int B, int H,
                                  int Nq, int Nq_pad, cudaStream_t s);
 
+// block-sparse attention: query blocks per CTA group are bounded by the rows
+// of the kernel shape used (kSparseQTiles 128-row Q tiles) and 8 blocks per
+// Q tile (membership masks are 16 bits wide)
+#ifndef MMDIT_SPARSE_QTILES
+#define MMDIT_SPARSE_QTILES 2
+#endif
+constexpr int kSparseQTiles = MMDIT_SPARSE_QTILES;
+constexpr int kGroupTokens = 128 * kSparseQTiles;
+constexpr int kGroupBlocks = 8 * kSparseQTiles;
+
 // block selection (select.cu)
 cudaError_t launch_pool(const __nv_bfloat16* q, const __nv_bfloat16* k, const mmdit_tensor_desc& d,
                         int T, int H, int W, int nblk, float* qbar, float* kbar, cudaStream_t s);

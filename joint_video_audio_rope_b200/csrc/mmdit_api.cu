@@ -187,13 +187,13 @@ int host_block_len(int T, int H, int W, int b) {
   return std::min(4, T - 4 * tb) * std::min(4, H - 4 * hb) * std::min(4, W - 4 * wb);
 }
 
-// greedy grouping of query blocks (<= 256 tokens, <= 16 blocks); the device
-// groups_kernel applies the same rule and writes the table.
+// greedy grouping of query blocks (<= kGroupTokens tokens, <= kGroupBlocks
+// blocks); the device groups_kernel applies the same rule and writes the table.
 int host_group_count(int T, int H, int W, int nblk) {
   int g = 0, nb = 0, tokens = 0;
   for (int b = 0; b < nblk; ++b) {
     const int len = host_block_len(T, H, W, b);
-    if (nb == 16 || tokens + len > 256) {
+    if (nb == kGroupBlocks || tokens + len > kGroupTokens) {
       ++g;
       nb = 0;
       tokens = 0;
@@ -582,6 +582,7 @@ int mmdit_sparse_attn(const void* q, const void* k, const void* v, void* o,
   pr.kv_per_split = 0;
   pr.ctas = ng * pr.H * pr.B;
   pr.mode = kModeSparse;
+  p.q_tiles = kSparseQTiles;
   pr.groups = groups;
   pr.ulist = ulist;
   pr.ucnt = ucnt;

@@ -17,8 +17,9 @@
 //                  (mass search) by bisection on the fp32 bit patterns, and an
 //                  ascending-id compaction with warp ballots.  Ranking is P
 //                  descending, ties by lower id.
-//   groups_kernel  partitions the query blocks into CTA groups of <= 256
-//                  tokens and <= 16 blocks (greedy, in block order).
+//   groups_kernel  partitions the query blocks into CTA groups of at most the
+//                  CTA's query rows and 8 blocks per Q tile (greedy, in block
+//                  order).
 //   union_kernel   per (group, head, batch): merges the group's selected
 //                  lists into one ascending list of 64-row key half-tiles;
 //                  an entry holds a start token, a length and a 16-bit
@@ -260,15 +261,16 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ q
   if (lane == 0) cnt[hb + row] = pos;
 }
 
-// Greedy partition of the query blocks into groups of <= 256 tokens and <= 16
-// blocks; must agree with the host-side count (see mmdit_api.cu).
+// Greedy partition of the query blocks into groups of <= kGroupTokens tokens
+// and <= kGroupBlocks blocks; must agree with the host-side count
+// (mmdit_api.cu).
 __global__ void groups_kernel(int T, int H, int W, int nblk, int4* groups) {
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
   int g = 0, first = 0, nb = 0, tokens = 0, start = 0;
   for (int b = 0; b < nblk; ++b) {
     int st, len;
     block_extent(T, H, W, b, st, len);
-    if (nb == 16 || tokens + len > 256) {
+    if (nb == kGroupBlocks || tokens + len > kGroupTokens) {
       groups[g++] = make_int4(first, nb, start, tokens);
       first = b;
       nb = 0;
