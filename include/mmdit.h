@@ -266,6 +266,15 @@ MMDIT_API int mmdit_num_blocks(const mmdit_layout* layout);
  * in a kernel since the last call, or MMDIT_ECUDA. */
 MMDIT_API int mmdit_device_status(mmdit_stream_t stream);
 
+/* Diagnostic, no counterpart on the source pages: launches one warp that
+ * waits on an mbarrier nothing ever arrives at, through the library's bounded
+ * device wait, with a limit of limit_ms (1..2000).  The wait gives up, records
+ * MMDIT_ETIMEOUT in the device error word (read and cleared by
+ * mmdit_device_status; until then the library's attention kernels skip their
+ * work) and writes 1 to the device int *waited_out.  Exercises failure
+ * detection without faulting or hanging the GPU.  Errors: EINVAL, ECUDA. */
+MMDIT_API int mmdit_selftest_wait_timeout(int limit_ms, int* waited_out, mmdit_stream_t stream);
+
 /* Thread-local description of the last error returned on this thread. */
 MMDIT_API const char* mmdit_last_error(void);
 

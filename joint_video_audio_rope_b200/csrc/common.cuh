@@ -139,16 +139,20 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 // kWaitLimitNs, records MMDIT_ETIMEOUT in the library's device error flag
 // (`err`, a per-device word owned by the host side) and returns false.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err) {
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, int* err,
+                                              uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       atomicExch(err, (int)MMDIT_ETIMEOUT);
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err) {
+  return mbar_wait_for(bar, parity, err, kWaitLimitNs);
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {

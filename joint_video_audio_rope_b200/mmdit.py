@@ -73,6 +73,7 @@ _SIGS = {
     "mmdit_sparse_attn_workspace_size": (C.c_size_t, [_D, _L, C.c_int]),
     "mmdit_num_blocks": (C.c_int, [_L]),
     "mmdit_device_status": (C.c_int, [_P]),
+    "mmdit_selftest_wait_timeout": (C.c_int, [C.c_int, _P, _P]),
     "mmdit_last_error": (C.c_char_p, []),
     "mmdit_version": (C.c_char_p, []),
 }
@@ -233,6 +234,10 @@ def num_blocks(layout: Layout) -> int:
 
 def device_status(stream=None) -> int:
     return _lib.mmdit_device_status(_stream(stream))
+
+
+def selftest_wait_timeout(limit_ms: int, waited_out, stream=None) -> None:
+    _check(_lib.mmdit_selftest_wait_timeout(limit_ms, _ptr(waited_out), _stream(stream)))
 
 
 def raw(name: str):

@@ -66,3 +66,39 @@ def test_reference_arm_other_ranks_exit_without_work(monkeypatch):
     monkeypatch.setenv("RANK", "1")
     monkeypatch.setenv("WORLD_SIZE", "2")
     assert bench.main(["--impl", "reference", "--workload", "tiny_f32"]) == 0
+
+
+def _worker_missing_peer(rank, world, port, out):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch.distributed as dist
+
+    import bench
+    r, w, _ = bench.dist_env()
+    dist.init_process_group("gloo", rank=r, world_size=w, timeout=datetime.timedelta(seconds=5))
+    if r == 1:
+        out.put((r, "left"))  # this rank leaves between steps, before the barrier
+        return
+    try:
+        bench.barrier(w)
+        out.put((r, "no error"))
+    except Exception as e:  # the short process-group timeout ends the wait
+        out.put((r, type(e).__name__))
+
+
+def test_rank_that_never_joins_is_detected():
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_missing_peer, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+    assert res[1] == "left"
+    assert res[0] != "no error"
