@@ -699,31 +699,45 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
 }
 
 // Merge split-KV partials: O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
-__global__ void split_combine_kernel(const float* __restrict__ part_o,
-                                     const float* __restrict__ part_ml, __nv_bfloat16* o,
-                                     long long o_st, long long o_sb, int n_splits, int B, int H,
-                                     int Nq, int Nq_pad) {
-  const int row = blockIdx.x;  // over B * H * Nq
-  const int q = row % Nq;
-  const int h = (row / Nq) % H;
-  const int b = row / (Nq * H);
-  const int c = threadIdx.x;   // channel (128 threads)
+// One warp per query row; lane l owns channels 4l..4l+3 (float4 loads of every
+// split's 512-byte partial row), split weights computed once per row.
+__global__ void __launch_bounds__(256) split_combine_kernel(const float* __restrict__ part_o,
+                                                            const float* __restrict__ part_ml,
+                                                            __nv_bfloat16* o, long long o_st,
+                                                            long long o_sb, int n_splits, int B,
+                                                            int H, int Nq, int Nq_pad) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);  // over B * H * Nq
+  if (row >= (long long)B * H * Nq) return;
+  const int q = (int)(row % Nq);
+  const int h = (int)((row / Nq) % H);
+  const int b = (int)(row / ((long long)Nq * H));
+  const long long stride = (long long)B * H * Nq_pad;  // rows between splits
+  const long long r0 = ((long long)b * H + h) * Nq_pad + q;
   float M = -INFINITY;
+  for (int s = lane; s < n_splits; s += 32) M = fmaxf(M, part_ml[(r0 + s * stride) * 2]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  float L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s = 0; s < n_splits; ++s) {
-    const long long pr = (((long long)s * B + b) * H + h) * Nq_pad + q;
-    M = fmaxf(M, part_ml[pr * 2]);
-  }
-  float L = 0.f, acc = 0.f;
-  for (int s = 0; s < n_splits; ++s) {
-    const long long pr = (((long long)s * B + b) * H + h) * Nq_pad + q;
+    const long long pr = r0 + s * stride;
     const float m = part_ml[pr * 2];
     if (m == -INFINITY) continue;
     const float f = exp2f(m - M);
     L += f * part_ml[pr * 2 + 1];
-    acc += f * part_o[pr * 128 + c];
+    const float4 v = *reinterpret_cast<const float4*>(part_o + pr * 128 + lane * 4);
+    acc.x += f * v.x;
+    acc.y += f * v.y;
+    acc.z += f * v.z;
+    acc.w += f * v.w;
   }
-  o[(long long)b * o_sb + (long long)q * o_st + (long long)h * 128 + c] =
-      __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  uint2 pk;
+  pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+  pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+  *reinterpret_cast<uint2*>(o + (long long)b * o_sb + (long long)q * o_st + (long long)h * 128 +
+                            lane * 4) = pk;
 }
 
 template <int QT, int ST, bool PERSIST>
@@ -764,9 +778,10 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
 cudaError_t launch_split_combine(const float* part_o, const float* part_ml, __nv_bfloat16* o,
                                  long long o_st, long long o_sb, int n_splits, int B, int H,
                                  int Nq, int Nq_pad, cudaStream_t s) {
-  if (B * H * Nq == 0) return cudaSuccess;
-  split_combine_kernel<<<B * H * Nq, 128, 0, s>>>(part_o, part_ml, o, o_st, o_sb, n_splits, B, H,
-                                                 Nq, Nq_pad);
+  const long long rows = (long long)B * H * Nq;
+  if (rows == 0) return cudaSuccess;
+  split_combine_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(part_o, part_ml, o, o_st, o_sb,
+                                                                 n_splits, B, H, Nq, Nq_pad);
   return cudaGetLastError();
 }
 
