@@ -599,65 +599,60 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
       const bool valid_row = row < w.q_valid;
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const int qrow = w.q0 + row;
+      // O row into registers with one TMEM round trip, then hand TMEM back to
+      // the MMA warp before any global store (the next item's first PV may
+      // overwrite O while this warpgroup stores)
+      uint32_t o0[32], o1[32], o2[32], o3[32];
+      if (nkv > 0) {
+        tmem_ld32(o_addr, o0);
+        tmem_ld32(o_addr + 32, o1);
+        tmem_ld32(o_addr + 64, o2);
+        tmem_ld32(o_addr + 96, o3);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o0[i] = o1[i] = o2[i] = o3[i] = 0u;
+      }
+      tc_fence_before();
+      mbar_arrive(bar(B_OEMPTY + t));
+      auto ov = [&](int c) -> uint32_t {  // column c of this row (compile-time c)
+        return c < 32 ? o0[c] : c < 64 ? o1[c - 32] : c < 96 ? o2[c - 64] : o3[c - 96];
+      };
       if (pr.part_o != nullptr) {
         // split-KV partial: unnormalised O, running max (log2 units) and sum
         const long long prow =
             (((long long)w.split * pr.B + w.b) * pr.H + w.h) * (long long)(pr.n_qtiles * C::kRows) +
             (long long)w.qtile * C::kRows + row;
         float* dst = pr.part_o + prow * 128;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          if (nkv > 0) {
-            tmem_ld32(o_addr + c * 32, v);
-            tmem_wait_ld();
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0u;
-          }
-          if (valid_row) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              *reinterpret_cast<float4*>(dst + c * 32 + i) =
-                  make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
-                              __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
-          }
-        }
         if (valid_row) {
+#pragma unroll
+          for (int i = 0; i < 128; i += 4)
+            *reinterpret_cast<float4*>(dst + i) =
+                make_float4(__uint_as_float(ov(i)), __uint_as_float(ov(i + 1)),
+                            __uint_as_float(ov(i + 2)), __uint_as_float(ov(i + 3)));
           pr.part_ml[prow * 2 + 0] = (m_used == -INFINITY) ? -INFINITY : m_used * sl2;
           pr.part_ml[prow * 2 + 1] = l;
         }
       } else {
         // normalised bf16 O: each round stages kStageCols channels of the
         // warp's 32 rows in shared memory (16-byte chunks XOR-swizzled by row,
-        // conflict-free both ways), then writes them back so that 8 lanes
-        // cover one row's contiguous bytes
+        // conflict-free both ways), then writes them back so that a group of
+        // lanes covers one row's contiguous bytes
         constexpr int SC = C::kStageCols;
         constexpr int CH = SC / 8;  // 16-byte chunks per staged row
         uint8_t* stage = smem + C::kStageOff + warp * C::kStageWarpBytes;
         const int wrow0 = (warp & 3) * 32;  // first row of this warp inside the tile
-#pragma unroll 1
+#pragma unroll
         for (int r = 0; r < 128 / SC; ++r) {
 #pragma unroll
-          for (int c = 0; c < SC / 32; ++c) {
-            uint32_t v[32];
-            if (nkv > 0) {
-              tmem_ld32(o_addr + r * SC + c * 32, v);
-              tmem_wait_ld();
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = 0u;
-            }
-#pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              uint4 pk;
-              pk.x = pack_bf16x2(__uint_as_float(v[i + 0]) * inv, __uint_as_float(v[i + 1]) * inv);
-              pk.y = pack_bf16x2(__uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv);
-              pk.z = pack_bf16x2(__uint_as_float(v[i + 4]) * inv, __uint_as_float(v[i + 5]) * inv);
-              pk.w = pack_bf16x2(__uint_as_float(v[i + 6]) * inv, __uint_as_float(v[i + 7]) * inv);
-              const int chunk = c * 4 + i / 8;
-              *reinterpret_cast<uint4*>(stage + lane * (SC * 2) + ((chunk ^ (lane % CH)) << 4)) = pk;
-            }
+          for (int chunk = 0; chunk < CH; ++chunk) {
+            const int c0 = r * SC + chunk * 8;
+            uint4 pk;
+            pk.x = pack_bf16x2(__uint_as_float(ov(c0 + 0)) * inv, __uint_as_float(ov(c0 + 1)) * inv);
+            pk.y = pack_bf16x2(__uint_as_float(ov(c0 + 2)) * inv, __uint_as_float(ov(c0 + 3)) * inv);
+            pk.z = pack_bf16x2(__uint_as_float(ov(c0 + 4)) * inv, __uint_as_float(ov(c0 + 5)) * inv);
+            pk.w = pack_bf16x2(__uint_as_float(ov(c0 + 6)) * inv, __uint_as_float(ov(c0 + 7)) * inv);
+            *reinterpret_cast<uint4*>(stage + lane * (SC * 2) + ((chunk ^ (lane % CH)) << 4)) = pk;
           }
           __syncwarp();
           constexpr int RPI = 32 / CH;  // rows per store instruction
@@ -682,9 +677,6 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
               l > 0.f ? (mref + log2f(l)) * 0.69314718055994531f : -INFINITY;
         }
       }
-      // O has been read out of TMEM: the next item's first PV may overwrite it
-      tc_fence_before();
-      mbar_arrive(bar(B_OEMPTY + t));
     }
   }
 
