@@ -111,7 +111,7 @@ constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0, 0);  // Q, K: K-major
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 0, 1);  // P (TMEM), V: MN-major
 
 struct Work {
-  int prob, b, h, split, qtile;
+  int b, h, split, qtile;
   int q0;       // first query token of the CTA (row 0 of Q tile 0)
   int q_valid;  // valid query rows of the CTA (<= rows per CTA)
   int kv_lo, kv_hi;  // dense: key range
@@ -121,7 +121,7 @@ struct Work {
 };
 
 __device__ __forceinline__ int total_items(const AttnParams& P) {
-  return P.prob[0].ctas + (P.n_prob > 1 ? P.prob[1].ctas : 0);
+  return P.prob.ctas;
 }
 
 // k-th work item of this CTA: the CTA's own item, or (persistent launches)
@@ -135,12 +135,7 @@ __device__ __forceinline__ int item_of(const AttnParams&, int k, int n_items) {
 __device__ __forceinline__ Work decode_work(const AttnParams& P, int item, int rows) {
   Work w;
   int idx = item;
-  w.prob = 0;
-  if (P.n_prob > 1 && idx >= P.prob[0].ctas) {
-    idx -= P.prob[0].ctas;
-    w.prob = 1;
-  }
-  const AttnProblem& pr = P.prob[w.prob];
+  const AttnProblem& pr = P.prob;
   w.qtile = idx % pr.n_qtiles;
   idx /= pr.n_qtiles;
   w.split = idx % pr.n_splits;
@@ -311,7 +306,7 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
       for (int item = item_of<PERSIST>(P, 0, n_items); item < n_items && ok;
            item = item_of<PERSIST>(P, ++it, n_items)) {
         const Work w = decode_work(P, item, C::kRows);
-        const AttnProblem& pr = P.prob[w.prob];
+        const AttnProblem& pr = P.prob;
         if (it == 0) {
           tma_prefetch_desc(&pr.tmQ);
           tma_prefetch_desc(&pr.tmK);
@@ -361,7 +356,7 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
       for (int item = item_of<PERSIST>(P, 0, n_items); item < n_items && ok;
            item = item_of<PERSIST>(P, ++it, n_items)) {
         const Work w = decode_work(P, item, C::kRows);
-        const AttnProblem& pr = P.prob[w.prob];
+        const AttnProblem& pr = P.prob;
         const int nkv = w.nkv;
         const int qbar = pr.rope_q ? B_QREADY : B_QFULL;
         for (int t = 0; t < QT && ok; ++t) ok = mbar_wait(bar(qbar + t), it & 1, err);
@@ -439,7 +434,7 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
     for (int item = item_of<PERSIST>(P, 0, n_items); item < n_items && ok;
            item = item_of<PERSIST>(P, ++it, n_items)) {
       const Work w = decode_work(P, item, C::kRows);
-      const AttnProblem& pr = P.prob[w.prob];
+      const AttnProblem& pr = P.prob;
       const int nkv = w.nkv;
 
       if (pr.rope_q) {
@@ -742,7 +737,7 @@ cudaError_t launch_shape(const AttnParams& p, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const int items = p.prob[0].ctas + (p.n_prob > 1 ? p.prob[1].ctas : 0);
+  const int items = p.prob.ctas;
   if (items == 0) return cudaSuccess;
   int grid = items;
   if (PERSIST) {

@@ -129,6 +129,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// As mbar_try_wait, but a thread whose phase is not complete yet may be
+// suspended for up to `hint_ns` (woken early when the phase completes), so
+// that waiting warps do not take issue slots from the working ones.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
@@ -139,12 +154,13 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 // kWaitLimitNs, records MMDIT_ETIMEOUT in the library's device error flag
 // (`err`, a per-device word owned by the host side) and returns false.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr uint32_t kWaitSleepNs = 1000000u;        // longest single suspension: 1 ms
 __device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, int* err,
                                               uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
     if (global_timer_ns() - t0 > limit_ns) {
       atomicExch(err, (int)MMDIT_ETIMEOUT);
       return false;

@@ -51,9 +51,11 @@ struct AttnProblem {
   int rope_q;                 // rotate Q tiles in shared memory after loading
 };
 
+// One attention problem per launch: every field of `prob` sits at a fixed
+// offset of the kernel's parameter block, so the kernel reads it with
+// immediate constant-bank operands instead of indexed loads.
 struct AttnParams {
-  AttnProblem prob[2];
-  int n_prob;
+  AttnProblem prob;
   int q_tiles;                // 128-row Q tiles per CTA: 2 (default) or 1
   int persistent;             // 0: one CTA per work item; 1: one CTA per SM slot, looping
   float scale_log2;           // softmax scale * log2(e)
@@ -63,6 +65,13 @@ struct AttnParams {
 };
 
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s);
+// Both directions of the audio<->video cross-attention on one stream: audio
+// queries over the video keys (split-KV partials into part_o / part_ml), video
+// queries over the audio keys, then the merge of the partials.
+int launch_cross(const void* qv, const void* kv, const void* vv, const void* qa, const void* ka,
+                 const void* va, void* o_video, void* o_audio, const mmdit_tensor_desc& video,
+                 const mmdit_tensor_desc& audio, float scale, int splits, int kv_per_split,
+                 float* part_o, float* part_ml, cudaStream_t s);
 int attn_rows_per_cta(int q_tiles);  // query rows one CTA covers
 cudaError_t launch_split_combine(const float* part_o, const float* part_ml, __nv_bfloat16* o,
                                  long long o_st, long long o_sb, int n_splits, int B, int H,

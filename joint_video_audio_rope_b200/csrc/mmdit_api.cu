@@ -236,6 +236,70 @@ CrossPlan plan_cross(const mmdit_tensor_desc* v, const mmdit_tensor_desc* a) {
   return p;
 }
 
+int launch_cross(const void* qv, const void* kv, const void* vv, const void* qa, const void* ka,
+                 const void* va, void* o_video, void* o_audio, const mmdit_tensor_desc& video,
+                 const mmdit_tensor_desc& audio, float scale, int splits, int kv_per_split,
+                 float* part_o, float* part_ml, cudaStream_t s) {
+  int rc;
+  int* err = device_error_flag();
+  if (err == nullptr) return fail(MMDIT_ECUDA, "device error flag unavailable");
+  // audio queries over the video keys: 2 Q tiles per CTA, keys split across
+  // CTAs, unnormalised partials merged by the combine kernel
+  AttnParams pa{};
+  AttnProblem& a2v = pa.prob;
+  if ((rc = make_map(&a2v.tmQ, qa, audio, audio.n_tokens, "qa")) ||
+      (rc = make_map(&a2v.tmK, kv, video, video.n_tokens, "kv")) ||
+      (rc = make_map(&a2v.tmV, vv, video, video.n_tokens, "vv")))
+    return rc;
+  a2v.o = nullptr;
+  a2v.part_o = part_o;
+  a2v.part_ml = part_ml;
+  a2v.Nq = audio.n_tokens;
+  a2v.Nkv = video.n_tokens;
+  a2v.H = audio.heads;
+  a2v.B = audio.batch;
+  a2v.n_qtiles = (audio.n_tokens + 255) / 256;
+  a2v.n_splits = splits;
+  a2v.kv_per_split = kv_per_split;
+  a2v.ctas = a2v.n_qtiles * a2v.n_splits * a2v.H * a2v.B;
+  a2v.mode = kModeDense;
+  pa.q_tiles = 2;
+  pa.persistent = 1;
+  pa.scale_log2 = scale * 1.4426950408889634f;
+  pa.err = err;
+  // video queries over the (short) audio keys: persistent CTAs, two per SM,
+  // hide each other's load and epilogue latency
+  AttnParams pv{};
+  AttnProblem& v2a = pv.prob;
+  if ((rc = make_map(&v2a.tmQ, qv, video, video.n_tokens, "qv")) ||
+      (rc = make_map(&v2a.tmK, ka, audio, audio.n_tokens, "ka")) ||
+      (rc = make_map(&v2a.tmV, va, audio, audio.n_tokens, "va")))
+    return rc;
+  v2a.o = (__nv_bfloat16*)o_video;
+  v2a.o_st = video.stride_tok;
+  v2a.o_sb = video.stride_batch;
+  v2a.Nq = video.n_tokens;
+  v2a.Nkv = audio.n_tokens;
+  v2a.H = video.heads;
+  v2a.B = video.batch;
+  v2a.n_qtiles = (video.n_tokens + 128 * kV2aQTiles - 1) / (128 * kV2aQTiles);
+  v2a.n_splits = 1;
+  v2a.kv_per_split = ((audio.n_tokens + 127) / 128) * 128;
+  v2a.ctas = v2a.n_qtiles * v2a.H * v2a.B;
+  v2a.mode = kModeDense;
+  pv.q_tiles = kV2aQTiles;
+  pv.persistent = 1;
+  pv.scale_log2 = pa.scale_log2;
+  pv.err = err;
+  cudaError_t e = launch_attn_tc(pa, s);
+  if (e == cudaSuccess) e = launch_attn_tc(pv, s);
+  if (e == cudaSuccess)
+    e = launch_split_combine(part_o, part_ml, (__nv_bfloat16*)o_audio, audio.stride_tok,
+                             audio.stride_batch, splits, audio.batch, audio.heads, audio.n_tokens,
+                             a2v.n_qtiles * 256, s);
+  return e == cudaSuccess ? MMDIT_OK : cuda_fail(e, "av_cross launch");
+}
+
 int* device_error_flag() {
   static int* cache[64] = {};
   int dev = 0;
@@ -344,7 +408,7 @@ int mmdit_joint_attn(const void* q, const void* k, const void* v, void* o, float
   }
   if ((rc = check_sm100())) return rc;
   AttnParams p{};
-  AttnProblem& pr = p.prob[0];
+  AttnProblem& pr = p.prob;
   if ((rc = make_map(&pr.tmQ, q, *desc, desc->n_tokens, "q")) ||
       (rc = make_map(&pr.tmK, k, *desc, desc->n_tokens, "k")) ||
       (rc = make_map(&pr.tmV, v, *desc, desc->n_tokens, "v")))
@@ -362,7 +426,6 @@ int mmdit_joint_attn(const void* q, const void* k, const void* v, void* o, float
   pr.ctas = pr.n_qtiles * pr.H * pr.B;
   pr.mode = kModeDense;
   pr.rope_q = rope_q != nullptr;
-  p.n_prob = 1;
   p.q_tiles = 2;
   p.persistent = 0;  // measured: one item per CTA is ~1% faster for long keys
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -421,64 +484,9 @@ int mmdit_av_cross_attn(const void* qv, const void* kv, const void* vv, const vo
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(MMDIT_EINVAL, "av_cross: workspace must be 256-byte aligned");
   if ((rc = check_sm100())) return rc;
-  // audio queries over the video keys: 2 Q tiles per CTA, keys split across
-  // CTAs, unnormalised partials merged by the combine kernel
-  AttnParams pa{};
-  AttnProblem& a2v = pa.prob[0];
-  if ((rc = make_map(&a2v.tmQ, qa, *audio, audio->n_tokens, "qa")) ||
-      (rc = make_map(&a2v.tmK, kv, *video, video->n_tokens, "kv")) ||
-      (rc = make_map(&a2v.tmV, vv, *video, video->n_tokens, "vv")))
-    return rc;
-  a2v.o = nullptr;
-  a2v.part_o = reinterpret_cast<float*>(workspace);
-  a2v.part_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + c.part_o_bytes);
-  a2v.Nq = audio->n_tokens;
-  a2v.Nkv = video->n_tokens;
-  a2v.H = audio->heads;
-  a2v.B = audio->batch;
-  a2v.n_qtiles = c.n_qtiles_a;
-  a2v.n_splits = c.splits;
-  a2v.kv_per_split = c.kv_per_split;
-  a2v.ctas = a2v.n_qtiles * a2v.n_splits * a2v.H * a2v.B;
-  a2v.mode = kModeDense;
-  pa.n_prob = 1;
-  pa.q_tiles = 2;
-  pa.persistent = 1;
-  pa.scale_log2 = scale * 1.4426950408889634f;
-  pa.err = device_error_flag();
-  if (pa.err == nullptr) return fail(MMDIT_ECUDA, "device error flag unavailable");
-  // video queries over the (short) audio keys: persistent CTAs, two per SM,
-  // hide each other's load and epilogue latency
-  AttnParams pv{};
-  AttnProblem& v2a = pv.prob[0];
-  if ((rc = make_map(&v2a.tmQ, qv, *video, video->n_tokens, "qv")) ||
-      (rc = make_map(&v2a.tmK, ka, *audio, audio->n_tokens, "ka")) ||
-      (rc = make_map(&v2a.tmV, va, *audio, audio->n_tokens, "va")))
-    return rc;
-  v2a.o = (__nv_bfloat16*)o_video;
-  v2a.o_st = video->stride_tok;
-  v2a.o_sb = video->stride_batch;
-  v2a.Nq = video->n_tokens;
-  v2a.Nkv = audio->n_tokens;
-  v2a.H = video->heads;
-  v2a.B = video->batch;
-  v2a.n_qtiles = (video->n_tokens + 128 * kV2aQTiles - 1) / (128 * kV2aQTiles);
-  v2a.n_splits = 1;
-  v2a.kv_per_split = ((audio->n_tokens + 127) / 128) * 128;
-  v2a.ctas = v2a.n_qtiles * v2a.H * v2a.B;
-  v2a.mode = kModeDense;
-  pv.n_prob = 1;
-  pv.q_tiles = kV2aQTiles;
-  pv.persistent = 1;
-  pv.scale_log2 = pa.scale_log2;
-  pv.err = pa.err;
-  cudaError_t e = launch_attn_tc(pa, s);
-  if (e == cudaSuccess) e = launch_attn_tc(pv, s);
-  if (e == cudaSuccess)
-    e = launch_split_combine(a2v.part_o, a2v.part_ml, (__nv_bfloat16*)o_audio, audio->stride_tok,
-                             audio->stride_batch, c.splits, audio->batch, audio->heads,
-                             audio->n_tokens, c.nq_pad, s);
-  return e == cudaSuccess ? MMDIT_OK : cuda_fail(e, "av_cross launch");
+  return launch_cross(qv, kv, vv, qa, ka, va, o_video, o_audio, *video, *audio, scale, c.splits,
+                      c.kv_per_split, reinterpret_cast<float*>(workspace),
+                      reinterpret_cast<float*>(static_cast<char*>(workspace) + c.part_o_bytes), s);
 }
 
 size_t mmdit_block_select_workspace_size(const mmdit_tensor_desc* desc, const mmdit_layout* layout) {
@@ -566,7 +574,7 @@ int mmdit_sparse_attn(const void* q, const void* k, const void* v, void* o,
                      T, H, W, ulist, ucnt, s);
   if (e != cudaSuccess) return cuda_fail(e, "sparse_attn prep launch");
   AttnParams p{};
-  AttnProblem& pr = p.prob[0];
+  AttnProblem& pr = p.prob;
   if ((rc = make_map(&pr.tmQ, q, *desc, desc->n_tokens, "q")) ||
       (rc = make_map(&pr.tmK, k, *desc, desc->n_tokens, "k")) ||
       (rc = make_map(&pr.tmV, v, *desc, desc->n_tokens, "v")))
@@ -590,7 +598,6 @@ int mmdit_sparse_attn(const void* q, const void* k, const void* v, void* o,
   pr.vT = T;
   pr.vH = H;
   pr.vW = W;
-  p.n_prob = 1;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.err = device_error_flag();
   if (p.err == nullptr) return fail(MMDIT_ECUDA, "device error flag unavailable");

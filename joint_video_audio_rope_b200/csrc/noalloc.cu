@@ -102,50 +102,9 @@ extern "C" int mmdit_av_cross_attn_noalloc(const void* qv, const void* kv, const
   void* scratch = nullptr;
   if ((rc = scratch_address(&scratch))) return rc;
 
-  AttnParams p{};
-  AttnProblem& a2v = p.prob[0];
-  if ((rc = make_map(&a2v.tmQ, qa, *audio, audio->n_tokens, "qa")) ||
-      (rc = make_map(&a2v.tmK, kv, *video, video->n_tokens, "kv")) ||
-      (rc = make_map(&a2v.tmV, vv, *video, video->n_tokens, "vv")))
-    return rc;
-  a2v.part_o = static_cast<float*>(scratch);
-  a2v.part_ml = reinterpret_cast<float*>(
+  float* part_o = static_cast<float*>(scratch);
+  float* part_ml = reinterpret_cast<float*>(
       static_cast<char*>(scratch) + align256((size_t)splits * rows_per_split * 128 * sizeof(float)));
-  a2v.Nq = audio->n_tokens;
-  a2v.Nkv = video->n_tokens;
-  a2v.H = audio->heads;
-  a2v.B = audio->batch;
-  a2v.n_qtiles = n_qtiles;
-  a2v.n_splits = splits;
-  a2v.kv_per_split = kv_per_split;
-  a2v.ctas = n_qtiles * splits * a2v.H * a2v.B;
-  a2v.mode = kModeDense;
-  AttnProblem& v2a = p.prob[1];
-  if ((rc = make_map(&v2a.tmQ, qv, *video, video->n_tokens, "qv")) ||
-      (rc = make_map(&v2a.tmK, ka, *audio, audio->n_tokens, "ka")) ||
-      (rc = make_map(&v2a.tmV, va, *audio, audio->n_tokens, "va")))
-    return rc;
-  v2a.o = (__nv_bfloat16*)o_video;
-  v2a.o_st = video->stride_tok;
-  v2a.o_sb = video->stride_batch;
-  v2a.Nq = video->n_tokens;
-  v2a.Nkv = audio->n_tokens;
-  v2a.H = video->heads;
-  v2a.B = video->batch;
-  v2a.n_qtiles = (video->n_tokens + 255) / 256;
-  v2a.n_splits = 1;
-  v2a.kv_per_split = ((audio->n_tokens + 127) / 128) * 128;
-  v2a.ctas = v2a.n_qtiles * v2a.H * v2a.B;
-  v2a.mode = kModeDense;
-  p.n_prob = 2;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.err = device_error_flag();
-  if (p.err == nullptr) return fail(MMDIT_ECUDA, "device error flag unavailable");
-  cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = launch_attn_tc(p, s);
-  if (e == cudaSuccess)
-    e = launch_split_combine(a2v.part_o, a2v.part_ml, (__nv_bfloat16*)o_audio, audio->stride_tok,
-                             audio->stride_batch, splits, audio->batch, audio->heads,
-                             audio->n_tokens, nq_pad, s);
-  return e == cudaSuccess ? MMDIT_OK : cuda_fail(e, "av_cross_noalloc launch");
+  return launch_cross(qv, kv, vv, qa, ka, va, o_video, o_audio, *video, *audio, scale, splits,
+                      kv_per_split, part_o, part_ml, (cudaStream_t)stream);
 }
