@@ -60,13 +60,15 @@ struct Cfg {
   static constexpr int kRows = 128 * QT;  // query rows per CTA
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = QT * kTileBytes;
-  static constexpr int kBarOff = kKVOff + ST * kTileBytes;
-  // epilogue staging: per softmax warp 32 rows x kStageCols bf16 channels,
-  // so O leaves as row-contiguous stores instead of one row per lane
+  // epilogue staging: per softmax warp 32 rows x kStageCols bf16 channels
+  // (one row of kStageCols * 2 bytes per lane, 16-byte chunks swizzled as the
+  // output map's 64- or 128-byte mode expects), so O leaves in whole 32-row
+  // boxes instead of one row per lane; 1024-byte aligned like the tiles
   static constexpr int kStageCols = QT == 2 ? 64 : 32;
   static constexpr int kStageWarpBytes = 32 * kStageCols * 2;
-  static constexpr int kStageOff = kBarOff + 256;
-  static constexpr int kSmemBytes = kStageOff + 4 * QT * kStageWarpBytes + 1024;  // + align slack
+  static constexpr int kStageOff = kKVOff + ST * kTileBytes;
+  static constexpr int kBarOff = kStageOff + 4 * QT * kStageWarpBytes;
+  static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + align slack
   static constexpr int kTmemCols = 256 * QT;               // S_t and O_t per tile
   static constexpr int kMinBlocks = QT == 1 ? 2 : 1;
   // Registers per thread: at launch 65,536 / (threads x CTAs per SM), rounded
@@ -311,6 +313,8 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
           tma_prefetch_desc(&pr.tmQ);
           tma_prefetch_desc(&pr.tmK);
           tma_prefetch_desc(&pr.tmV);
+          if (pr.mode == kModeDense && pr.o != nullptr && pr.part_o == nullptr)
+            tma_prefetch_desc(&pr.tmO);
         }
         for (int t = 0; t < QT && ok; ++t) {
           if (it > 0 && !(ok = mbar_wait(bar(B_QEMPTY + t), (it - 1) & 1, err))) break;
@@ -628,8 +632,48 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
           pr.part_ml[prow * 2 + 0] = (m_used == -INFINITY) ? -INFINITY : m_used * sl2;
           pr.part_ml[prow * 2 + 1] = l;
         }
+      } else if (pr.mode == kModeDense) {
+        // normalised bf16 O through the TMA engine: each round packs
+        // kStageCols channels of the warp's 32 rows into the warp's staging
+        // buffer and one lane issues a bulk tensor store of that box; the
+        // buffer is rewritten only once the previous store has read it.  Rows
+        // past the end of the sequence lie outside the map and are not written.
+        constexpr int SC = C::kStageCols;
+        constexpr int CH = SC / 8;  // 16-byte chunks per staged row
+        const int wrow = t * 128 + (warp & 3) * 32;  // first row of this warp inside the CTA
+        if (wrow < w.q_valid) {
+          uint8_t* stg = smem + C::kStageOff + warp * C::kStageWarpBytes;
+          const int sw = ((lane * SC * 2) >> 7) & (CH - 1);  // swizzle of this lane's row
+#pragma unroll
+          for (int r = 0; r < 128 / SC; ++r) {
+            if (lane == 0) bulk_wait_read<0>();
+            __syncwarp();
+#pragma unroll
+            for (int chunk = 0; chunk < CH; ++chunk) {
+              const int c0 = r * SC + chunk * 8;
+              uint4 pk;
+              pk.x = pack_bf16x2(__uint_as_float(ov(c0 + 0)) * inv, __uint_as_float(ov(c0 + 1)) * inv);
+              pk.y = pack_bf16x2(__uint_as_float(ov(c0 + 2)) * inv, __uint_as_float(ov(c0 + 3)) * inv);
+              pk.z = pack_bf16x2(__uint_as_float(ov(c0 + 4)) * inv, __uint_as_float(ov(c0 + 5)) * inv);
+              pk.w = pack_bf16x2(__uint_as_float(ov(c0 + 6)) * inv, __uint_as_float(ov(c0 + 7)) * inv);
+              *reinterpret_cast<uint4*>(stg + lane * (SC * 2) + ((chunk ^ sw) << 4)) = pk;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_4d(&pr.tmO, smem_u32(stg), r * SC, w.h, w.q0 + wrow, w.b);
+              bulk_commit();
+            }
+          }
+        }
+        if (pr.lse != nullptr && valid_row) {
+          const float mref = (m_used == -INFINITY) ? 0.f : m_used * sl2;
+          pr.lse[((long long)w.b * pr.H + w.h) * pr.Nq + qrow] =
+              l > 0.f ? (mref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        }
       } else {
-        // normalised bf16 O: each round stages kStageCols channels of the
+        // normalised bf16 O (sparse mode, where the rows past a query group
+        // belong to the next group): each round stages kStageCols channels of the
         // warp's 32 rows in shared memory (16-byte chunks XOR-swizzled by row,
         // conflict-free both ways), then writes them back so that a group of
         // lanes covers one row's contiguous bytes
@@ -676,6 +720,8 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
   }
 
   // ------------------------------------------------------------ teardown
+  // output stores issued from shared memory complete before the CTA exits
+  bulk_wait<0>();
   tc_fence_before();
   __syncthreads();
   if (warp == C::kMmaWarp) {
@@ -753,6 +799,10 @@ cudaError_t launch_shape(const AttnParams& p, cudaStream_t s) {
 }
 
 }  // namespace
+
+int attn_store_cols(int q_tiles) {
+  return q_tiles == 1 ? Cfg<1, 2>::kStageCols : Cfg<2, 4>::kStageCols;
+}
 
 int attn_rows_per_cta(int q_tiles) { return 128 * q_tiles; }
 

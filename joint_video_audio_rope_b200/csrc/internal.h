@@ -31,6 +31,7 @@ enum AttnMode { kModeDense = 0, kModeSparse = 1 };
 
 struct AttnProblem {
   CUtensorMap tmQ, tmK, tmV;  // 4D maps {channel, head, token, batch}, box {64,1,64,1}
+  CUtensorMap tmO;            // bf16 output (dense mode), box {32 or 64,1,32,1}
   __nv_bfloat16* o;           // output (dense/sparse), or nullptr when writing partials
   long long o_st, o_sb;       // output strides (elements)
   float* lse;                 // [B, H, Nq] or nullptr
@@ -73,6 +74,7 @@ int launch_cross(const void* qv, const void* kv, const void* vv, const void* qa,
                  const mmdit_tensor_desc& audio, float scale, int splits, int kv_per_split,
                  float* part_o, float* part_ml, cudaStream_t s);
 int attn_rows_per_cta(int q_tiles);  // query rows one CTA covers
+int attn_store_cols(int q_tiles);    // channels per output store box
 cudaError_t launch_split_combine(const float* part_o, const float* part_ml, __nv_bfloat16* o,
                                  long long o_st, long long o_sb, int n_splits, int B, int H,
                                  int Nq, int Nq_pad, cudaStream_t s);
@@ -108,6 +110,11 @@ bool aligned16(const void* p);
 int check_desc(const mmdit_tensor_desc* d, const char* name);
 int make_map(CUtensorMap* m, const void* base, const mmdit_tensor_desc& d, int n_tokens,
              const char* name);
+// Store map of a bf16 [B, N, heads, 128] output with the strides of `d`: box
+// {cols channels, 1 head, 32 tokens, 1}, cols = 32 or 64 with the 64- or
+// 128-byte swizzle (the attention epilogue's staging layout).
+int make_store_map(CUtensorMap* m, void* base, const mmdit_tensor_desc& d, int n_tokens,
+                   int cols, const char* name);
 int check_sm100();
 size_t align256(size_t x);
 

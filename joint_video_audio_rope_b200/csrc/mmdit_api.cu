@@ -149,6 +149,24 @@ int make_map(CUtensorMap* m, const void* base, const mmdit_tensor_desc& d, int n
   return MMDIT_OK;
 }
 
+int make_store_map(CUtensorMap* m, void* base, const mmdit_tensor_desc& d, int n_tokens,
+                   int cols, const char* name) {
+  if (cols != 32 && cols != 64) return fail(MMDIT_EINVAL, "%s: store box of %d channels", name, cols);
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(MMDIT_ECUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[4] = {128, (cuuint64_t)d.heads, (cuuint64_t)n_tokens, (cuuint64_t)d.batch};
+  cuuint64_t strides[3] = {128 * 2, (cuuint64_t)d.stride_tok * 2,
+                           (cuuint64_t)(d.batch > 1 ? d.stride_batch : d.stride_tok * n_tokens) * 2};
+  cuuint32_t box[4] = {(cuuint32_t)cols, 1, 32, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MMDIT_ECUDA, "%s: tensor map encoding failed (%d)", name, (int)r);
+  return MMDIT_OK;
+}
+
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 int check_sm100() {
@@ -221,6 +239,9 @@ constexpr int kCrossTargetCtas = 2 * 148;
 #endif
 constexpr int kV2aQTiles = MMDIT_V2A_QTILES;
 
+// Q tiles per CTA of the dense joint attention: two, one CTA per SM.
+constexpr int kJointQTiles = 2;
+
 CrossPlan plan_cross(const mmdit_tensor_desc* v, const mmdit_tensor_desc* a) {
   CrossPlan p{};
   p.n_qtiles_a = (a->n_tokens + 255) / 256;
@@ -275,6 +296,8 @@ int launch_cross(const void* qv, const void* kv, const void* vv, const void* qa,
       (rc = make_map(&v2a.tmK, ka, audio, audio.n_tokens, "ka")) ||
       (rc = make_map(&v2a.tmV, va, audio, audio.n_tokens, "va")))
     return rc;
+  if ((rc = make_store_map(&v2a.tmO, o_video, video, video.n_tokens,
+                           attn_store_cols(kV2aQTiles), "o_video"))) return rc;
   v2a.o = (__nv_bfloat16*)o_video;
   v2a.o_st = video.stride_tok;
   v2a.o_sb = video.stride_batch;
@@ -413,6 +436,7 @@ int mmdit_joint_attn(const void* q, const void* k, const void* v, void* o, float
       (rc = make_map(&pr.tmK, k, *desc, desc->n_tokens, "k")) ||
       (rc = make_map(&pr.tmV, v, *desc, desc->n_tokens, "v")))
     return rc;
+  if ((rc = make_store_map(&pr.tmO, o, *desc, desc->n_tokens, attn_store_cols(kJointQTiles), "o"))) return rc;
   pr.o = (__nv_bfloat16*)o;
   pr.o_st = desc->stride_tok;
   pr.o_sb = desc->stride_batch;
@@ -426,7 +450,7 @@ int mmdit_joint_attn(const void* q, const void* k, const void* v, void* o, float
   pr.ctas = pr.n_qtiles * pr.H * pr.B;
   pr.mode = kModeDense;
   pr.rope_q = rope_q != nullptr;
-  p.q_tiles = 2;
+  p.q_tiles = kJointQTiles;
   p.persistent = 0;  // measured: one item per CTA is ~1% faster for long keys
   p.scale_log2 = scale * 1.4426950408889634f;
   p.layout = to_dev(layout);
