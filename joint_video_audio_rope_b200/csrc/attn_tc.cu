@@ -76,7 +76,7 @@ struct Cfg {
   // softmax warpgroups rise to kRegsHigh, keeping
   // 128 * (QT * kRegsHigh + kRegsLow) <= kThreads * kRegsLaunch.
   static constexpr int kRegsLaunch = (65536 / (kThreads * kMinBlocks)) / 8 * 8;
-  static constexpr int kRegsLow = QT == 2 ? 104 : 56;
+  static constexpr int kRegsLow = QT == 2 ? 104 : 64;
   static constexpr int kRegsHigh = ((kThreads * kRegsLaunch / 128 - kRegsLow) / QT) / 8 * 8;
   static_assert(128 * (QT * kRegsHigh + kRegsLow) <= kThreads * kRegsLaunch, "register split");
 };
@@ -122,28 +122,59 @@ struct Work {
   int g_first, g_nblk;
 };
 
-__device__ __forceinline__ int total_items(const AttnParams& P) {
-  return P.prob.ctas;
-}
 
-// k-th work item of this CTA: the CTA's own item, or (persistent launches)
-// items blockIdx.x + k * gridDim.x.
-template <bool PERSIST>
-__device__ __forceinline__ int item_of(const AttnParams&, int k, int n_items) {
-  if (!PERSIST) return k == 0 ? (int)blockIdx.x : n_items;
-  return (int)blockIdx.x + k * (int)gridDim.x;
-}
+// Position of a work item in the mixed radix (query tile, split, head, batch),
+// query tile fastest.
+struct ItemPos {
+  int qtile, split, h, b;
+};
 
-__device__ __forceinline__ Work decode_work(const AttnParams& P, int item, int rows) {
-  Work w;
-  int idx = item;
-  const AttnProblem& pr = P.prob;
-  w.qtile = idx % pr.n_qtiles;
-  idx /= pr.n_qtiles;
-  w.split = idx % pr.n_splits;
+__device__ __forceinline__ ItemPos item_pos(const AttnProblem& pr, int item) {
+  ItemPos p;
+  p.qtile = item % pr.n_qtiles;
+  int idx = item / pr.n_qtiles;
+  p.split = idx % pr.n_splits;
   idx /= pr.n_splits;
-  w.h = idx % pr.H;
-  w.b = idx / pr.H;
+  p.h = idx % pr.H;
+  p.b = idx / pr.H;
+  return p;
+}
+
+// The work items of this CTA: blockIdx.x and, in persistent launches, every
+// gridDim.x-th item after it.  The stride's digits are found once, so a step
+// is digit-wise addition with carry instead of four divisions; the walk ends
+// when the batch digit reaches B (item >= n_qtiles * n_splits * H * B).
+template <bool PERSIST>
+struct ItemWalk {
+  ItemPos cur, stride;
+  __device__ __forceinline__ explicit ItemWalk(const AttnProblem& pr)
+      : cur(item_pos(pr, (int)blockIdx.x)), stride(item_pos(pr, PERSIST ? (int)gridDim.x : 0)) {}
+  __device__ __forceinline__ bool more(const AttnProblem& pr) const { return cur.b < pr.B; }
+  __device__ __forceinline__ void next(const AttnProblem& pr) {
+    if (!PERSIST) {
+      cur.b = pr.B;
+      return;
+    }
+    const int q = cur.qtile + stride.qtile;
+    int cy = q >= pr.n_qtiles;
+    cur.qtile = cy ? q - pr.n_qtiles : q;
+    const int sp = cur.split + stride.split + cy;
+    cy = sp >= pr.n_splits;
+    cur.split = cy ? sp - pr.n_splits : sp;
+    const int h = cur.h + stride.h + cy;
+    cy = h >= pr.H;
+    cur.h = cy ? h - pr.H : h;
+    cur.b += stride.b + cy;
+  }
+};
+
+__device__ __forceinline__ Work decode_work(const AttnParams& P, const ItemPos& pos, int rows) {
+  Work w;
+  const AttnProblem& pr = P.prob;
+  w.qtile = pos.qtile;
+  w.split = pos.split;
+  w.h = pos.h;
+  w.b = pos.b;
   if (pr.mode == kModeDense) {
     w.q0 = w.qtile * rows;
     w.q_valid = min(rows, pr.Nq - w.q0);
@@ -263,7 +294,6 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + 8 * B_COUNT);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_items = PERSIST ? total_items(P) : (int)blockIdx.x + 1;
   int* err = P.err;
   const bool skip = *(volatile int*)err != 0;  // an earlier kernel timed out
 
@@ -305,9 +335,8 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
       bool ok = true;
       int ld = 0;  // ring loads issued so far (all items)
       int it = 0;  // items of this CTA so far
-      for (int item = item_of<PERSIST>(P, 0, n_items); item < n_items && ok;
-           item = item_of<PERSIST>(P, ++it, n_items)) {
-        const Work w = decode_work(P, item, C::kRows);
+      for (ItemWalk<PERSIST> wk(P.prob); wk.more(P.prob) && ok; wk.next(P.prob), ++it) {
+        const Work w = decode_work(P, wk.cur, C::kRows);
         const AttnProblem& pr = P.prob;
         if (it == 0) {
           tma_prefetch_desc(&pr.tmQ);
@@ -357,9 +386,8 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
       int cs = 0;   // ring loads consumed so far (all items)
       int pt = 0;   // key tiles processed so far (P barrier phases)
       int it = 0;
-      for (int item = item_of<PERSIST>(P, 0, n_items); item < n_items && ok;
-           item = item_of<PERSIST>(P, ++it, n_items)) {
-        const Work w = decode_work(P, item, C::kRows);
+      for (ItemWalk<PERSIST> wk(P.prob); wk.more(P.prob) && ok; wk.next(P.prob), ++it) {
+        const Work w = decode_work(P, wk.cur, C::kRows);
         const AttnProblem& pr = P.prob;
         const int nkv = w.nkv;
         const int qbar = pr.rope_q ? B_QREADY : B_QFULL;
@@ -435,9 +463,8 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
     bool ok = !skip;
     int st = 0;  // S tiles consumed so far (all items)
     int it = 0;
-    for (int item = item_of<PERSIST>(P, 0, n_items); item < n_items && ok;
-           item = item_of<PERSIST>(P, ++it, n_items)) {
-      const Work w = decode_work(P, item, C::kRows);
+    for (ItemWalk<PERSIST> wk(P.prob); wk.more(P.prob) && ok; wk.next(P.prob), ++it) {
+      const Work w = decode_work(P, wk.cur, C::kRows);
       const AttnProblem& pr = P.prob;
       const int nkv = w.nkv;
 
