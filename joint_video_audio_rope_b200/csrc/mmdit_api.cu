@@ -228,9 +228,11 @@ struct CrossPlan {
 };
 
 // Split of the video keys for the audio-query direction: enough splits that
-// the (few) audio query tiles x heads x batch fill two waves of the B200's 148
-// SMs, each split a whole number of 128-key tiles.
-constexpr int kCrossTargetCtas = 2 * 148;
+// the (few) audio query tiles x heads x batch fill one wave of the B200's 148
+// SMs, each split a whole number of 128-key tiles.  One wave of long items
+// measured faster than two waves of half-length items (less pipeline fill and
+// drain per key, half the partials to merge).
+constexpr int kCrossTargetCtas = 148;
 
 // Q tiles per CTA of the video-query direction (short key sequence): one tile,
 // two CTAs per SM (measured faster than two tiles with resident K/V).
