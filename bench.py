@@ -96,7 +96,7 @@ def dense_step_flops(w: WL.Workload) -> dict:
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only while the kernel
 # source is the one that was captured (sha1 of attn_tc.cu + common.cuh).
 NCU_TRAFFIC = {
-    "480p": {"src": "02951c1f1e606e13", "bytes": 845995008},  # profiles/attn_tc_joint_480p.md
+    "480p": {"src": "d0e11d9c8339b3b8", "bytes": 834778112},  # ncu, one joint launch
 }
 
 

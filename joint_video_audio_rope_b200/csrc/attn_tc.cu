@@ -106,7 +106,8 @@ enum {
   B_QEMPTY = 18,  // 2: last QK of the item done (Q buffer reusable)
   B_OEMPTY = 20,  // 2: epilogue has read O out of TMEM (128 arrivals)
   B_MMADONE = 22, // 1: every MMA of the CTA done (teardown)
-  B_COUNT = 23
+  B_PHALF = 23,   // 2: first 64 keys of the P tile written (128 arrivals)
+  B_COUNT = 25
 };
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0, 0);  // Q, K: K-major
@@ -238,6 +239,15 @@ __device__ __forceinline__ void mma_qk(uint32_t s_tmem, uint32_t q_smem, uint32_
 // tensor memory (16 bf16 per row = 8 columns per K step).  V is MN-major:
 // 64-channel halves are LBO = kHalfCol apart, 8-row groups SBO = 1024 apart,
 // and 16 key rows (one K step) are 2048 bytes.
+template <int K0, int K1>
+__device__ __forceinline__ void mma_pv_part(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem,
+                                            bool accumulate) {
+#pragma unroll
+  for (int kk = K0; kk < K1; ++kk) {
+    const uint64_t b = smem_desc_sw128(v_smem + kk * 2048, kHalfCol, 1024);
+    tc_mma_ts(o_tmem, p_tmem + kk * 8, b, kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
 __device__ __forceinline__ void mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem,
                                        bool accumulate) {
 #pragma unroll
@@ -303,6 +313,7 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
       mbar_init(bar(B_QREADY + t), 128);
       mbar_init(bar(B_SFULL + t), 1);
       mbar_init(bar(B_PFULL + t), 128);
+      mbar_init(bar(B_PHALF + t), 128);
       mbar_init(bar(B_OFULL + t), 1);
       mbar_init(bar(B_QEMPTY + t), 1);
       mbar_init(bar(B_OEMPTY + t), 128);
@@ -379,8 +390,12 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
     // Issue order per key tile j (t = Q tiles of the CTA):
     //   PV_t(j) then QK_t(j+1), tile after tile, so that P_t (which aliases S_t
     //   in TMEM) is consumed by PV_t before QK_t(j+1) overwrites S_t, and the
-    //   completion of QK_t(j+1) also implies PV_t(j) is done.  Across items the
-    //   first PV_t of an item waits until the epilogue has read O_t out.
+    //   completion of QK_t(j+1) also implies PV_t(j) is done.  PV_t(j) goes in
+    //   two halves: keys 0..63 as soon as the softmax has written that half of
+    //   P (p_half), keys 64..127 once the whole tile is written (p_full), so
+    //   the tensor core starts while the second half is still being
+    //   exponentiated.  Across items the first PV_t of an item waits until the
+    //   epilogue has read O_t out.
     if (lane == 0 && !skip) {
       bool ok = true;
       int cs = 0;   // ring loads consumed so far (all items)
@@ -416,11 +431,14 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
             if (!(ok = mbar_wait(bar(B_KVFULL + sv), ring_parity(2 * j + 1), err))) break;
 #pragma unroll
             for (int t = 0; t < QT; ++t) {
-              if (!(ok = mbar_wait(bar(B_PFULL + t), (pt + j) & 1, err))) break;
+              if (!(ok = mbar_wait(bar(B_PHALF + t), (pt + j) & 1, err))) break;
               if (j == 0 && it > 0 && !(ok = mbar_wait(bar(B_OEMPTY + t), (it - 1) & 1, err)))
                 break;
               tc_fence_after();
-              mma_pv(tmem + QT * 128 + t * 128, tmem + t * 128, v_smem, j > 0);
+              mma_pv_part<0, 4>(tmem + QT * 128 + t * 128, tmem + t * 128, v_smem, j > 0);
+              if (!(ok = mbar_wait(bar(B_PFULL + t), (pt + j) & 1, err))) break;
+              tc_fence_after();
+              mma_pv_part<4, 8>(tmem + QT * 128 + t * 128, tmem + t * 128, v_smem, true);
               if (t == QT - 1) tc_commit(bar(B_KVEMPTY + sv));
               if (more) {
                 if (t == 0) {
@@ -602,6 +620,11 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
             acc[i & 3] = add_f32x2(acc[i & 3], pack_f32x2(p0, p1));
           }
           tmem_st16(s_addr + c * 16, pk);  // P: 2 bf16 per column
+          if (c == 1) {  // keys 0..63 of P written: the first half of PV may start
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(B_PHALF + t));
+          }
         }
         tmem_wait_st();
         {
