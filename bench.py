@@ -96,7 +96,7 @@ def dense_step_flops(w: WL.Workload) -> dict:
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only while the kernel
 # source is the one that was captured (sha1 of attn_tc.cu + common.cuh).
 NCU_TRAFFIC = {
-    "480p": {"src": "d0e11d9c8339b3b8", "bytes": 834778112},  # ncu, one joint launch
+    "480p": {"src": "21f71342ae8922c8", "bytes": 837867008},  # ncu, one joint launch
 }
 
 
