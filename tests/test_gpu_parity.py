@@ -228,6 +228,13 @@ CROSS_CASES = {
                                                  WL.audio(218), WL.text(16)], batch=2),
     "split_kv": lambda: _custom("480p", [WL.video(21, 14, 16), WL.audio(218), WL.text(8)]),
     "short_audio": lambda: _custom("480p", [WL.video(4, 5, 7), WL.audio(3)]),
+    # enough work items that the persistent CTAs walk several each, carrying
+    # across query tile, split, head and batch: 5,120 video tokens x 5 heads x
+    # batch 2 = 400 video-query items on 296 CTAs; 1,000 audio tokens = 4 query
+    # tiles x 4 key splits x 5 heads x 2 = 160 audio-query items on 148 CTAs
+    "multi_item_b2": lambda: _custom("720p_cond_b2", [WL.video(1, 8, 16, t0=-1),
+                                                      WL.video(39, 8, 16), WL.audio(1000),
+                                                      WL.text(16)], heads=5, batch=2),
 }
 
 
