@@ -411,6 +411,35 @@ def run_gpu(args) -> int:
                for j, name in enumerate(["rope", "select" if sparse else "none",
                                          "sparse" if sparse else "joint", "cross"])}
 
+    # --------------------------------------------- text cross-attention
+    # The reinforced text cross-attention (video queries over the text keys)
+    # is a call of its own, outside the step the metric is defined on: timed
+    # here on its own, the same number of launches, after the same warm-up.
+    text_cross_ms = None
+    tx0, tx1 = WL._kind_range(w.segments, WL.SEG_TEXT)
+    if tx1 > tx0:
+        o_text = torch.empty_like(q)
+        dtx = M.desc_of(k[:, tx0:tx1])
+
+        def text_cross():
+            M.text_cross_attn(q[:, v0:v1], k[:, tx0:tx1], v[:, tx0:tx1], o_text[:, v0:v1], dv, dtx,
+                              scale, stream)
+
+        for _ in range(args.warmup):
+            text_cross()
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            text_cross()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        text_cross_ms = reduce_max(e0.elapsed_time(e1), world, dev) / args.steps
+        if M.device_status(stream) != 0:
+            raise RuntimeError("device status after the text cross-attention: " + M.last_error())
+
     # ---------------------------------------------------------- end to end
     pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
     hq, hk, hv = pin(x["q"]), pin(x["k"]), pin(x["v"])
@@ -481,6 +510,13 @@ def run_gpu(args) -> int:
                      "peak_source": f"bf16_tflops_sustained of {peak_src}"},
         "clocks": clocks,
     }
+    if text_cross_ms is not None:
+        tf = attn_flops(w.n_video, tx1 - tx0, w.head_dim, w.heads, w.batch)
+        line["text_cross"] = {"ms": round(text_cross_ms, 4), "flops": tf,
+                              "tflops": round(tf / (text_cross_ms / 1e3) / 1e12, 2),
+                              "frac": round(tf / (text_cross_ms / 1e3) / 1e12 / peak, 4),
+                              "text_tokens": tx1 - tx0, "launches": args.steps,
+                              "note": "separate call, not part of the step or its value"}
     if sparse:
         line["block_density"] = round(density, 4)
     if world == 1 and not args.no_cpu_baseline:

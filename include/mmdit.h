@@ -183,6 +183,23 @@ MMDIT_API size_t mmdit_av_cross_attn_workspace_size(const mmdit_tensor_desc* vid
                                           const mmdit_tensor_desc* audio);
 
 /*
+ * mmdit_text_cross_attn -- reinforced text cross-attention (digest step 3:
+ *   in every layer the video tokens query the text embedding, beside the
+ *   bidirectional audio<->video cross-attention):
+ *     o_video = softmax(qv kt^T * scale) vt     (video queries, text keys)
+ *   qv, o_video : device, described by `video` (N = video tokens, conditioning
+ *                 frames included); o_video may not alias qv
+ *   kt, vt      : device, described by `text` (N = text tokens, >= 1)
+ *   Both descriptors must agree on batch, heads, head_dim and dtype.  Inputs
+ *   are expected to be RoPE-rotated already (text tokens sit at position
+ *   (0, 0, 0), where the rotation is the identity).  No workspace.
+ *   Errors : EINVAL, EUNSUPPORTED, ECUDA.
+ */
+MMDIT_API int mmdit_text_cross_attn(const void* qv, const void* kt, const void* vt, void* o_video,
+                          const mmdit_tensor_desc* video, const mmdit_tensor_desc* text,
+                          float scale, mmdit_stream_t stream);
+
+/*
  * mmdit_av_cross_attn_noalloc -- the same cross-attention as
  *   mmdit_av_cross_attn, for callers that cannot allocate device memory or
  *   size a workspace (a plugin inside a runtime that owns every device

@@ -248,14 +248,6 @@ __device__ __forceinline__ void mma_pv_part(uint32_t o_tmem, uint32_t p_tmem, ui
     tc_mma_ts(o_tmem, p_tmem + kk * 8, b, kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
-__device__ __forceinline__ void mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem,
-                                       bool accumulate) {
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    const uint64_t b = smem_desc_sw128(v_smem + kk * 2048, kHalfCol, 1024);
-    tc_mma_ts(o_tmem, p_tmem + kk * 8, b, kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
-  }
-}
 
 // Rotate this thread's Q row (row r of the tile at q_smem) in place by the
 // 3D RoPE angles of token `tok`.

@@ -234,12 +234,12 @@ struct CrossPlan {
 // drain per key, half the partials to merge).
 constexpr int kCrossTargetCtas = 148;
 
-// Q tiles per CTA of the video-query direction (short key sequence): one tile,
-// two CTAs per SM (measured faster than two tiles with resident K/V).
-#ifndef MMDIT_V2A_QTILES
-#define MMDIT_V2A_QTILES 1
+// Q tiles per CTA of video queries over a short key sequence (audio, text):
+// one tile, two CTAs per SM (measured faster than two tiles with resident K/V).
+#ifndef MMDIT_SHORT_KV_QTILES
+#define MMDIT_SHORT_KV_QTILES 1
 #endif
-constexpr int kV2aQTiles = MMDIT_V2A_QTILES;
+constexpr int kShortKvQTiles = MMDIT_SHORT_KV_QTILES;
 
 // Q tiles per CTA of the dense joint attention: two, one CTA per SM.
 constexpr int kJointQTiles = 2;
@@ -257,6 +257,39 @@ CrossPlan plan_cross(const mmdit_tensor_desc* v, const mmdit_tensor_desc* a) {
   p.part_o_bytes = align256(rows * 128 * sizeof(float));
   p.part_ml_bytes = align256(rows * 2 * sizeof(float));
   return p;
+}
+
+// Video queries over a short key sequence (the audio or the text tokens):
+// persistent CTAs of kShortKvQTiles Q tiles (two CTAs per SM for one tile, so
+// that each hides the other's load and epilogue latency), all key tiles in one
+// work item, bf16 O written through the output tensor map.
+int short_kv_params(AttnParams& p, const void* q, const void* k, const void* v, void* o,
+                    const mmdit_tensor_desc& qd, const mmdit_tensor_desc& kd, float scale,
+                    int* err, const char* qname, const char* kname) {
+  int rc;
+  AttnProblem& pr = p.prob;
+  if ((rc = make_map(&pr.tmQ, q, qd, qd.n_tokens, qname)) ||
+      (rc = make_map(&pr.tmK, k, kd, kd.n_tokens, kname)) ||
+      (rc = make_map(&pr.tmV, v, kd, kd.n_tokens, kname)) ||
+      (rc = make_store_map(&pr.tmO, o, qd, qd.n_tokens, attn_store_cols(kShortKvQTiles), qname)))
+    return rc;
+  pr.o = (__nv_bfloat16*)o;
+  pr.o_st = qd.stride_tok;
+  pr.o_sb = qd.stride_batch;
+  pr.Nq = qd.n_tokens;
+  pr.Nkv = kd.n_tokens;
+  pr.H = qd.heads;
+  pr.B = qd.batch;
+  pr.n_qtiles = (qd.n_tokens + 128 * kShortKvQTiles - 1) / (128 * kShortKvQTiles);
+  pr.n_splits = 1;
+  pr.kv_per_split = ((kd.n_tokens + 127) / 128) * 128;
+  pr.ctas = pr.n_qtiles * pr.H * pr.B;
+  pr.mode = kModeDense;
+  p.q_tiles = kShortKvQTiles;
+  p.persistent = 1;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.err = err;
+  return MMDIT_OK;
 }
 
 int launch_cross(const void* qv, const void* kv, const void* vv, const void* qa, const void* ka,
@@ -290,32 +323,10 @@ int launch_cross(const void* qv, const void* kv, const void* vv, const void* qa,
   pa.persistent = 1;
   pa.scale_log2 = scale * 1.4426950408889634f;
   pa.err = err;
-  // video queries over the (short) audio keys: persistent CTAs, two per SM,
-  // hide each other's load and epilogue latency
+  // video queries over the (short) audio keys
   AttnParams pv{};
-  AttnProblem& v2a = pv.prob;
-  if ((rc = make_map(&v2a.tmQ, qv, video, video.n_tokens, "qv")) ||
-      (rc = make_map(&v2a.tmK, ka, audio, audio.n_tokens, "ka")) ||
-      (rc = make_map(&v2a.tmV, va, audio, audio.n_tokens, "va")))
+  if ((rc = short_kv_params(pv, qv, ka, va, o_video, video, audio, scale, err, "video", "audio")))
     return rc;
-  if ((rc = make_store_map(&v2a.tmO, o_video, video, video.n_tokens,
-                           attn_store_cols(kV2aQTiles), "o_video"))) return rc;
-  v2a.o = (__nv_bfloat16*)o_video;
-  v2a.o_st = video.stride_tok;
-  v2a.o_sb = video.stride_batch;
-  v2a.Nq = video.n_tokens;
-  v2a.Nkv = audio.n_tokens;
-  v2a.H = video.heads;
-  v2a.B = video.batch;
-  v2a.n_qtiles = (video.n_tokens + 128 * kV2aQTiles - 1) / (128 * kV2aQTiles);
-  v2a.n_splits = 1;
-  v2a.kv_per_split = ((audio.n_tokens + 127) / 128) * 128;
-  v2a.ctas = v2a.n_qtiles * v2a.H * v2a.B;
-  v2a.mode = kModeDense;
-  pv.q_tiles = kV2aQTiles;
-  pv.persistent = 1;
-  pv.scale_log2 = pa.scale_log2;
-  pv.err = err;
   cudaError_t e = launch_attn_tc(pa, s);
   if (e == cudaSuccess) e = launch_attn_tc(pv, s);
   if (e == cudaSuccess)
@@ -513,6 +524,43 @@ int mmdit_av_cross_attn(const void* qv, const void* kv, const void* vv, const vo
   return launch_cross(qv, kv, vv, qa, ka, va, o_video, o_audio, *video, *audio, scale, c.splits,
                       c.kv_per_split, reinterpret_cast<float*>(workspace),
                       reinterpret_cast<float*>(static_cast<char*>(workspace) + c.part_o_bytes), s);
+}
+
+int mmdit_text_cross_attn(const void* qv, const void* kt, const void* vt, void* o_video,
+                          const mmdit_tensor_desc* video, const mmdit_tensor_desc* text,
+                          float scale, mmdit_stream_t stream) {
+  int rc;
+  if ((rc = check_desc(video, "video")) || (rc = check_desc(text, "text"))) return rc;
+  if (video->batch != text->batch || video->heads != text->heads ||
+      video->head_dim != text->head_dim || video->dtype != text->dtype)
+    return fail(MMDIT_EINVAL, "text_cross: video and text descriptors disagree");
+  const void* ptrs[4] = {qv, kt, vt, o_video};
+  for (const void* p : ptrs) {
+    if (p == nullptr) return fail(MMDIT_EINVAL, "text_cross: every tensor must be non-NULL");
+    if (!aligned16(p)) return fail(MMDIT_EINVAL, "text_cross: tensors must be 16-byte aligned");
+  }
+  if (o_video == qv) return fail(MMDIT_EINVAL, "text_cross: o_video aliases qv");
+  if (text->n_tokens < 1) return fail(MMDIT_EINVAL, "text_cross: at least one text token");
+  if (!(scale > 0.f) || !isfinite(scale)) return fail(MMDIT_EINVAL, "text_cross: scale must be > 0");
+  if (video->n_tokens == 0) return MMDIT_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (video->dtype == MMDIT_F32) {
+    F32AttnArgs a{(const float*)qv, (const float*)kt, (const float*)vt, (float*)o_video, nullptr,
+                  video->batch, video->heads, video->head_dim, video->n_tokens, text->n_tokens,
+                  video->stride_tok, video->stride_batch, text->stride_tok, text->stride_batch,
+                  text->stride_tok, text->stride_batch, video->stride_tok, video->stride_batch,
+                  scale};
+    cudaError_t e = launch_attn_f32(a, s);
+    return e == cudaSuccess ? MMDIT_OK : cuda_fail(e, "attn_f32 launch");
+  }
+  if ((rc = check_sm100())) return rc;
+  int* err = device_error_flag();
+  if (err == nullptr) return fail(MMDIT_ECUDA, "device error flag unavailable");
+  AttnParams p{};
+  if ((rc = short_kv_params(p, qv, kt, vt, o_video, *video, *text, scale, err, "video", "text")))
+    return rc;
+  cudaError_t e = launch_attn_tc(p, s);
+  return e == cudaSuccess ? MMDIT_OK : cuda_fail(e, "text_cross launch");
 }
 
 size_t mmdit_block_select_workspace_size(const mmdit_tensor_desc* desc, const mmdit_layout* layout) {

@@ -63,6 +63,7 @@ _SIGS = {
     "mmdit_av_cross_attn": (C.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _D, _D, C.c_float, _P,
                                       C.c_size_t, _P]),
     "mmdit_av_cross_attn_workspace_size": (C.c_size_t, [_D, _D]),
+    "mmdit_text_cross_attn": (C.c_int, [_P, _P, _P, _P, _D, _D, C.c_float, _P]),
     "mmdit_av_cross_attn_noalloc": (C.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _D, _D, C.c_float,
                                               _P]),
     "mmdit_block_select": (C.c_int, [_P, _P, _D, _L, C.c_int, C.c_float, C.c_float, C.c_int,
@@ -190,6 +191,12 @@ def av_cross_attn(qv, kv, vv, qa, ka, va, o_video, o_audio, video: TensorDesc,
 
 def av_cross_attn_workspace_size(video: TensorDesc, audio: TensorDesc) -> int:
     return _lib.mmdit_av_cross_attn_workspace_size(C.byref(video), C.byref(audio))
+
+
+def text_cross_attn(qv, kt, vt, o_video, video: TensorDesc, text: TensorDesc, scale: float,
+                    stream=None) -> None:
+    _check(_lib.mmdit_text_cross_attn(_ptr(qv), _ptr(kt), _ptr(vt), _ptr(o_video), C.byref(video),
+                                      C.byref(text), scale, _stream(stream)))
 
 
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024  # MMDIT_NOALLOC_SCRATCH_BYTES

@@ -246,6 +246,14 @@ def av_cross_attn(qv, kv, vv, qa, ka, va, scale):
     return o_v, o_a
 
 
+def text_cross_attn(qv, kt, vt, scale):
+    """Reinforced text cross-attention ([SKY-D] step 3: in every layer the
+    video tokens query the text embedding): softmax(qv kt^T * scale) vt per
+    (batch, head), no mask.  Returns o_video."""
+    o_v, _ = attn_bshd(qv, kt, vt, scale)
+    return o_v
+
+
 # ---------------------------------------------------------------------------
 # a5 - a7: block-sparse mode
 # ---------------------------------------------------------------------------

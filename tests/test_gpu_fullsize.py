@@ -1,6 +1,7 @@
 """Full-size parity: the benchmark workloads at their full sizes, run through
 the same C-ABI calls and launch configuration that bench.py times, checked
-against the fp64 oracle on sampled outputs it can compute one by one.
+against the fp64 oracle on sampled outputs it can compute one by one (the
+text cross-attention, a call of its own, runs in the same dense step).
 
 Sampled rows per (batch, head): seeded random query rows, the first and last
 rows of the sequence and of every segment (the edge tiles, conditioning
@@ -77,21 +78,27 @@ def _run_dense_step(M, w, x):
     ws = torch.empty(n, dtype=torch.uint8, device="cuda")
     M.av_cross_attn(q[:, v0:v1], k[:, v0:v1], v[:, v0:v1], q[:, a0:a1], k[:, a0:a1], v[:, a0:a1],
                     oc[:, v0:v1], oc[:, a0:a1], dv, da, scale, ws, n)
+    # reinforced text cross-attention: video queries over the text keys
+    t0, t1 = WL._kind_range(w.segments, WL.SEG_TEXT)
+    ot = torch.empty_like(q)
+    M.text_cross_attn(q[:, v0:v1], k[:, t0:t1], v[:, t0:t1], ot[:, v0:v1], dv,
+                      M.desc_of(k[:, t0:t1]), scale)
     torch.cuda.synchronize()
     assert M.device_status() == M.OK
-    return q, k, o, oc
+    return q, k, o, oc, ot
 
 
 @pytest.mark.parametrize("name", ["480p", "720p", "720p_cond_b2"])
 def test_dense_workload_full_size(M, name):
     w = WL.WORKLOADS[name]
     x = WL.generate(w)
-    q, k, o, oc = _run_dense_step(M, w, x)
+    q, k, o, oc, ot = _run_dense_step(M, w, x)
     rng = np.random.default_rng(1234)
     pos = O.positions(oracle_layout(w.segments))
     scale = 1 / math.sqrt(128)
     v0, v1 = w.video_range()
     a0, a1 = w.audio_range()
+    t0, t1 = WL._kind_range(w.segments, WL.SEG_TEXT)
     for b in range(w.batch):
         kk = O.rope(WL.as_f64(x["k"][b], "bf16"), pos, w.theta)        # every key
         vv = WL.as_f64(x["v"][b], "bf16")
@@ -114,6 +121,11 @@ def test_dense_workload_full_size(M, name):
         for h in range(w.heads):
             ref_v[:, h], _ = O.attn(qr[sel, h], kk[a0:a1, h], vv[a0:a1, h], scale)
         assert_close(got_v[sel], ref_v, "bf16", f"{name} cross v<-a b{b}")
+        # text cross: the same sampled video rows over the text keys
+        ref_t = np.zeros((len(vr), w.heads, 128))
+        for h in range(w.heads):
+            ref_t[:, h], _ = O.attn(qr[sel, h], kk[t0:t1, h], vv[t0:t1, h], scale)
+        assert_close(_f64(ot[b, vr]), ref_t, "bf16", f"{name} text cross b{b}")
         # cross: every audio row over the video keys
         qa = bf16_round(O.rope(WL.as_f64(x["q"][b, a0:a1], "bf16"), pos[a0:a1], w.theta))
         ref_a = np.zeros((a1 - a0, w.heads, 128))

@@ -249,6 +249,82 @@ def test_cross_bf16(M, case):
     assert_close(to_host_f64(oa), ra, "bf16", "cross a<-v")
 
 
+# ------------------------------------------------------ text cross-attention
+
+def _text_range(w):
+    return WL._kind_range(w.segments, WL.SEG_TEXT)
+
+
+def _text_cross(M, w, dev):
+    v0, v1 = w.video_range()
+    t0, t1 = _text_range(w)
+    qv = dev["q"][:, v0:v1]
+    kt, vt = dev["k"][:, t0:t1], dev["v"][:, t0:t1]
+    o_full = torch.full_like(dev["q"], float("nan"))
+    ov = o_full[:, v0:v1]
+    M.text_cross_attn(qv, kt, vt, ov, M.desc_of(qv), M.desc_of(kt), 1 / math.sqrt(w.head_dim))
+    torch.cuda.synchronize()
+    return ov, o_full
+
+
+def _text_cross_oracle(host, w):
+    v0, v1 = w.video_range()
+    t0, t1 = _text_range(w)
+    return O.text_cross_attn(host["q"][:, v0:v1], host["k"][:, t0:t1], host["v"][:, t0:t1],
+                             1 / math.sqrt(w.head_dim))
+
+
+def test_text_cross_f32_tiny(M):
+    w = WL.WORKLOADS["tiny_f32"]
+    _, host, dev = _make(w)
+    ov, _ = _text_cross(M, w, dev)
+    assert_close(to_host_f64(ov), _text_cross_oracle(host, w), "f32", "text cross")
+
+
+TEXT_CASES = {
+    # 512 text tokens (four key tiles), 4,704 video tokens (ragged last tile)
+    "text512": lambda: _custom("480p", [WL.video(21, 14, 16), WL.audio(218), WL.text(512)]),
+    # a single partial key tile
+    "short_text": lambda: _custom("480p", [WL.video(4, 5, 7), WL.audio(9), WL.text(3)]),
+    # several items per persistent CTA, batch 2: 5,120 x 5 heads x 2 = 400
+    # items on 296 CTAs; 300 text tokens (3 key tiles, the last partial)
+    "multi_item_b2": lambda: _custom("720p_cond_b2", [WL.video(1, 8, 16, t0=-1),
+                                                      WL.video(39, 8, 16), WL.audio(218),
+                                                      WL.text(300)], heads=5, batch=2),
+}
+
+
+@pytest.mark.parametrize("case", list(TEXT_CASES))
+def test_text_cross_bf16(M, case):
+    w = TEXT_CASES[case]()
+    _, host, dev = _make(w)
+    ov, o_full = _text_cross(M, w, dev)
+    assert M.device_status() == 0
+    assert_close(to_host_f64(ov), _text_cross_oracle(host, w), "bf16", "text cross")
+    # nothing outside the video rows of the output buffer is written
+    v0, v1 = w.video_range()
+    rest = torch.cat([o_full[:, :v0], o_full[:, v1:]], dim=1)
+    assert bool(torch.isnan(rest.float()).all())
+
+
+def test_text_cross_rejects_bad_arguments(M):
+    w = TEXT_CASES["short_text"]()
+    _, _, dev = _make(w)
+    v0, v1 = w.video_range()
+    t0, t1 = _text_range(w)
+    qv, kt, vt = dev["q"][:, v0:v1], dev["k"][:, t0:t1], dev["v"][:, t0:t1]
+    ov = torch.empty_like(qv)
+    dv, dt = M.desc_of(qv), M.desc_of(kt)
+    with pytest.raises(M.MmditError):
+        M.text_cross_attn(qv, kt, vt, qv, dv, dt, 0.1)  # output aliases the queries
+    bad = M.desc_of(kt)
+    bad.heads = dv.heads + 1
+    with pytest.raises(M.MmditError):
+        M.text_cross_attn(qv, kt, vt, ov, dv, bad, 0.1)  # descriptors disagree
+    with pytest.raises(M.MmditError):
+        M.text_cross_attn(qv, kt, vt, ov, dv, dt, 0.0)  # scale must be > 0
+
+
 # ------------------------------------------------------------ block-sparse mode
 
 SPARSE_CASES = {

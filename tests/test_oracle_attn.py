@@ -106,3 +106,31 @@ def test_av_cross_directions():
     # o_video rows are convex combinations of audio V rows
     assert np.all(ov <= va.max(axis=1, keepdims=True) + 1e-12)
     assert np.all(ov >= va.min(axis=1, keepdims=True) - 1e-12)
+
+
+def test_text_cross_closed_forms():
+    qv, kt, vt = _r((2, 9, 3, 8), 31), _r((2, 4, 3, 8), 32), _r((2, 4, 3, 8), 33)
+    o = O.text_cross_attn(qv, kt, vt, 0.4)
+    assert o.shape == qv.shape
+    # one text token: every video query returns that token's value row
+    o1 = O.text_cross_attn(qv, kt[:, :1], vt[:, :1], 0.4)
+    assert np.allclose(o1, np.broadcast_to(vt[:, :1], qv.shape))
+    # identical text keys: uniform weights, the mean of the value rows
+    ksame = np.broadcast_to(kt[:, :1], kt.shape).copy()
+    om = O.text_cross_attn(qv, ksame, vt, 0.4)
+    assert np.allclose(om, np.broadcast_to(vt.mean(axis=1, keepdims=True), qv.shape))
+    # worked value with two keys: q = a e0, k0 = e0, k1 = 0 -> weights
+    # (e^(a s), 1) / (e^(a s) + 1)
+    a, s = 2.5, 0.4
+    q = np.zeros((1, 1, 1, 8)); q[0, 0, 0, 0] = a
+    k = np.zeros((1, 2, 1, 8)); k[0, 0, 0, 0] = 1.0
+    v = _r((1, 2, 1, 8), 34)
+    w0 = math.exp(a * s) / (math.exp(a * s) + 1.0)
+    assert np.allclose(O.text_cross_attn(q, k, v, s)[0, 0, 0], w0 * v[0, 0, 0] + (1 - w0) * v[0, 1, 0])
+    # permuting the text tokens (keys with their values) changes nothing
+    perm = np.array([2, 0, 3, 1])
+    assert np.allclose(O.text_cross_attn(qv, kt[:, perm], vt[:, perm], 0.4), o)
+    # heads are independent: another head's text keys do not move this head
+    kt2 = kt.copy(); kt2[:, :, 1] *= -3.0
+    o2 = O.text_cross_attn(qv, kt2, vt, 0.4)
+    assert np.array_equal(o2[:, :, 0], o[:, :, 0]) and np.array_equal(o2[:, :, 2], o[:, :, 2])
