@@ -440,6 +440,35 @@ def run_gpu(args) -> int:
         if M.device_status(stream) != 0:
             raise RuntimeError("device status after the text cross-attention: " + M.last_error())
 
+    # ------------------------- mask-guided region-restricted attention
+    # Workloads that carry the mask M also time the Refiner's region-restricted
+    # attention (rows of masked video tokens only), as a separate call.
+    masked_ms = None
+    if w.mask and not sparse:
+        o_mask = torch.empty_like(q)
+        mask_dev = torch.from_numpy(x["mask"]).to(dev)
+        nmw = M.masked_joint_attn_workspace_size(desc, lay)
+        ws_mask = torch.empty(nmw, dtype=torch.uint8, device=dev)
+
+        def masked():
+            M.masked_joint_attn(q, k, v, o_mask, desc, lay, scale, mask_dev, ws_mask, nmw, stream)
+
+        for _ in range(args.warmup):
+            masked()
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            masked()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        masked_ms = reduce_max(e0.elapsed_time(e1), world, dev) / args.steps
+        if M.device_status(stream) != 0:
+            raise RuntimeError("device status after the masked attention: " + M.last_error())
+        del ws_mask, o_mask
+
     # ---------------------------------------------------------- end to end
     pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
     hq, hk, hv = pin(x["q"]), pin(x["k"]), pin(x["v"])
@@ -517,6 +546,15 @@ def run_gpu(args) -> int:
                               "frac": round(tf / (text_cross_ms / 1e3) / 1e12 / peak, 4),
                               "text_tokens": tx1 - tx0, "launches": args.steps,
                               "note": "separate call, not part of the step or its value"}
+    if masked_ms is not None:
+        n_rows = int(np.count_nonzero(x["mask"]))  # one mask entry per video token
+        mf = 4.0 * n_rows * w.n_tokens * w.head_dim * w.heads
+        line["masked_joint"] = {"ms": round(masked_ms, 4), "flops": mf,
+                                "tflops": round(mf / (masked_ms / 1e3) / 1e12, 2),
+                                "frac": round(mf / (masked_ms / 1e3) / 1e12 / peak, 4),
+                                "masked_rows": n_rows, "launches": args.steps,
+                                "note": "separate call (rows of masked video tokens over every "
+                                        "key), not part of the step or its value"}
     if sparse:
         line["block_density"] = round(density, 4)
     if world == 1 and not args.no_cpu_baseline:

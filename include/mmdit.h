@@ -200,6 +200,34 @@ MMDIT_API int mmdit_text_cross_attn(const void* qv, const void* kt, const void* 
                           float scale, mmdit_stream_t stream);
 
 /*
+ * mmdit_masked_joint_attn -- mask-guided region-restricted attention of the
+ *   Refiner (blog section 4.2: with a spatial mask, only the target region is
+ *   refined): for every video token whose mask value is non-zero, its row of
+ *   O = softmax(Q K^T * scale) V over all tokens of its batch item (as in
+ *   mmdit_joint_attn); every other row of o is left as it was.
+ *   q, k, v, o : device [B, N, heads, 128] bf16 described by `desc`, Q and K
+ *                already rotated (o may not alias q, k or v).
+ *   layout     : segment table; video segments in raster order, all with the
+ *                same H and W.
+ *   mask       : device uint8 [B, F, H, W], F = frames of all video segments
+ *                in sequence order (the binary mask M of digest step 2);
+ *                mask_elems must equal B*F*H*W (0 and NULL allowed when the
+ *                layout has no video token).
+ *   workspace  : mmdit_masked_joint_attn_workspace_size(desc, layout) bytes,
+ *                256-byte aligned: the row lists and compact copies of the
+ *                masked Q and O rows (sized for every video token, since the
+ *                count is only known on the device).
+ *   Errors     : EINVAL, EUNSUPPORTED (fp32, block-major video), EWORKSPACE,
+ *                ECUDA.
+ */
+MMDIT_API int mmdit_masked_joint_attn(const void* q, const void* k, const void* v, void* o,
+                            const mmdit_tensor_desc* desc, const mmdit_layout* layout,
+                            float scale, const uint8_t* mask, int64_t mask_elems,
+                            void* workspace, size_t ws_bytes, mmdit_stream_t stream);
+MMDIT_API size_t mmdit_masked_joint_attn_workspace_size(const mmdit_tensor_desc* desc,
+                                              const mmdit_layout* layout);
+
+/*
  * mmdit_av_cross_attn_noalloc -- the same cross-attention as
  *   mmdit_av_cross_attn, for callers that cannot allocate device memory or
  *   size a workspace (a plugin inside a runtime that owns every device

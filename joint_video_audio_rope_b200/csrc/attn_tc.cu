@@ -177,11 +177,13 @@ __device__ __forceinline__ Work decode_work(const AttnParams& P, const ItemPos& 
   w.h = pos.h;
   w.b = pos.b;
   if (pr.mode == kModeDense) {
+    const int nq = pr.q_count != nullptr ? min(pr.Nq, pr.q_count[w.b]) : pr.Nq;
     w.q0 = w.qtile * rows;
-    w.q_valid = min(rows, pr.Nq - w.q0);
+    w.q_valid = min(rows, nq - w.q0);
     w.kv_lo = w.split * pr.kv_per_split;
     w.kv_hi = min(pr.Nkv, w.kv_lo + pr.kv_per_split);
-    w.nkv = w.kv_hi > w.kv_lo ? (w.kv_hi - w.kv_lo + 127) / 128 : 0;
+    // an item past the valid rows of its batch item computes nothing
+    w.nkv = (w.kv_hi > w.kv_lo && w.q_valid > 0) ? (w.kv_hi - w.kv_lo + 127) / 128 : 0;
     w.ubase = 0;
     w.g_first = w.g_nblk = 0;
   } else {

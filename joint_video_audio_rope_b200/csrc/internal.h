@@ -50,6 +50,8 @@ struct AttnProblem {
   int ucap;
   int vT, vH, vW;             // block-major video grid (sparse mode)
   int rope_q;                 // rotate Q tiles in shared memory after loading
+  const int* q_count;         // dense mode, optional: valid query rows per batch item
+                              // (device; rows from q_count[b] on are not computed)
 };
 
 // One attention problem per launch: every field of `prob` sits at a fixed
@@ -108,6 +110,7 @@ int fail(int code, const char* fmt, ...);  // sets the thread-local message
 int cuda_fail(cudaError_t e, const char* what);
 bool aligned16(const void* p);
 int check_desc(const mmdit_tensor_desc* d, const char* name);
+int check_layout(const mmdit_layout* L, int n_tokens);  // segments sum to n_tokens, valid kinds
 int make_map(CUtensorMap* m, const void* base, const mmdit_tensor_desc& d, int n_tokens,
              const char* name);
 // Store map of a bf16 [B, N, heads, 128] output with the strides of `d`: box

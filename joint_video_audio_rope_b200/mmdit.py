@@ -64,6 +64,9 @@ _SIGS = {
                                       C.c_size_t, _P]),
     "mmdit_av_cross_attn_workspace_size": (C.c_size_t, [_D, _D]),
     "mmdit_text_cross_attn": (C.c_int, [_P, _P, _P, _P, _D, _D, C.c_float, _P]),
+    "mmdit_masked_joint_attn": (C.c_int, [_P, _P, _P, _P, _D, _L, C.c_float, _P, C.c_int64, _P,
+                                          C.c_size_t, _P]),
+    "mmdit_masked_joint_attn_workspace_size": (C.c_size_t, [_D, _L]),
     "mmdit_av_cross_attn_noalloc": (C.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _D, _D, C.c_float,
                                               _P]),
     "mmdit_block_select": (C.c_int, [_P, _P, _D, _L, C.c_int, C.c_float, C.c_float, C.c_int,
@@ -197,6 +200,18 @@ def text_cross_attn(qv, kt, vt, o_video, video: TensorDesc, text: TensorDesc, sc
                     stream=None) -> None:
     _check(_lib.mmdit_text_cross_attn(_ptr(qv), _ptr(kt), _ptr(vt), _ptr(o_video), C.byref(video),
                                       C.byref(text), scale, _stream(stream)))
+
+
+def masked_joint_attn(q, k, v, o, desc: TensorDesc, layout: Layout, scale: float, mask,
+                      workspace=None, ws_bytes: int = 0, stream=None) -> None:
+    n = 0 if mask is None else mask.numel()
+    _check(_lib.mmdit_masked_joint_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), C.byref(desc),
+                                        C.byref(layout), scale, _ptr(mask), n, _ptr(workspace),
+                                        ws_bytes, _stream(stream)))
+
+
+def masked_joint_attn_workspace_size(desc: TensorDesc, layout: Layout) -> int:
+    return _lib.mmdit_masked_joint_attn_workspace_size(C.byref(desc), C.byref(layout))
 
 
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024  # MMDIT_NOALLOC_SCRATCH_BYTES

@@ -254,6 +254,45 @@ def text_cross_attn(qv, kt, vt, scale):
     return o_v
 
 
+def masked_rows(layout: Layout, mask: np.ndarray) -> List[np.ndarray]:
+    """Per batch item, the sequence indices of the video tokens whose mask
+    value is non-zero, in sequence order.  ``mask`` is [B, F, H, W] over the
+    frames of all video segments in sequence order (the binary mask M of
+    [SKY-D] step 2); video segments are in raster order."""
+    out = []
+    for b in range(mask.shape[0]):
+        rows = []
+        start, frame = 0, 0
+        for s in layout.segments:
+            if s.kind == SEG_VIDEO:
+                if s.order != ORDER_RASTER:
+                    raise ValueError("masked rows need raster-order video segments")
+                for t in range(s.T):
+                    for h in range(s.H):
+                        for w in range(s.W):
+                            if mask[b, frame + t, h, w] != 0:
+                                rows.append(start + (t * s.H + h) * s.W + w)
+                frame += s.T
+            start += s.n_tokens
+        out.append(np.array(rows, dtype=np.int64))
+    return out
+
+
+def masked_joint_attn(q, k, v, o_init, rows, scale):
+    """Mask-guided region-restricted attention ([SKY-B] 4.2: with a spatial
+    mask the Refiner refines only the target region): the rows ``rows[b]`` of
+    the output get their joint-attention row over every key of batch item b;
+    every other row keeps its value from ``o_init``."""
+    o = np.array(o_init, dtype=np.float64, copy=True)
+    for b in range(q.shape[0]):
+        r = rows[b]
+        if len(r) == 0:
+            continue
+        for h in range(q.shape[2]):
+            o[b, r, h], _ = attn(q[b, r, h], k[b, :, h], v[b, :, h], scale)
+    return o
+
+
 # ---------------------------------------------------------------------------
 # a5 - a7: block-sparse mode
 # ---------------------------------------------------------------------------

@@ -1,7 +1,8 @@
 """Full-size parity: the benchmark workloads at their full sizes, run through
 the same C-ABI calls and launch configuration that bench.py times, checked
 against the fp64 oracle on sampled outputs it can compute one by one (the
-text cross-attention, a call of its own, runs in the same dense step).
+text cross-attention, a call of its own, runs in the same dense step, and so
+does the mask-guided region-restricted attention on the workload with a mask).
 
 Sampled rows per (batch, head): seeded random query rows, the first and last
 rows of the sequence and of every segment (the edge tiles, conditioning
@@ -83,16 +84,26 @@ def _run_dense_step(M, w, x):
     ot = torch.empty_like(q)
     M.text_cross_attn(q[:, v0:v1], k[:, t0:t1], v[:, t0:t1], ot[:, v0:v1], dv,
                       M.desc_of(k[:, t0:t1]), scale)
+    om = None
+    if w.mask:
+        # mask-guided region-restricted attention over the same rotated Q/K;
+        # unmasked rows keep the fill value
+        om = torch.full_like(q, 7.0)
+        md = torch.from_numpy(x["mask"]).cuda()
+        nm = M.masked_joint_attn_workspace_size(desc, lay)
+        wm = torch.empty(nm, dtype=torch.uint8, device="cuda")
+        M.masked_joint_attn(q, k, v, om, desc, lay, scale, md, wm, nm)
     torch.cuda.synchronize()
     assert M.device_status() == M.OK
-    return q, k, o, oc, ot
+    return q, k, o, oc, ot, om
 
 
 @pytest.mark.parametrize("name", ["480p", "720p", "720p_cond_b2"])
 def test_dense_workload_full_size(M, name):
     w = WL.WORKLOADS[name]
     x = WL.generate(w)
-    q, k, o, oc, ot = _run_dense_step(M, w, x)
+    q, k, o, oc, ot, om = _run_dense_step(M, w, x)
+    mrows = O.masked_rows(oracle_layout(w.segments), x["mask"]) if w.mask else None
     rng = np.random.default_rng(1234)
     pos = O.positions(oracle_layout(w.segments))
     scale = 1 / math.sqrt(128)
@@ -114,6 +125,13 @@ def test_dense_workload_full_size(M, name):
         for h in range(w.heads):
             ref_o[:, h], _ = O.attn(qr[:, h], kk[:, h], vv[:, h], scale)
         assert_close(got_o, ref_o, "bf16", f"{name} joint b{b}")
+        if om is not None:
+            # masked rows are joint-attention rows; the others keep the fill
+            inm = np.isin(rows, mrows[b])
+            assert inm.any() and (~inm).any()
+            got_m = _f64(om[b, rows])
+            assert_close(got_m[inm], ref_o[inm], "bf16", f"{name} masked rows b{b}")
+            assert np.all(got_m[~inm] == 7.0), f"{name} unmasked rows changed b{b}"
         # cross: sampled video rows over the audio keys
         vr = rows[(rows >= v0) & (rows < v1)]
         sel = np.isin(rows, vr)

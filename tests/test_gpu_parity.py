@@ -325,6 +325,93 @@ def test_text_cross_rejects_bad_arguments(M):
         M.text_cross_attn(qv, kt, vt, ov, dv, dt, 0.0)  # scale must be > 0
 
 
+# ----------------------------------------- mask-guided region-restricted attention
+
+def _box_mask(w, seed, kind):
+    vids = [sg for sg in w.segments if sg["kind"] == WL.SEG_VIDEO]
+    F = sum(sg["T"] for sg in vids)
+    H, W = vids[0]["H"], vids[0]["W"]
+    if kind == "boxes":  # the 720p_cond_b2 recipe: random boxes until >= 30 % covered
+        return WL._mask(w, np.random.Generator(np.random.PCG64(seed)))
+    m = np.zeros((w.batch, F, H, W), np.uint8)
+    if kind == "all":
+        m[:] = 1
+    elif kind == "single":
+        m[-1, F - 1, H - 1, W - 1] = 1
+    return m
+
+
+MASK_CASES = {
+    "boxes_b2": (lambda: _custom("720p_cond_b2", [WL.video(2, 6, 10, t0=-2), WL.video(12, 6, 10),
+                                                  WL.audio(218), WL.text(12)], batch=2), "boxes"),
+    "all_rows": (lambda: _custom("720p_cond_b2", [WL.video(1, 6, 10, t0=-1), WL.video(5, 6, 10),
+                                                  WL.audio(40), WL.text(12)]), "all"),
+    "empty": (lambda: _custom("720p_cond_b2", [WL.video(3, 6, 10), WL.audio(40)], batch=2), "none"),
+    "single_row": (lambda: _custom("720p_cond_b2", [WL.video(3, 6, 10), WL.audio(40)], batch=2),
+                   "single"),
+    # several 256-row query tiles per batch item: ~1,500 masked rows of 5,120
+    "boxes_large": (lambda: _custom("720p_cond_b2", [WL.video(1, 8, 16, t0=-1),
+                                                     WL.video(39, 8, 16), WL.audio(218),
+                                                     WL.text(16)], heads=3, batch=2), "boxes"),
+}
+
+
+@pytest.mark.parametrize("case", list(MASK_CASES))
+def test_masked_joint_bf16(M, case):
+    make, kind = MASK_CASES[case]
+    w = make()
+    x, host, dev = _make(w)
+    mask = _box_mask(w, 77, kind)
+    fill = WL.f32_to_bf16_bits(np.random.default_rng(5).standard_normal(x["q"].shape,
+                                                                          dtype=np.float32))
+    o = to_device(fill, "bf16")
+    d = M.desc_of(dev["q"])
+    lay = M.make_layout(w.segments)
+    n = M.masked_joint_attn_workspace_size(d, lay)
+    ws = torch.empty(max(n, 256), dtype=torch.uint8, device="cuda")
+    md = torch.from_numpy(mask).cuda()
+    M.masked_joint_attn(dev["q"], dev["k"], dev["v"], o, d, lay, 1 / math.sqrt(128), md, ws, n)
+    torch.cuda.synchronize()
+    assert M.device_status() == 0
+    rows = O.masked_rows(oracle_layout(w.segments), mask)
+    ref = O.masked_joint_attn(host["q"], host["k"], host["v"], WL.as_f64(fill, "bf16"), rows,
+                              1 / math.sqrt(128))
+    got = to_host_f64(o)
+    for b in range(w.batch):
+        r = rows[b]
+        keep = np.setdiff1d(np.arange(w.n_tokens), r)
+        if len(r):
+            assert_close(got[b, r], ref[b, r], "bf16", f"masked rows b{b}")
+        assert np.array_equal(got[b, keep], ref[b, keep]), f"unmasked rows changed b{b}"
+
+
+def test_masked_joint_rejects_bad_arguments(M):
+    w = MASK_CASES["empty"][0]()
+    _, _, dev = _make(w)
+    d = M.desc_of(dev["q"])
+    lay = M.make_layout(w.segments)
+    o = torch.empty_like(dev["q"])
+    n = M.masked_joint_attn_workspace_size(d, lay)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    good = torch.zeros((w.batch, 3, 6, 10), dtype=torch.uint8, device="cuda")
+    with pytest.raises(M.MmditError):  # mask of the wrong size
+        M.masked_joint_attn(dev["q"], dev["k"], dev["v"], o, d, lay, 0.1, good[:, :2], ws, n)
+    with pytest.raises(M.MmditError):  # workspace too small
+        M.masked_joint_attn(dev["q"], dev["k"], dev["v"], o, d, lay, 0.1, good, ws, n - 256)
+    with pytest.raises(M.MmditError):  # output aliases an input
+        M.masked_joint_attn(dev["q"], dev["k"], dev["v"], dev["v"], d, lay, 0.1, good, ws, n)
+    # block-major video is not supported by this call
+    qb = torch.zeros((1, 256, 2, 128), dtype=torch.bfloat16, device="cuda")
+    db = M.desc_of(qb)
+    bl = M.make_layout([WL.video(4, 8, 8, order=WL.ORDER_BLOCK444)])
+    assert M.masked_joint_attn_workspace_size(db, bl) == 0
+    mb = torch.zeros((1, 4, 8, 8), dtype=torch.uint8, device="cuda")
+    with pytest.raises(M.MmditError) as e:
+        M.masked_joint_attn(qb, qb.clone(), qb.clone(), torch.empty_like(qb), db, bl, 0.1, mb,
+                            ws, n)
+    assert e.value.status == M.EUNSUPPORTED
+
+
 # ------------------------------------------------------------ block-sparse mode
 
 SPARSE_CASES = {

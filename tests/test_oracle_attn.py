@@ -134,3 +134,53 @@ def test_text_cross_closed_forms():
     kt2 = kt.copy(); kt2[:, :, 1] *= -3.0
     o2 = O.text_cross_attn(qv, kt2, vt, 0.4)
     assert np.array_equal(o2[:, :, 0], o[:, :, 0]) and np.array_equal(o2[:, :, 2], o[:, :, 2])
+
+
+def _mask_layout():
+    segs = [O.Segment(O.SEG_VIDEO, 2 * 3 * 4, 2, 3, 4, t0=-2), O.Segment(O.SEG_VIDEO, 3 * 3 * 4, 3, 3, 4),
+            O.Segment(O.SEG_AUDIO, 7, t_num=21, t_den=218), O.Segment(O.SEG_TEXT, 5)]
+    return O.Layout(segs)
+
+
+def test_masked_rows_follow_positions():
+    lay = _mask_layout()
+    rng = np.random.default_rng(41)
+    mask = (rng.random((2, 5, 3, 4)) < 0.4).astype(np.uint8)
+    rows = O.masked_rows(lay, mask)
+    pos = O.positions(lay)
+    for b in range(2):
+        # every masked (frame, h, w) appears exactly once, at the token whose
+        # position is (frame - 2, h, w): the first two frames are the
+        # conditioning frames at t = -2, -1
+        want = sorted((f - 2, h, w) for f, h, w in zip(*np.nonzero(mask[b])))
+        got = sorted(tuple(int(x) for x in pos[r]) for r in rows[b])
+        assert got == want
+        assert np.all(np.diff(rows[b]) > 0)  # sequence order, no repeats
+        assert np.all(rows[b] < 60)          # video tokens only (audio/text start at 60)
+
+
+def test_masked_joint_special_cases():
+    lay = _mask_layout()
+    n = lay.n_tokens
+    q, k, v = _r((2, n, 2, 8), 42), _r((2, n, 2, 8), 43), _r((2, n, 2, 8), 44)
+    o0 = _r((2, n, 2, 8), 45)
+    full, _ = O.joint_attn(q, k, v, 0.3)
+    # all video tokens masked: the video rows are the joint-attention rows and
+    # the audio/text rows keep their initial value
+    rows = O.masked_rows(lay, np.ones((2, 5, 3, 4), np.uint8))
+    o = O.masked_joint_attn(q, k, v, o0, rows, 0.3)
+    assert np.allclose(o[:, :60], full[:, :60]) and np.array_equal(o[:, 60:], o0[:, 60:])
+    # empty mask: nothing changes
+    rows0 = O.masked_rows(lay, np.zeros((2, 5, 3, 4), np.uint8))
+    assert np.array_equal(O.masked_joint_attn(q, k, v, o0, rows0, 0.3), o0)
+    # a partial mask: masked rows equal those of full joint attention (each
+    # row sees every key), the others are untouched
+    mask = np.zeros((2, 5, 3, 4), np.uint8)
+    mask[0, 1, 2, 3] = 1
+    mask[1, 3:, :2, 1:3] = 1
+    rows = O.masked_rows(lay, mask)
+    o = O.masked_joint_attn(q, k, v, o0, rows, 0.3)
+    for b in range(2):
+        keep = np.setdiff1d(np.arange(n), rows[b])
+        assert np.allclose(o[b, rows[b]], full[b, rows[b]])
+        assert np.array_equal(o[b, keep], o0[b, keep])
