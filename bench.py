@@ -95,6 +95,10 @@ def dense_step_flops(w: WL.Workload) -> dict:
 # DRAM bytes per launch of the dominant kernel from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only while the kernel
 # source is the one that was captured (sha1 of attn_tc.cu + common.cuh).
+# Channels of the video latent that the flow-matching step interpolates (the
+# pages leave the latent width open; 16 is taken).
+LATENT_CHANNELS = 16
+
 NCU_TRAFFIC = {
     "480p": {"src": "21f71342ae8922c8", "bytes": 837867008},  # ncu, one joint launch
 }
@@ -469,6 +473,46 @@ def run_gpu(args) -> int:
             raise RuntimeError("device status after the masked attention: " + M.last_error())
         del ws_mask, o_mask
 
+    # ------------------------------------------- flow-matching elementwise
+    # The noised input / velocity target and the loss term of the video
+    # stream's latent (the video token grid x LATENT_CHANNELS values per item),
+    # separate calls: at the workload's batch (1 MB-scale tensors, launch-bound)
+    # and at a 64-item batch of the same latent (larger than L2, HBM-bound).
+    flow = {}
+    n_lat = w.n_video * LATENT_CHANNELS
+    for label, items in (("workload_batch", w.batch), ("batch64", 64)):
+        g = torch.Generator(device=dev).manual_seed(9)
+        z0_l, eps_l, v_l = (torch.randn((items, n_lat), generator=g, device=dev,
+                                        dtype=torch.float32).to(torch.bfloat16) for _ in range(3))
+        t_l = torch.rand(items, generator=g, device=dev)
+        zt_l, u_l = torch.empty_like(z0_l), torch.empty_like(z0_l)
+        loss_l = torch.empty(items, device=dev)
+        nfw = M.flow_loss_workspace_size(items, n_lat)
+        ws_l = torch.empty(max(nfw, 256), dtype=torch.uint8, device=dev)
+        times = []
+        for fn in (lambda: M.flow_noise(z0_l, eps_l, t_l, zt_l, u_l, stream),
+                   lambda: M.flow_loss(v_l, z0_l, eps_l, loss_l, ws_l, nfw, stream)):
+            for _ in range(args.warmup):
+                fn()
+            torch.cuda.synchronize(dev)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            times.append(reduce_max(e0.elapsed_time(e1), world, dev) / args.steps)
+        nb = items * n_lat * 2
+        flow[label] = {"items": items, "values_per_item": n_lat,
+                       "noise_us": round(times[0] * 1e3, 2),
+                       "noise_gbs": round(4 * nb / (times[0] / 1e3) / 1e9, 1),
+                       "loss_us": round(times[1] * 1e3, 2),
+                       "loss_gbs": round(3 * nb / (times[1] / 1e3) / 1e9, 1)}
+        del z0_l, eps_l, v_l, zt_l, u_l, ws_l
+    if M.device_status(stream) != 0:
+        raise RuntimeError("device status after the flow-matching kernels: " + M.last_error())
+
     # ---------------------------------------------------------- end to end
     pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
     hq, hk, hv = pin(x["q"]), pin(x["k"]), pin(x["v"])
@@ -555,6 +599,12 @@ def run_gpu(args) -> int:
                                 "masked_rows": n_rows, "launches": args.steps,
                                 "note": "separate call (rows of masked video tokens over every "
                                         "key), not part of the step or its value"}
+    hbm = peaks.get("hbm_gbs") or FALLBACK_PEAKS["hbm_gbs"]
+    for f_ in flow.values():
+        f_["noise_frac_hbm"] = round(f_["noise_gbs"] / hbm, 4)
+        f_["loss_frac_hbm"] = round(f_["loss_gbs"] / hbm, 4)
+    line["flow_matching"] = dict(flow, note="separate calls on bf16 latents; bytes = 2 reads + 2 "
+                                            "writes (noise) or 3 reads (loss) per value")
     if sparse:
         line["block_density"] = round(density, 4)
     if world == 1 and not args.no_cpu_baseline:

@@ -228,6 +228,44 @@ MMDIT_API size_t mmdit_masked_joint_attn_workspace_size(const mmdit_tensor_desc*
                                               const mmdit_layout* layout);
 
 /*
+ * mmdit_flow_noise -- flow-matching input and target of one stream (digest
+ *   step 4: z_t = t z_0 + (1 - t) eps, and the model is trained to predict the
+ *   velocity z_0 - eps), fused in one elementwise pass:
+ *     zt[b, i] = t[b] * z0[b, i] + (1 - t[b]) * eps[b, i]
+ *     u[b, i]  = z0[b, i] - eps[b, i]
+ *   for i < n of every batch item b < batch; math in fp32.
+ *   z0, eps   : device, batch items of n values `stride` elements apart
+ *               (stride >= n); the noise is an input, drawn by the caller.
+ *   t         : device float [batch], the flow time of each item.
+ *   zt, u     : device outputs with the same shape and stride; either may be
+ *               NULL (not written), not both.
+ *   dtype     : MMDIT_BF16 or MMDIT_F32 for all of z0, eps, zt, u.
+ *   Pointers must be 16-byte aligned and stride * element size a multiple of
+ *   16 bytes.  The video and the audio stream are separate calls.
+ *   Errors : EINVAL, EUNSUPPORTED, ECUDA.
+ */
+MMDIT_API int mmdit_flow_noise(const void* z0, const void* eps, const float* t, void* zt, void* u,
+                     int32_t batch, int64_t n, int64_t stride, int32_t dtype,
+                     mmdit_stream_t stream);
+
+/*
+ * mmdit_flow_loss -- the flow-matching loss term of one stream (digest step 4:
+ *   || v_theta - (z_0 - eps) ||^2), per batch item:
+ *     loss[b] = sum over i < n of (v[b, i] - (z0[b, i] - eps[b, i]))^2
+ *   in fp32, summed in a fixed order (the same bits on every call).  The
+ *   layer's loss is the batch mean of loss_video[b] + loss_audio[b].
+ *   v, z0, eps : device, same shape, stride and dtype rules as mmdit_flow_noise
+ *   loss       : device float [batch] output
+ *   workspace  : mmdit_flow_loss_workspace_size(batch, n) bytes, 256-byte
+ *                aligned (per-block partial sums).
+ *   Errors : EINVAL, EUNSUPPORTED, EWORKSPACE, ECUDA.
+ */
+MMDIT_API int mmdit_flow_loss(const void* v, const void* z0, const void* eps, float* loss,
+                    int32_t batch, int64_t n, int64_t stride, int32_t dtype, void* workspace,
+                    size_t ws_bytes, mmdit_stream_t stream);
+MMDIT_API size_t mmdit_flow_loss_workspace_size(int32_t batch, int64_t n);
+
+/*
  * mmdit_av_cross_attn_noalloc -- the same cross-attention as
  *   mmdit_av_cross_attn, for callers that cannot allocate device memory or
  *   size a workspace (a plugin inside a runtime that owns every device

@@ -67,6 +67,11 @@ _SIGS = {
     "mmdit_masked_joint_attn": (C.c_int, [_P, _P, _P, _P, _D, _L, C.c_float, _P, C.c_int64, _P,
                                           C.c_size_t, _P]),
     "mmdit_masked_joint_attn_workspace_size": (C.c_size_t, [_D, _L]),
+    "mmdit_flow_noise": (C.c_int, [_P, _P, _P, _P, _P, C.c_int32, C.c_int64, C.c_int64,
+                                   C.c_int32, _P]),
+    "mmdit_flow_loss": (C.c_int, [_P, _P, _P, _P, C.c_int32, C.c_int64, C.c_int64, C.c_int32, _P,
+                                  C.c_size_t, _P]),
+    "mmdit_flow_loss_workspace_size": (C.c_size_t, [C.c_int32, C.c_int64]),
     "mmdit_av_cross_attn_noalloc": (C.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _D, _D, C.c_float,
                                               _P]),
     "mmdit_block_select": (C.c_int, [_P, _P, _D, _L, C.c_int, C.c_float, C.c_float, C.c_int,
@@ -212,6 +217,32 @@ def masked_joint_attn(q, k, v, o, desc: TensorDesc, layout: Layout, scale: float
 
 def masked_joint_attn_workspace_size(desc: TensorDesc, layout: Layout) -> int:
     return _lib.mmdit_masked_joint_attn_workspace_size(C.byref(desc), C.byref(layout))
+
+
+def _items(x):
+    """(batch, n, stride, dtype) of a [B, ...] tensor whose items are contiguous
+    runs (the trailing dimensions of each item packed)."""
+    import torch
+    b = x.shape[0]
+    n = x[0].numel() if b else 0
+    dt = {torch.bfloat16: BF16, torch.float32: F32}[x.dtype]
+    return b, n, (x.stride(0) if b else n), dt
+
+
+def flow_noise(z0, eps, t, zt=None, u=None, stream=None) -> None:
+    b, n, st, dt = _items(z0)
+    _check(_lib.mmdit_flow_noise(_ptr(z0), _ptr(eps), _ptr(t), _ptr(zt), _ptr(u), b, n, st, dt,
+                                 _stream(stream)))
+
+
+def flow_loss_workspace_size(batch: int, n: int) -> int:
+    return _lib.mmdit_flow_loss_workspace_size(batch, n)
+
+
+def flow_loss(v, z0, eps, loss, workspace=None, ws_bytes: int = 0, stream=None) -> None:
+    b, n, st, dt = _items(z0)
+    _check(_lib.mmdit_flow_loss(_ptr(v), _ptr(z0), _ptr(eps), _ptr(loss), b, n, st, dt,
+                                _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024  # MMDIT_NOALLOC_SCRATCH_BYTES

@@ -293,6 +293,24 @@ def masked_joint_attn(q, k, v, o_init, rows, scale):
     return o
 
 
+def flow_noise(z0, eps, t):
+    """Flow-matching input and velocity target of one stream ([SKY-D] step 4):
+    z_t = t z_0 + (1 - t) eps for each batch item's time t[b], and the
+    velocity the model is trained to predict, z_0 - eps.  Arrays are [B, ...];
+    returns (z_t, target) in float64."""
+    z0 = np.asarray(z0, np.float64)
+    eps = np.asarray(eps, np.float64)
+    tb = np.asarray(t, np.float64).reshape((-1,) + (1,) * (z0.ndim - 1))
+    return tb * z0 + (1.0 - tb) * eps, z0 - eps
+
+
+def flow_loss(v, z0, eps):
+    """The stream's loss term per batch item ([SKY-D] step 4): the squared
+    L2 norm || v - (z_0 - eps) ||^2 over the item's values, float64 [B]."""
+    d = np.asarray(v, np.float64) - (np.asarray(z0, np.float64) - np.asarray(eps, np.float64))
+    return (d.reshape(d.shape[0], -1) ** 2).sum(axis=1)
+
+
 # ---------------------------------------------------------------------------
 # a5 - a7: block-sparse mode
 # ---------------------------------------------------------------------------
