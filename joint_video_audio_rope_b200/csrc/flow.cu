@@ -178,7 +178,7 @@ extern "C" {
 int mmdit_flow_noise(const void* z0, const void* eps, const float* t, void* zt, void* u,
                      int32_t batch, int64_t n, int64_t stride, int32_t dtype,
                      mmdit_stream_t stream) {
-  int rc = check_flow("flow_noise", batch, n, stride, dtype, {z0, eps, t, zt, u});
+  int rc = check_flow("flow_noise", batch, n, stride, dtype, {z0, eps, zt, u});  // t: scalar reads
   if (rc) return rc;
   if (!z0 || !eps || !t) return fail(MMDIT_EINVAL, "flow_noise: z0, eps, t must be non-NULL");
   if (!zt && !u) return fail(MMDIT_EINVAL, "flow_noise: zt and u are both NULL");

@@ -154,3 +154,63 @@ def test_sparse_attn_validation():
     assert _rc(M.sparse_attn, *args, d, L, FAKE, FAKE, 3000, 0.088, FAKE, ws) == M.EINVAL
     assert _rc(M.sparse_attn, *args, d, L, FAKE, FAKE, 3060, 0.088, FAKE, ws - 1) == M.EWORKSPACE
     assert _rc(M.sparse_attn, *args, d, L, FAKE, FAKE, 3060, 0.088, FAKE + 8, ws) == M.EINVAL
+
+
+def test_text_cross_validation():
+    f = M.raw("mmdit_text_cross_attn")
+    dv, dt = _desc(n_tokens=64), _desc(n_tokens=16)
+    assert f(None, FAKE, FAKE, FAKE, C.byref(dv), C.byref(dt), 0.1, None) == M.EINVAL
+    bad = _desc(n_tokens=16, heads=3)
+    assert f(FAKE, FAKE, FAKE, FAKE * 2, C.byref(dv), C.byref(bad), 0.1, None) == M.EINVAL
+    empty = _desc(n_tokens=0)
+    assert f(FAKE, FAKE, FAKE, FAKE * 2, C.byref(dv), C.byref(empty), 0.1, None) == M.EINVAL
+    assert f(FAKE, FAKE, FAKE, FAKE, C.byref(dv), C.byref(dt), 0.1, None) == M.EINVAL  # o is q
+    assert f(FAKE, FAKE, FAKE, FAKE * 2, C.byref(dv), C.byref(dt), 0.0, None) == M.EINVAL
+    assert f(FAKE + 4, FAKE, FAKE, FAKE * 2, C.byref(dv), C.byref(dt), 0.1, None) == M.EINVAL
+    f32 = _desc(n_tokens=16, dtype=M.F32)
+    assert f(FAKE, FAKE, FAKE, FAKE * 2, C.byref(dv), C.byref(f32), 0.1, None) == M.EINVAL
+
+
+def _cond_layout():
+    return M.make_layout([dict(kind=M.SEG_VIDEO, n_tokens=32, T=2, H=4, W=4, t0=-2),
+                          dict(kind=M.SEG_VIDEO, n_tokens=48, T=3, H=4, W=4),
+                          dict(kind=M.SEG_TEXT, n_tokens=32)])
+
+
+def test_masked_joint_validation_and_workspace():
+    f = M.raw("mmdit_masked_joint_attn")
+    d, lay = _desc(batch=2), _cond_layout()
+    need = M.masked_joint_attn_workspace_size(d, lay)
+    # row counts + row lists + compact Q and O rows of all 80 video tokens
+    assert need >= 2 * 80 * 2 * 128 * 2 * 2
+    ws = 0x100000
+    elems = 2 * 5 * 16
+    ok = (FAKE, FAKE * 2, FAKE * 3, FAKE * 4, C.byref(d), C.byref(lay), C.c_float(0.1), FAKE * 5)
+    assert f(*ok, elems - 1, ws, need, None) == M.EINVAL          # mask size
+    assert f(*ok, elems, ws, need - 256, None) == M.EWORKSPACE    # workspace size
+    assert f(*ok, elems, ws + 16, need, None) == M.EINVAL         # workspace alignment
+    d32 = _desc(batch=2, dtype=M.F32)
+    assert f(FAKE, FAKE * 2, FAKE * 3, FAKE * 4, C.byref(d32), C.byref(lay), C.c_float(0.1),
+             FAKE * 5, elems, ws, need, None) == M.EUNSUPPORTED
+    assert f(FAKE, FAKE * 2, FAKE * 3, FAKE * 2, C.byref(d), C.byref(lay), C.c_float(0.1),
+             FAKE * 5, elems, ws, need, None) == M.EINVAL         # o aliases k
+    blk = M.make_layout([dict(kind=M.SEG_VIDEO, n_tokens=112, T=7, H=4, W=4,
+                              order=M.ORDER_BLOCK444)])
+    assert M.masked_joint_attn_workspace_size(_desc(), blk) == 0
+    assert f(FAKE, FAKE * 2, FAKE * 3, FAKE * 4, C.byref(_desc()), C.byref(blk), C.c_float(0.1),
+             FAKE * 5, 7 * 16, ws, need, None) == M.EUNSUPPORTED
+
+
+def test_flow_validation_and_workspace():
+    noise, loss = M.raw("mmdit_flow_noise"), M.raw("mmdit_flow_loss")
+    assert noise(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 100, 104, 7, None) == M.EUNSUPPORTED
+    assert noise(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 100, 96, M.BF16, None) == M.EINVAL   # stride < n
+    assert noise(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 100, 100, M.BF16, None) == M.EINVAL  # 200 B stride
+    assert noise(FAKE, FAKE, FAKE, None, None, 2, 100, 104, M.BF16, None) == M.EINVAL  # no output
+    assert noise(FAKE + 2, FAKE, FAKE, FAKE, FAKE, 2, 100, 104, M.BF16, None) == M.EINVAL
+    assert noise(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 100, 104, M.BF16, None) == M.EINVAL  # batch 0
+    n1, n2 = M.flow_loss_workspace_size(2, 1000), M.flow_loss_workspace_size(2, 10 ** 7)
+    assert 0 < n1 <= n2 and n2 % 256 == 0
+    assert loss(FAKE, FAKE, FAKE, FAKE, 2, 1000, 1000, M.F32, None, 0, None) == M.EWORKSPACE
+    assert loss(FAKE, FAKE, FAKE, FAKE, 2, 1000, 1000, M.F32, 0x100010, n1, None) == M.EINVAL
+    assert loss(FAKE, FAKE, None, FAKE, 2, 1000, 1000, M.F32, 0x100000, n1, None) == M.EINVAL
