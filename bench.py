@@ -420,7 +420,7 @@ def run_gpu(args) -> int:
     # is a call of its own, outside the step the metric is defined on: timed
     # here on its own, the same number of launches, after the same warm-up.
     text_cross_ms = None
-    tx0, tx1 = WL._kind_range(w.segments, WL.SEG_TEXT)
+    tx0, tx1 = w.text_range()
     if tx1 > tx0:
         o_text = torch.empty_like(q)
         dtx = M.desc_of(k[:, tx0:tx1])

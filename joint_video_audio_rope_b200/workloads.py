@@ -77,6 +77,9 @@ class Workload:
     def audio_range(self) -> Tuple[int, int]:
         return _kind_range(self.segments, SEG_AUDIO)
 
+    def text_range(self) -> Tuple[int, int]:
+        return _kind_range(self.segments, SEG_TEXT)
+
 
 def _kind_range(segs, kind):
     start = 0

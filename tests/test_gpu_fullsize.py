@@ -80,7 +80,7 @@ def _run_dense_step(M, w, x):
     M.av_cross_attn(q[:, v0:v1], k[:, v0:v1], v[:, v0:v1], q[:, a0:a1], k[:, a0:a1], v[:, a0:a1],
                     oc[:, v0:v1], oc[:, a0:a1], dv, da, scale, ws, n)
     # reinforced text cross-attention: video queries over the text keys
-    t0, t1 = WL._kind_range(w.segments, WL.SEG_TEXT)
+    t0, t1 = w.text_range()
     ot = torch.empty_like(q)
     M.text_cross_attn(q[:, v0:v1], k[:, t0:t1], v[:, t0:t1], ot[:, v0:v1], dv,
                       M.desc_of(k[:, t0:t1]), scale)
@@ -109,7 +109,7 @@ def test_dense_workload_full_size(M, name):
     scale = 1 / math.sqrt(128)
     v0, v1 = w.video_range()
     a0, a1 = w.audio_range()
-    t0, t1 = WL._kind_range(w.segments, WL.SEG_TEXT)
+    t0, t1 = w.text_range()
     for b in range(w.batch):
         kk = O.rope(WL.as_f64(x["k"][b], "bf16"), pos, w.theta)        # every key
         vv = WL.as_f64(x["v"][b], "bf16")

@@ -252,7 +252,7 @@ def test_cross_bf16(M, case):
 # ------------------------------------------------------ text cross-attention
 
 def _text_range(w):
-    return WL._kind_range(w.segments, WL.SEG_TEXT)
+    return w.text_range()
 
 
 def _text_cross(M, w, dev):
