@@ -16,9 +16,13 @@ reader can check it against the sources by eye:
     and the list of novelties (4th: time-offset 3D RoPE with negative
     temporal indices; 5th: audio RoPE frequency scaling 21/218).
   - [SKY-B] "SkyReels-V4: dual-stream MMDiT ..." -- trdm.cn blog, sections
-    2.1 (dual stream then single stream, joint self-attention) and 2.2
+    2.1 (dual stream then single stream, joint self-attention), 2.2
     (bidirectional audio<->video cross-attention in every block; 21 video
-    frames aligned with 218 audio tokens through RoPE frequency scaling).
+    frames aligned with 218 audio tokens through RoPE frequency scaling) and
+    4.2 (the Refiner refines only the target region of a spatial mask).
+  The digest's step 3 also names the reinforced text cross-attention (video
+  queries over the text embedding) and its step 4 the flow-matching input,
+  target and loss.
   - [PRISM] "Prism: dynamic sparse attention for native 2K joint video-audio
     generation" -- reading guide of arXiv 2610.05416, Method section 3
     (mean-pooled key blocks, block probabilities P_i, and the attended set
