@@ -234,8 +234,8 @@ MMDIT_API size_t mmdit_masked_joint_attn_workspace_size(const mmdit_tensor_desc*
  *     zt[b, i] = t[b] * z0[b, i] + (1 - t[b]) * eps[b, i]
  *     u[b, i]  = z0[b, i] - eps[b, i]
  *   for i < n of every batch item b < batch; math in fp32.
- *   z0, eps   : device, batch items of n values `stride` elements apart
- *               (stride >= n); the noise is an input, drawn by the caller.
+ *   z0, eps   : device, batch items (1..65535) of n values `stride` elements
+ *               apart (stride >= n); the noise is an input, drawn by the caller.
  *   t         : device float [batch], the flow time of each item.
  *   zt, u     : device outputs with the same shape and stride; either may be
  *               NULL (not written), not both.

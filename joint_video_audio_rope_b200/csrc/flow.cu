@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(32) flow_loss_final_kernel(const float* __rest
 
 int check_flow(const char* who, int batch, long long n, long long stride, int dtype,
                std::initializer_list<const void*> ptrs) {
-  if (batch < 1 || n < 0 || stride < n)
+  if (batch < 1 || batch > 65535 || n < 0 || stride < n)  // batch items are grid rows
     return fail(MMDIT_EINVAL, "%s: batch %d, n %lld, stride %lld out of range", who, batch, n, stride);
   if (dtype != MMDIT_BF16 && dtype != MMDIT_F32)
     return fail(MMDIT_EUNSUPPORTED, "%s: dtype %d not supported", who, dtype);

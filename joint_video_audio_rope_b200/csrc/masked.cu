@@ -8,11 +8,13 @@
 //   1. mask_rows_kernel   -- per batch item, the sequence index of every
 //                            masked video token (arbitrary order) and their
 //                            count;
-//   2. gather_rows_kernel -- those Q rows into a compact [B, Nv, H, 128] buffer;
+//   2. move_rows_kernel<true>  -- those Q rows into a compact [B, Nv, H, 128]
+//                            buffer (gather);
 //   3. attn_tc_kernel     -- dense attention of the compact rows over every
 //                            key, the per-batch count bounding the query rows
 //                            (work items past it compute nothing);
-//   4. scatter_rows_kernel-- the compact O rows back to their tokens.
+//   4. move_rows_kernel<false> -- the compact O rows back to their tokens
+//                            (scatter).
 // Rows are independent in attention, so the order of the row list changes no
 // value.  Nv (video tokens per batch item) sizes the scratch: the count is
 // only known on the device, and nothing here waits for it on the host.
@@ -151,6 +153,8 @@ int mmdit_masked_joint_attn(const void* q, const void* k, const void* v, void* o
     return fail(MMDIT_EINVAL, "masked_joint: tensors must be 16-byte aligned");
   if (o == q || o == k || o == v) return fail(MMDIT_EINVAL, "masked_joint: o aliases an input");
   if (!(scale > 0.f) || !isfinite(scale)) return fail(MMDIT_EINVAL, "masked_joint: scale must be > 0");
+  if (desc->batch > 65535)  // batch items are grid rows of the row kernels
+    return fail(MMDIT_EINVAL, "masked_joint: batch %d > 65535", desc->batch);
   MaskedPlan p;
   if ((rc = plan_masked(*desc, layout, p))) return rc;
   const long long expect = (long long)desc->batch * p.vr.frames * p.vr.hw;

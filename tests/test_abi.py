@@ -214,3 +214,12 @@ def test_flow_validation_and_workspace():
     assert loss(FAKE, FAKE, FAKE, FAKE, 2, 1000, 1000, M.F32, None, 0, None) == M.EWORKSPACE
     assert loss(FAKE, FAKE, FAKE, FAKE, 2, 1000, 1000, M.F32, 0x100010, n1, None) == M.EINVAL
     assert loss(FAKE, FAKE, None, FAKE, 2, 1000, 1000, M.F32, 0x100000, n1, None) == M.EINVAL
+
+
+def test_batch_limits_of_row_grids():
+    noise = M.raw("mmdit_flow_noise")
+    assert noise(FAKE, FAKE, FAKE, FAKE, FAKE, 65536, 100, 104, M.BF16, None) == M.EINVAL
+    f = M.raw("mmdit_masked_joint_attn")
+    d, lay = _desc(batch=65536), _cond_layout()
+    assert f(FAKE, FAKE * 2, FAKE * 3, FAKE * 4, C.byref(d), C.byref(lay), C.c_float(0.1),
+             FAKE * 5, 65536 * 80, 0x100000, 1 << 40, None) == M.EINVAL
