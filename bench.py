@@ -262,12 +262,12 @@ def oracle_sample(w: WL.Workload, host: dict, rows: int, seed: int = 0):
 
 def calibrate_rows(w: WL.Workload, host: dict, target_s: float) -> int:
     """Number of sampled query rows whose oracle sample takes about target_s
-    (grown geometrically from a small probe; the fixed cost of rotating every
-    key is part of each probe)."""
+    (grown geometrically from a small probe until a probe takes at least 0.7 x
+    target_s; the fixed cost of rotating every key is part of each probe)."""
     rows = 8
     for _ in range(6):
         dt, _ = oracle_sample(w, host, rows, seed=1)
-        if dt >= 0.5 * target_s or rows >= w.n_tokens:
+        if dt >= 0.7 * target_s or rows >= w.n_tokens:
             break
         rows = int(min(w.n_tokens, rows * min(8.0, max(2.0, 0.8 * target_s / max(dt, 1e-3)))))
     return max(8, rows)
