@@ -203,12 +203,17 @@ def av_cross_attn_workspace_size(video: TensorDesc, audio: TensorDesc) -> int:
 
 def text_cross_attn(qv, kt, vt, o_video, video: TensorDesc, text: TensorDesc, scale: float,
                     stream=None) -> None:
+    """o_video = softmax(qv kt^T * scale) vt: video queries over the text
+    keys (the reinforced text cross-attention); no workspace."""
     _check(_lib.mmdit_text_cross_attn(_ptr(qv), _ptr(kt), _ptr(vt), _ptr(o_video), C.byref(video),
                                       C.byref(text), scale, _stream(stream)))
 
 
 def masked_joint_attn(q, k, v, o, desc: TensorDesc, layout: Layout, scale: float, mask,
                       workspace=None, ws_bytes: int = 0, stream=None) -> None:
+    """Joint-attention rows of the video tokens whose uint8 mask [B, F, H, W]
+    value is non-zero; every other row of o is left as it was.  Workspace from
+    masked_joint_attn_workspace_size."""
     n = 0 if mask is None else mask.numel()
     _check(_lib.mmdit_masked_joint_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), C.byref(desc),
                                         C.byref(layout), scale, _ptr(mask), n, _ptr(workspace),
@@ -230,6 +235,8 @@ def _items(x):
 
 
 def flow_noise(z0, eps, t, zt=None, u=None, stream=None) -> None:
+    """zt = t z0 + (1 - t) eps and u = z0 - eps per batch item (t: float
+    [B] on the device); [B, ...] tensors whose items are contiguous runs."""
     b, n, st, dt = _items(z0)
     _check(_lib.mmdit_flow_noise(_ptr(z0), _ptr(eps), _ptr(t), _ptr(zt), _ptr(u), b, n, st, dt,
                                  _stream(stream)))
@@ -240,6 +247,8 @@ def flow_loss_workspace_size(batch: int, n: int) -> int:
 
 
 def flow_loss(v, z0, eps, loss, workspace=None, ws_bytes: int = 0, stream=None) -> None:
+    """loss[b] = sum over item b of (v - (z0 - eps))^2, fp32, fixed summation
+    order.  Workspace from flow_loss_workspace_size."""
     b, n, st, dt = _items(z0)
     _check(_lib.mmdit_flow_loss(_ptr(v), _ptr(z0), _ptr(eps), _ptr(loss), b, n, st, dt,
                                 _ptr(workspace), ws_bytes, _stream(stream)))
