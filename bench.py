@@ -10,11 +10,16 @@ video self-attention, then the bidirectional audio<->video cross-attention.
 Inputs are seeded synthetic tensors of the workload's shape, resident in HBM
 before timing; they are larger than L2 (126 MB), so no flush is needed.
 
-The JSON line reports algorithmic TFLOP/s (4 * Nq * Nkv * d per head for
-every attention; for sparse attention only the selected token pairs), video
-tokens/s, an end-to-end figure through the same C-ABI calls with pinned host
-buffers copied in and results copied out every step, the live roofline of
-the dominant kernel (CUDA events around its launches), SM clocks sampled
+The headline workload (default: 720p_cond_b2, the largest dense layer that
+fits one GPU) gives the line's value; the other workloads (480p, 720p,
+1080p_sparse) follow under "per_config", timed the same way.  The JSON line
+reports algorithmic TFLOP/s (4 * Nq * Nkv * d per head for every attention;
+for sparse attention only the selected token pairs), video tokens/s, an
+end-to-end figure through the same C-ABI calls with pinned host buffers
+copied in and results copied out every step (copies overlapped with compute
+on two copy streams), the live roofline of the dominant kernel (CUDA events
+around its launches) against the sustained bf16 peak when the timed region
+lasts a second or more and the burst peak otherwise, SM clocks sampled
 during the timed region, and the fp64 oracle timed on a bounded sample on
 the host cores (CPU baseline).
 
@@ -92,13 +97,16 @@ def dense_step_flops(w: WL.Workload) -> dict:
             "cross": attn_flops(nv, na, d, H, B) + attn_flops(na, nv, d, H, B)}
 
 
-# DRAM bytes per launch of the dominant kernel from one ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum), valid only while the kernel
-# source is the one that was captured (sha1 of attn_tc.cu + common.cuh).
 # Channels of the video latent that the flow-matching step interpolates (the
 # pages leave the latent width open; 16 is taken).
 LATENT_CHANNELS = 16
 
+# Workloads timed after the headline one, each reported under "per_config".
+PER_CONFIG = ("480p", "720p", "720p_cond_b2", "1080p_sparse")
+
+# DRAM bytes per launch of the dominant kernel from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), valid only while the kernel
+# source is the one that was captured (sha1 of attn_tc.cu + common.cuh).
 NCU_TRAFFIC = {
     "480p": {"src": "5ac8cc44391153b7", "bytes": 833501184},  # ncu, one joint launch
 }
@@ -285,6 +293,281 @@ def cpu_baseline(w: WL.Workload, host: dict, target_s: float = 15.0) -> dict:
 
 # ----------------------------------------------------------------- GPU arm
 
+# A timed region at least this long runs the GPU at its power-capped sustained
+# clock: a dominant kernel timed inside it is compared with the sustained bf16
+# peak, a shorter one (a burst) with the burst peak.
+SUSTAINED_REGION_MS = 1000.0
+
+
+def pick_peak(peaks: dict, region_ms: float):
+    """(peak TFLOP/s, name) of the bf16 peak that matches a timed region."""
+    if region_ms >= SUSTAINED_REGION_MS:
+        key = "bf16_tflops_sustained"
+    else:
+        key = "bf16_tflops"
+    return peaks.get(key) or FALLBACK_PEAKS[key], key
+
+
+class Layer:
+    """Device tensors of one workload and the call sequence of one step:
+    RoPE of Q and K in place, then joint attention (dense workloads) or block
+    selection + sparse attention (the block-sparse workload), then both
+    directions of the audio<->video cross-attention."""
+
+    def __init__(self, M, w, x, dev):
+        import torch
+        self.M, self.w = M, w
+        up = lambda a: (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev))
+        self.q, self.k, self.v = up(x["q"]), up(x["k"]), up(x["v"])
+        self.o = torch.empty_like(self.q)
+        self.oc = torch.empty_like(self.q)  # video and audio slices take the cross outputs
+        q = self.q
+        self.desc = M.desc_of(q)
+        self.lay = M.make_layout(w.segments)
+        self.rope = M.rope_params(w.theta, 44, 42, 42)
+        self.scale = 1.0 / math.sqrt(w.head_dim)
+        self.v0, self.v1 = w.video_range()
+        self.a0, self.a1 = w.audio_range()
+        v0, v1, a0, a1 = self.v0, self.v1, self.a0, self.a1
+        self.dv, self.da = M.desc_of(q[:, v0:v1]), M.desc_of(q[:, a0:a1])
+        ws_cross = M.av_cross_attn_workspace_size(self.dv, self.da)
+        self.sparse = w.sparse
+        ws_sel = ws_sp = 0
+        if self.sparse:
+            self.vlay = M.make_layout([s for s in w.segments if s["kind"] == WL.SEG_VIDEO])
+            self.nb = M.num_blocks(self.vlay)
+            self.idx = torch.empty((w.batch, w.heads, self.nb, self.nb), dtype=torch.int32,
+                                   device=dev)
+            self.cnt = torch.empty((w.batch, w.heads, self.nb), dtype=torch.int32, device=dev)
+            ws_sel = M.block_select_workspace_size(self.dv, self.vlay)
+            ws_sp = M.sparse_attn_workspace_size(self.dv, self.vlay, self.nb)
+        self.ws = torch.empty(max(ws_cross, ws_sel, ws_sp, 256), dtype=torch.uint8, device=dev)
+        # launches of this library's kernels per step: RoPE 1; joint 1 or
+        # pooling + selection 2 and groups + union + sparse attention 3; cross 3
+        self.launches = 1 + (5 if self.sparse else 1) + 3
+
+    def step(self, stream, ev=None):
+        M, w = self.M, self.w
+        q, k, v, o, oc = self.q, self.k, self.v, self.o, self.oc
+        v0, v1, a0, a1 = self.v0, self.v1, self.a0, self.a1
+        if ev is not None:
+            ev[0].record(stream)
+        M.rope_apply(q, k, self.desc, self.lay, self.rope, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        if self.sparse:
+            M.block_select(q[:, v0:v1], k[:, v0:v1], self.dv, self.vlay, w.top_k, w.top_p,
+                           self.scale, self.nb, self.idx, self.cnt, self.ws, self.ws.numel(),
+                           stream)
+            if ev is not None:
+                ev[2].record(stream)
+            M.sparse_attn(q[:, v0:v1], k[:, v0:v1], v[:, v0:v1], o[:, v0:v1], self.dv, self.vlay,
+                          self.idx, self.cnt, self.nb, self.scale, self.ws, self.ws.numel(),
+                          stream)
+        else:
+            if ev is not None:
+                ev[2].record(stream)
+            M.joint_attn(q, k, v, o, self.desc, self.lay, self.scale, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+        M.av_cross_attn(q[:, v0:v1], k[:, v0:v1], v[:, v0:v1], q[:, a0:a1], k[:, a0:a1],
+                        v[:, a0:a1], oc[:, v0:v1], oc[:, a0:a1], self.dv, self.da, self.scale,
+                        self.ws, self.ws.numel(), stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+
+def selected_pair_flops(w, idx_h, cnt_h):
+    """Algorithmic flops of block-sparse attention: 4 d per selected
+    (query token, key token) pair, summed over every (batch, head, block)."""
+    seg = w.segments[0]
+    nb = idx_h.shape[2]
+    blen = np.array([_block_len(seg["T"], seg["H"], seg["W"], b) for b in range(nb)], np.int64)
+    pairs = 0
+    for b in range(w.batch):
+        for h in range(w.heads):
+            for i in range(nb):
+                pairs += blen[i] * blen[idx_h[b, h, i, :cnt_h[b, h, i]]].sum()
+    return 4.0 * pairs * w.head_dim
+
+
+def time_steps(L, args, dev, stream, world, sampler=None, restore=None):
+    """Warm up, then time args.steps steps with CUDA events on `stream`
+    (barrier + synchronize on both sides, max over ranks).  Returns
+    (ms per step, mean ms of each part, host-time window)."""
+    import torch
+    M = L.M
+
+    def one(ev=None):
+        if restore is not None:
+            restore()
+        L.step(stream, ev)
+
+    for _ in range(args.warmup):
+        one()
+    torch.cuda.synchronize(dev)
+    if M.device_status(stream) != 0:
+        raise RuntimeError("device status after warm-up: " + M.last_error())
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    if sampler is not None:
+        sampler.start()
+        time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    host_t0 = time.time()
+    t_start.record(stream)
+    for i in range(args.steps):
+        one(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    host_t1 = time.time()
+    barrier(world, dev)
+    if M.device_status(stream) != 0:
+        raise RuntimeError("device status after timing: " + M.last_error())
+    ms_total = reduce_max(t_start.elapsed_time(t_end), world, dev)
+    names = ["rope", "select" if L.sparse else "none", "sparse" if L.sparse else "joint", "cross"]
+    part_ms = {name: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
+               for j, name in enumerate(names) if name != "none"}
+    return ms_total / args.steps, part_ms, (host_t0, host_t1)
+
+
+def time_call(fn, args, dev, stream, world):
+    """Mean device ms of `fn` over args.steps back-to-back calls after
+    args.warmup untimed ones (CUDA events, max over ranks)."""
+    import torch
+    for _ in range(args.warmup):
+        fn()
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    return reduce_max(e0.elapsed_time(e1), world, dev) / args.steps
+
+
+def measure_workload(M, w, args, dev, stream, world, peaks, sampler=None):
+    """Timed steps of one workload with inputs resident in HBM: step time,
+    algorithmic TFLOP/s, video tokens/s and the dominant kernel against the
+    bf16 peak that matches the length of the timed region."""
+    import torch
+    x = WL.generate(w)
+    L = Layer(M, w, x, dev)
+    restore = None
+    if L.sparse:
+        # the selected blocks (so the work) depend on the values: every step
+        # starts from the generated Q and K (a device copy counted in the step)
+        q0, k0 = L.q.clone(), L.k.clone()
+
+        def restore():
+            L.q.copy_(q0)
+            L.k.copy_(k0)
+    ms_step, part_ms, window = time_steps(L, args, dev, stream, world, sampler, restore)
+    flops = dense_step_flops(w)
+    res = {}
+    if L.sparse:
+        idx_h, cnt_h = L.idx.cpu().numpy(), L.cnt.cpu().numpy()
+        flops = {"joint": selected_pair_flops(w, idx_h, cnt_h), "cross": flops["cross"]}
+        res["block_density"] = round(float(cnt_h.mean() / L.nb), 4)
+        del idx_h
+    step_flops = flops["joint"] + flops["cross"]
+    dom = "sparse" if L.sparse else "joint"
+    region_ms = ms_step * args.steps
+    peak, peak_key = pick_peak(peaks, region_ms)
+    achieved = flops["joint"] / (part_ms[dom] / 1e3) / 1e12
+    res.update({
+        "ms_per_step": round(ms_step, 4),
+        "tflops": round(step_flops * world / (ms_step / 1e3) / 1e12, 2),
+        "video_tokens_per_s": round(w.batch * w.n_video * world / (ms_step / 1e3), 1),
+        "parts_ms": {k_: round(v_, 4) for k_, v_ in part_ms.items()},
+        "flops_per_step": flops,
+        "dominant": {"kernel": "attn_tc_kernel (" + dom + ")", "achieved": round(achieved, 2),
+                     "peak": peak, "frac": round(achieved / peak, 4),
+                     "peak_source": f"{peak_key} (timed region {region_ms / 1e3:.2f} s)"},
+        "cross_frac": round(flops["cross"] / (part_ms["cross"] / 1e3) / 1e12 / peak, 4),
+        "step": "rope+select+sparse+cross" if L.sparse else "rope+joint+cross",
+        "launches_per_step": L.launches,
+    })
+    return res, L, x, window, step_flops
+
+
+def e2e_overlapped(L, x, args, dev, stream, world, step_flops):
+    """End-to-end steps through the same C-ABI calls from pinned host memory:
+    every step copies its Q, K, V in and its outputs (joint or sparse O and
+    the cross-attention O) out.  Two device sets of tensors alternate, so the
+    input copy of step i+1 (one copy stream) and the output copy of step i
+    (another) overlap the compute of the next step; the timed region runs from
+    the first input copy to the last output copy."""
+    import torch
+    M, w = L.M, L.w
+    pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hq, hk, hv = pin(x["q"]), pin(x["k"]), pin(x["v"])
+    ho = torch.empty(L.o.shape, dtype=L.o.dtype).pin_memory()
+    hoc = torch.empty(L.oc.shape, dtype=L.o.dtype).pin_memory()
+    sets = [L, Layer(M, w, x, dev)]
+    h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    n = max(2, min(args.steps, 6))
+    mk = lambda: [torch.cuda.Event() for _ in range(2)]
+    ev_in, ev_comp, ev_out = mk(), mk(), mk()
+
+    def h2d(i):
+        S = sets[i % 2]
+        if i >= 2:
+            h2d_s.wait_event(ev_comp[i % 2])  # step i-2 has finished with this set
+        with torch.cuda.stream(h2d_s):
+            S.q.copy_(hq, non_blocking=True)
+            S.k.copy_(hk, non_blocking=True)
+            S.v.copy_(hv, non_blocking=True)
+        ev_in[i % 2].record(h2d_s)
+
+    def run(n_steps, e0=None):
+        if e0 is not None:
+            h2d_s.wait_event(e0)
+        h2d(0)
+        for i in range(n_steps):
+            if i + 1 < n_steps:
+                h2d(i + 1)
+            S = sets[i % 2]
+            stream.wait_event(ev_in[i % 2])
+            if i >= 2:
+                stream.wait_event(ev_out[i % 2])  # outputs of step i-2 are out
+            S.step(stream)
+            ev_comp[i % 2].record(stream)
+            d2h_s.wait_event(ev_comp[i % 2])
+            with torch.cuda.stream(d2h_s):
+                ho.copy_(S.o, non_blocking=True)
+                hoc.copy_(S.oc, non_blocking=True)
+            ev_out[i % 2].record(d2h_s)
+        for j in range(min(2, n_steps)):
+            stream.wait_event(ev_out[(n_steps - 1 - j) % 2])
+
+    run(2)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    run(n, e0)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if M.device_status(stream) != 0:
+        raise RuntimeError("device status after the end-to-end steps: " + M.last_error())
+    ms = reduce_max(e0.elapsed_time(e1), world, dev) / n
+    h2d_b = 3 * L.q.numel() * L.q.element_size()
+    d2h_b = 2 * L.o.numel() * L.o.element_size()
+    sets.pop()
+    return {"value": round(step_flops * world / (ms / 1e3) / 1e12, 2), "unit": UNIT,
+            "h2d_bytes_per_step": h2d_b, "d2h_bytes_per_step": d2h_b, "ms_per_step": round(ms, 3),
+            "steps": n, "copy_gbs_needed": round((h2d_b + d2h_b) / (ms / 1e3) / 1e9, 1),
+            "note": "pinned host buffers; input copy of step i+1 and output copy of step i "
+                    "on two copy streams, overlapping the compute (two device sets)"}
+
+
 def run_gpu(args) -> int:
     import torch
 
@@ -301,174 +584,45 @@ def run_gpu(args) -> int:
     barrier(world, dev)
     from joint_video_audio_rope_b200 import mmdit as M
 
-    w = WL.WORKLOADS[args.workload]
-    x = WL.generate(w)
-    to_dev = lambda a: (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
-                        .to(dev, non_blocking=False))
-    q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
-    o = torch.empty_like(q)
-    o_cross = torch.empty_like(q)  # video and audio slices receive the cross outputs
-    desc = M.desc_of(q)
-    lay = M.make_layout(w.segments)
-    rope = M.rope_params(w.theta, 44, 42, 42)
-    scale = 1.0 / math.sqrt(w.head_dim)
-    v0, v1 = w.video_range()
-    a0, a1 = w.audio_range()
-    dv, da = M.desc_of(q[:, v0:v1]), M.desc_of(q[:, a0:a1])
-    ws_cross = M.av_cross_attn_workspace_size(dv, da)
-    sparse = w.sparse
-    if sparse:
-        vlay = M.make_layout([s for s in w.segments if s["kind"] == WL.SEG_VIDEO])
-        vd = M.desc_of(q[:, v0:v1])
-        nb = M.num_blocks(vlay)
-        idx = torch.empty((w.batch, w.heads, nb, nb), dtype=torch.int32, device=dev)
-        cnt = torch.empty((w.batch, w.heads, nb), dtype=torch.int32, device=dev)
-        ws_sel = M.block_select_workspace_size(vd, vlay)
-        ws_sp = M.sparse_attn_workspace_size(vd, vlay, nb)
-    else:
-        ws_sel = ws_sp = 0
-    ws = torch.empty(max(ws_cross, ws_sel, ws_sp, 256), dtype=torch.uint8, device=dev)
+    peaks, peak_src = read_peaks()
     stream = torch.cuda.current_stream(dev)
-    # RoPE works in place.  On the block-sparse workload the selected blocks (so
-    # the work) depend on the values, so every step starts from the generated
-    # Q and K (a device copy counted in the step); dense work does not depend
-    # on the values and the step rotates the previous step's tensors again.
-    q0k0 = (q.clone(), k.clone()) if sparse else None
+    w = WL.WORKLOADS[args.workload]
 
-    def step(ev=None):
-        if q0k0 is not None:
-            q.copy_(q0k0[0])
-            k.copy_(q0k0[1])
-        if ev is not None:
-            ev[0].record(stream)
-        M.rope_apply(q, k, desc, lay, rope, stream)
-        if ev is not None:
-            ev[1].record(stream)
-        if sparse:
-            M.block_select(q[:, v0:v1], k[:, v0:v1], vd, vlay, w.top_k, w.top_p, scale, nb, idx,
-                           cnt, ws, ws.numel(), stream)
-            if ev is not None:
-                ev[2].record(stream)
-            M.sparse_attn(q[:, v0:v1], k[:, v0:v1], v[:, v0:v1], o[:, v0:v1], vd, vlay, idx, cnt,
-                          nb, scale, ws, ws.numel(), stream)
-        else:
-            if ev is not None:
-                ev[2].record(stream)
-            M.joint_attn(q, k, v, o, desc, lay, scale, stream=stream)
-        if ev is not None:
-            ev[3].record(stream)
-        M.av_cross_attn(q[:, v0:v1], k[:, v0:v1], v[:, v0:v1], q[:, a0:a1], k[:, a0:a1],
-                        v[:, a0:a1], o_cross[:, v0:v1], o_cross[:, a0:a1], dv, da, scale, ws,
-                        ws.numel(), stream)
-        if ev is not None:
-            ev[4].record(stream)
-
-    # launches of this library's kernels per step
-    launches_per_step = 1 + (2 + 3 if sparse else 1) + 3
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    if M.device_status(stream) != 0:
-        raise RuntimeError("device status after warm-up: " + M.last_error())
-
-    flops = dense_step_flops(w)
-    if sparse:
-        # algorithmic work of sparse attention: selected token pairs only
-        cnt_h = cnt.cpu().numpy()
-        idx_h = idx.cpu().numpy()
-        seg = w.segments[0]
-        blen = np.array([_block_len(seg["T"], seg["H"], seg["W"], b) for b in range(nb)], np.int64)
-        pairs = 0
-        for b in range(w.batch):
-            for h in range(w.heads):
-                for i in range(nb):
-                    pairs += blen[i] * blen[idx_h[b, h, i, :cnt_h[b, h, i]]].sum()
-        flops = {"joint": 4.0 * pairs * w.head_dim, "cross": flops["cross"]}
-        density = float(cnt_h.mean() / nb)
-    step_flops = flops["joint"] + flops["cross"]
-
-    # ---------------------------------------------------------- timed region
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    # ---------------------------------------------------------- headline
     sampler = ClockSampler(local)
-    barrier(world, dev)
-    torch.cuda.synchronize(dev)
-    sampler.start()
-    time.sleep(0.3)
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    host_t0 = time.time()
-    t_start.record(stream)
-    for i in range(args.steps):
-        step(evs[i])
-    t_end.record(stream)
-    torch.cuda.synchronize(dev)
-    host_t1 = time.time()
+    head, L, x, window, step_flops = measure_workload(M, w, args, dev, stream, world, peaks,
+                                                      sampler)
     time.sleep(0.15)
-    clocks = sampler.stop((host_t0, host_t1))
-    barrier(world, dev)
-    if M.device_status(stream) != 0:
-        raise RuntimeError("device status after timing: " + M.last_error())
-    ms_total = reduce_max(t_start.elapsed_time(t_end), world, dev)
-    ms_step = ms_total / args.steps
-    part_ms = {name: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
-               for j, name in enumerate(["rope", "select" if sparse else "none",
-                                         "sparse" if sparse else "joint", "cross"])}
+    clocks = sampler.stop(window)
+    v0, v1 = L.v0, L.v1
+    q, k, v = L.q, L.k, L.v
 
     # --------------------------------------------- text cross-attention
     # The reinforced text cross-attention (video queries over the text keys)
-    # is a call of its own, outside the step the metric is defined on: timed
-    # here on its own, the same number of launches, after the same warm-up.
+    # is a call of its own, outside the step the metric is defined on.
     text_cross_ms = None
     tx0, tx1 = w.text_range()
     if tx1 > tx0:
         o_text = torch.empty_like(q)
         dtx = M.desc_of(k[:, tx0:tx1])
-
-        def text_cross():
-            M.text_cross_attn(q[:, v0:v1], k[:, tx0:tx1], v[:, tx0:tx1], o_text[:, v0:v1], dv, dtx,
-                              scale, stream)
-
-        for _ in range(args.warmup):
-            text_cross()
-        barrier(world, dev)
-        torch.cuda.synchronize(dev)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            text_cross()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        text_cross_ms = reduce_max(e0.elapsed_time(e1), world, dev) / args.steps
+        text_cross_ms = time_call(
+            lambda: M.text_cross_attn(q[:, v0:v1], k[:, tx0:tx1], v[:, tx0:tx1], o_text[:, v0:v1],
+                                      L.dv, dtx, L.scale, stream), args, dev, stream, world)
         if M.device_status(stream) != 0:
             raise RuntimeError("device status after the text cross-attention: " + M.last_error())
+        del o_text
 
     # ------------------------- mask-guided region-restricted attention
-    # Workloads that carry the mask M also time the Refiner's region-restricted
-    # attention (rows of masked video tokens only), as a separate call.
     masked_ms = None
-    if w.mask and not sparse:
+    n_masked_rows = int(np.count_nonzero(x["mask"])) if w.mask else 0  # one entry per video token
+    if w.mask and not L.sparse:
         o_mask = torch.empty_like(q)
         mask_dev = torch.from_numpy(x["mask"]).to(dev)
-        nmw = M.masked_joint_attn_workspace_size(desc, lay)
+        nmw = M.masked_joint_attn_workspace_size(L.desc, L.lay)
         ws_mask = torch.empty(nmw, dtype=torch.uint8, device=dev)
-
-        def masked():
-            M.masked_joint_attn(q, k, v, o_mask, desc, lay, scale, mask_dev, ws_mask, nmw, stream)
-
-        for _ in range(args.warmup):
-            masked()
-        barrier(world, dev)
-        torch.cuda.synchronize(dev)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            masked()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        masked_ms = reduce_max(e0.elapsed_time(e1), world, dev) / args.steps
+        masked_ms = time_call(
+            lambda: M.masked_joint_attn(q, k, v, o_mask, L.desc, L.lay, L.scale, mask_dev, ws_mask,
+                                        nmw, stream), args, dev, stream, world)
         if M.device_status(stream) != 0:
             raise RuntimeError("device status after the masked attention: " + M.last_error())
         del ws_mask, o_mask
@@ -476,8 +630,8 @@ def run_gpu(args) -> int:
     # ------------------------------------------- flow-matching elementwise
     # The noised input / velocity target and the loss term of the video
     # stream's latent (the video token grid x LATENT_CHANNELS values per item),
-    # separate calls: at the workload's batch (1 MB-scale tensors, launch-bound)
-    # and at a 64-item batch of the same latent (larger than L2, HBM-bound).
+    # separate calls: at the workload's batch and at a 64-item batch of the
+    # same latent (larger than L2, HBM-bound).
     flow = {}
     n_lat = w.n_video * LATENT_CHANNELS
     for label, items in (("workload_batch", w.batch), ("batch64", 64)):
@@ -489,100 +643,70 @@ def run_gpu(args) -> int:
         loss_l = torch.empty(items, device=dev)
         nfw = M.flow_loss_workspace_size(items, n_lat)
         ws_l = torch.empty(max(nfw, 256), dtype=torch.uint8, device=dev)
-        times = []
-        for fn in (lambda: M.flow_noise(z0_l, eps_l, t_l, zt_l, u_l, stream),
-                   lambda: M.flow_loss(v_l, z0_l, eps_l, loss_l, ws_l, nfw, stream)):
-            for _ in range(args.warmup):
-                fn()
-            torch.cuda.synchronize(dev)
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(args.steps):
-                fn()
-            e1.record(stream)
-            torch.cuda.synchronize(dev)
-            times.append(reduce_max(e0.elapsed_time(e1), world, dev) / args.steps)
-        nb = items * n_lat * 2
+        t_noise = time_call(lambda: M.flow_noise(z0_l, eps_l, t_l, zt_l, u_l, stream), args, dev,
+                            stream, world)
+        t_loss = time_call(lambda: M.flow_loss(v_l, z0_l, eps_l, loss_l, ws_l, nfw, stream), args,
+                           dev, stream, world)
+        nbytes = items * n_lat * 2
         flow[label] = {"items": items, "values_per_item": n_lat,
-                       "noise_us": round(times[0] * 1e3, 2),
-                       "noise_gbs": round(4 * nb / (times[0] / 1e3) / 1e9, 1),
-                       "loss_us": round(times[1] * 1e3, 2),
-                       "loss_gbs": round(3 * nb / (times[1] / 1e3) / 1e9, 1)}
+                       "noise_us": round(t_noise * 1e3, 2),
+                       "noise_gbs": round(4 * nbytes / (t_noise / 1e3) / 1e9, 1),
+                       "loss_us": round(t_loss * 1e3, 2),
+                       "loss_gbs": round(3 * nbytes / (t_loss / 1e3) / 1e9, 1)}
         del z0_l, eps_l, v_l, zt_l, u_l, ws_l
     if M.device_status(stream) != 0:
         raise RuntimeError("device status after the flow-matching kernels: " + M.last_error())
 
     # ---------------------------------------------------------- end to end
-    pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
-    hq, hk, hv = pin(x["q"]), pin(x["k"]), pin(x["v"])
-    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    hoc = torch.empty(o_cross.shape, dtype=o.dtype).pin_memory()
-    e2e_steps = max(1, min(args.steps, 5))
+    e2e = e2e_overlapped(L, x, args, dev, stream, world, step_flops)
+    del L, x, q, k, v
+    torch.cuda.empty_cache()
 
-    def e2e_step():
-        q.copy_(hq, non_blocking=True)
-        k.copy_(hk, non_blocking=True)
-        v.copy_(hv, non_blocking=True)
-        if q0k0 is not None:  # the fresh host inputs are the step's inputs
-            q0k0[0].copy_(q)
-            q0k0[1].copy_(k)
-        step()
-        ho.copy_(o, non_blocking=True)
-        hoc.copy_(o_cross, non_blocking=True)
-
-    e2e_step()
-    torch.cuda.synchronize(dev)
-    barrier(world, dev)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = reduce_max(e0.elapsed_time(e1), world, dev) / e2e_steps
-    h2d = 3 * q.numel() * q.element_size()
-    d2h = 2 * o.numel() * o.element_size()
+    # ------------------------------------------- the other workloads
+    per_config = {}
+    if not args.no_per_config:
+        for name in PER_CONFIG:
+            if name == w.name:
+                continue
+            r, Lc, xc, _, _ = measure_workload(M, WL.WORKLOADS[name], args, dev, stream, world,
+                                               peaks)
+            per_config[name] = r
+            del Lc, xc
+            torch.cuda.empty_cache()
 
     # ---------------------------------------------------------- report
-    peaks, peak_src = read_peaks()
-    dom = "sparse" if sparse else "joint"
-    dom_ms = part_ms[dom]
-    achieved = flops["joint"] / (dom_ms / 1e3) / 1e12
-    peak = peaks.get("bf16_tflops_sustained") or FALLBACK_PEAKS["bf16_tflops_sustained"]
-    value = step_flops * world / (ms_step / 1e3) / 1e12
-    tokens_s = w.batch * w.n_video * world / (ms_step / 1e3)
     if rank != 0:
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()
         return 0
+    dom = head["dominant"]
     line = {
-        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "metric": METRIC, "value": head["tflops"], "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "seq_len": w.n_tokens,
                    "video_tokens": w.n_video, "audio_tokens": w.n_audio, "heads": w.heads,
                    "head_dim": w.head_dim, "parallelism": f"replica x{world} (no collective)",
-                   "l2": "inputs larger than L2 (no flush needed)",
-                   "step": ("rope+select+sparse+cross" if sparse else "rope+joint+cross")},
-        "video_tokens_per_s": round(tokens_s, 1),
-        "frac_of_peak": round(value / world / peak, 4),
-        "parts_ms": {k_: round(v_, 4) for k_, v_ in part_ms.items() if k_ != "none"},
-        "flops_per_step": {k_: v_ for k_, v_ in flops.items()},
-        "e2e": {"value": round(step_flops * world / (e2e_ms / 1e3) / 1e12, 2), "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": round(e2e_ms, 3)},
-        "gpu_launches": launches_per_step * args.steps,
-        "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (" + dom + ")",
-                     "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": ncu_traffic(w.name),
+                   "l2": "inputs larger than L2 (no flush needed)", "step": head["step"]},
+        "video_tokens_per_s": head["video_tokens_per_s"],
+        "frac_of_peak": round(head["tflops"] / world / dom["peak"], 4),
+        "parts_ms": head["parts_ms"],
+        "flops_per_step": head["flops_per_step"],
+        "e2e": e2e,
+        "gpu_launches": head.pop("launches_per_step") * args.steps,
+        "roofline": {"bound": "tensor", "kernel": dom["kernel"], "achieved": dom["achieved"],
+                     "peak": dom["peak"], "unit": "TFLOP/s", "frac": dom["frac"],
+                     "traffic": ncu_traffic(w.name),
                      "traffic_unit": "bytes per launch (ncu dram read + write)",
-                     "peak_source": f"bf16_tflops_sustained of {peak_src}"},
+                     "peak_source": f"{dom['peak_source']} of {peak_src}"},
+        "cross_frac": head["cross_frac"],
         "clocks": clocks,
     }
+    if "block_density" in head:
+        line["block_density"] = head["block_density"]
+    peak = dom["peak"]
     if text_cross_ms is not None:
         tf = attn_flops(w.n_video, tx1 - tx0, w.head_dim, w.heads, w.batch)
         line["text_cross"] = {"ms": round(text_cross_ms, 4), "flops": tf,
@@ -591,7 +715,7 @@ def run_gpu(args) -> int:
                               "text_tokens": tx1 - tx0, "launches": args.steps,
                               "note": "separate call, not part of the step or its value"}
     if masked_ms is not None:
-        n_rows = int(np.count_nonzero(x["mask"]))  # one mask entry per video token
+        n_rows = n_masked_rows
         mf = 4.0 * n_rows * w.n_tokens * w.head_dim * w.heads
         line["masked_joint"] = {"ms": round(masked_ms, 4), "flops": mf,
                                 "tflops": round(mf / (masked_ms / 1e3) / 1e12, 2),
@@ -605,10 +729,10 @@ def run_gpu(args) -> int:
         f_["loss_frac_hbm"] = round(f_["loss_gbs"] / hbm, 4)
     line["flow_matching"] = dict(flow, note="separate calls on bf16 latents; bytes = 2 reads + 2 "
                                             "writes (noise) or 3 reads (loss) per value")
-    if sparse:
-        line["block_density"] = round(density, 4)
+    if per_config:
+        line["per_config"] = per_config
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, x, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(w, WL.generate(w), args.cpu_seconds)
     print(json.dumps(line), flush=True)
     return 0
 
@@ -662,7 +786,9 @@ def main(argv=None) -> int:
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="480p", choices=sorted(WL.WORKLOADS))
+    ap.add_argument("--workload", default="720p_cond_b2", choices=sorted(WL.WORKLOADS))
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time only the headline workload")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -52,7 +52,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
     if not force and not _stale():
         return OUT
     os.makedirs(BUILD, exist_ok=True)
-    objs = []
+    objs, cmds = [], []
     for src in sources():
         obj = os.path.join(BUILD, os.path.basename(src) + ".o")
         cmd = [nvcc(), *ARCH, *FLAGS, "-c", src, "-o", obj]
@@ -60,8 +60,15 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
             cmd += ["-Xptxas", "-v"]
         if verbose:
             print(" ".join(cmd), flush=True)
-        subprocess.run(cmd, check=True)
+        cmds.append(cmd)
         objs.append(obj)
+    # the translation units are independent: compile them concurrently
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max(1, min(len(cmds), os.cpu_count() or 1))) as ex:
+        for r in ex.map(lambda c: subprocess.run(c, capture_output=True, text=True), cmds):
+            if r.stdout or r.stderr:
+                print(r.stdout + r.stderr, end="", flush=True)
+            r.check_returncode()
     tmp = OUT + ".tmp"
     cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-Xcompiler", "-fPIC"]
     if verbose:

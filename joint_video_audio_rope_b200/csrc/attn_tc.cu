@@ -43,9 +43,9 @@ constexpr int kHalfCol = 128 * 128;       // bytes of one 64-channel column half
 constexpr int kBoxBytes = 64 * 128;       // one TMA box: 64 rows x 64 channels
 
 // Kernel shape: QT Q tiles of 128 rows per CTA (one softmax warpgroup each)
-// and an ST-slot K/V ring.  QT = 2 fills the SM (198 KB smem, 512 TMEM
+// and an ST-slot K/V ring.  QT = 2 fills the SM (225 KB smem, 512 TMEM
 // columns) and lets the two tiles ping-pong on the tensor core; QT = 1 with a
-// 2-slot ring needs 97 KB and 256 columns, so two CTAs share an SM and hide
+// 2-slot ring needs 105 KB and 256 columns, so two CTAs share an SM and hide
 // each other's load and epilogue latency (used for short key sequences).
 template <int QT, int ST>
 struct Cfg {
@@ -81,16 +81,6 @@ struct Cfg {
   static_assert(128 * (QT * kRegsHigh + kRegsLow) <= kThreads * kRegsLaunch, "register split");
 };
 constexpr float kRescaleLog2 = 8.0f;      // move the max only beyond a factor 2^8
-// 32-column chunks of S whose exponentials run on the FMA pipe (polynomial)
-// instead of the MUFU, on tiles without masked columns: bit c = chunk c.
-// Measured on B200 (480p joint attention): 0 chunks 1113 TFLOP/s, 1 chunk
-// 961, 2 chunks 849 -- the softmax is bound by the latency of its per-tile
-// handoffs, not by MUFU throughput, so the default keeps every exponential on
-// the MUFU.
-#ifndef MMDIT_POLY_CHUNKS
-#define MMDIT_POLY_CHUNKS 0x0
-#endif
-constexpr int kPolyChunks = MMDIT_POLY_CHUNKS;
 
 // barrier indices (8 bytes each)
 // Phases: Q, O and their "empty" barriers complete once per work item; S and
@@ -589,27 +579,19 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
         }
         const float mref = (m_used == -INFINITY) ? 0.f : m_used * sl2;
         const uint64_t nm2 = pack_f32x2(-mref, -mref);
-        // Exponentials: MUFU ex2 for most columns; on tiles without masked
-        // columns, the columns of kPolyChunks go to the FMA pipe instead.
-        const bool poly_ok = !__any_sync(0xffffffffu, masked);
+        // exponentials on the MUFU (ex2), arguments formed two at a time
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
-          const bool poly = poly_ok && ((kPolyChunks >> c) & 1);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const uint64_t x2 = ffma_f32x2(pack_f32x2(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]),
                                            sl2x2, nm2);
             float p0, p1;
-            if (poly) {
-              exp2_poly_f32x2(x2, p0, p1);
-            } else {
-              float x0, x1;
-              unpack_f32x2(x2, x0, x1);
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
-            }
+            unpack_f32x2(x2, p0, p1);
+            p0 = ex2_approx(p0);
+            p1 = ex2_approx(p1);
             pk[i] = pack_bf16x2(p0, p1);
             acc[i & 3] = add_f32x2(acc[i & 3], pack_f32x2(p0, p1));
           }
@@ -820,21 +802,22 @@ __global__ void __launch_bounds__(256) split_combine_kernel(const float* __restr
 template <int QT, int ST, bool PERSIST>
 cudaError_t launch_shape(const AttnParams& p, cudaStream_t s) {
   using C = Cfg<QT, ST>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<QT, ST, PERSIST>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  // the dynamic shared-memory limit is a per-device function attribute
+  e = once_per_device(dev, [] {
+    return cudaFuncSetAttribute(attn_tc_kernel<QT, ST, PERSIST>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  });
+  if (e != cudaSuccess) return e;
   const int items = p.prob.ctas;
   if (items == 0) return cudaSuccess;
   int grid = items;
   if (PERSIST) {
     // one CTA per resident slot; each CTA walks items blockIdx.x + k*gridDim.x
-    int dev = 0, sms = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     grid = std::min(items, sms * C::kMinBlocks);
   }

@@ -381,34 +381,6 @@ __device__ __forceinline__ float row_max128(const float (&s)[128]) {
   return max3f(max3f(a[0], a[1], a[2]), max3f(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
 }
 
-// 2^x on the FMA pipe for two lanes, x <= 8 (used on part of the softmax
-// columns to unload the MUFU).  Range reduction after Cody and Waite: j =
-// round(x) by the 1.5*2^23 shift, f = x - j in [-1/2, 1/2] exactly; 2^f by a
-// degree-3 polynomial fitted for relative error (coefficients from
-// csrc/fit_exp2_poly.py, max relative error 7.5e-5 in fp32); 2^j is added to
-// the exponent field: bits(t) << 23 equals j << 23 modulo 2^32 because the
-// shift constant's low nine bits are zero.  x is clamped at -125 so the result
-// stays a normal number (values that small vanish against the row sum >= 1).
-__device__ __forceinline__ void exp2_poly_f32x2(uint64_t x2, float& p0, float& p1) {
-  float x0, x1;
-  unpack_f32x2(x2, x0, x1);
-  const uint64_t x = pack_f32x2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-  const uint64_t magic = pack_f32x2(12582912.f, 12582912.f);
-  const uint64_t nmagic = pack_f32x2(-12582912.f, -12582912.f);
-  const uint64_t t = add_f32x2(x, magic);
-  const uint64_t jf = add_f32x2(t, nmagic);
-  const uint64_t f = ffma_f32x2(jf, pack_f32x2(-1.f, -1.f), x);
-  uint64_t p = ffma_f32x2(pack_f32x2(0.05517132207751274f, 0.05517132207751274f), f,
-                          pack_f32x2(0.24261054396629333f, 0.24261054396629333f));
-  p = ffma_f32x2(p, f, pack_f32x2(0.6932609677314758f, 0.6932609677314758f));
-  p = ffma_f32x2(p, f, pack_f32x2(0.9999281167984009f, 0.9999281167984009f));
-  float pa, pb, ta, tb;
-  unpack_f32x2(p, pa, pb);
-  unpack_f32x2(t, ta, tb);
-  p0 = __int_as_float(__float_as_int(pa) + (__float_as_int(ta) << 23));
-  p1 = __int_as_float(__float_as_int(pb) + (__float_as_int(tb) << 23));
-}
-
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -25,6 +25,7 @@ __global__ void wait_timeout_kernel(int* err, uint64_t limit_ns, int* waited) {
 using namespace mmdit;
 
 extern "C" int mmdit_selftest_wait_timeout(int limit_ms, int* waited_out, mmdit_stream_t stream) {
+  MMDIT_NVTX("mmdit_selftest_wait_timeout");
   if (limit_ms < 1 || limit_ms > 2000)
     return fail(MMDIT_EINVAL, "selftest: limit_ms must be in [1, 2000]");
   if (waited_out == nullptr || (reinterpret_cast<uintptr_t>(waited_out) & 3u) != 0)

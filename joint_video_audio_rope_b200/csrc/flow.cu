@@ -178,6 +178,7 @@ extern "C" {
 int mmdit_flow_noise(const void* z0, const void* eps, const float* t, void* zt, void* u,
                      int32_t batch, int64_t n, int64_t stride, int32_t dtype,
                      mmdit_stream_t stream) {
+  MMDIT_NVTX("mmdit_flow_noise");
   int rc = check_flow("flow_noise", batch, n, stride, dtype, {z0, eps, zt, u});  // t: scalar reads
   if (rc) return rc;
   if (!z0 || !eps || !t) return fail(MMDIT_EINVAL, "flow_noise: z0, eps, t must be non-NULL");
@@ -207,6 +208,7 @@ size_t mmdit_flow_loss_workspace_size(int32_t batch, int64_t n) {
 int mmdit_flow_loss(const void* v, const void* z0, const void* eps, float* loss, int32_t batch,
                     int64_t n, int64_t stride, int32_t dtype, void* workspace, size_t ws_bytes,
                     mmdit_stream_t stream) {
+  MMDIT_NVTX("mmdit_flow_loss");
   int rc = check_flow("flow_loss", batch, n, stride, dtype, {v, z0, eps});
   if (rc) return rc;
   if (!v || !z0 || !eps || !loss)

@@ -6,9 +6,44 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <nvtx3/nvToolsExt.h>
+
+#include <atomic>
+#include <mutex>
+
 #include "common.cuh"
 
 namespace mmdit {
+
+// NVTX range around one C-ABI call (named after the call), so that a
+// profiler timeline shows which library call launched which kernels.  The
+// NVTX header is a no-op unless a tool injects itself.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define MMDIT_NVTX(name) ::mmdit::NvtxRange mmdit_nvtx_range_(name)
+
+constexpr int kMaxDevices = 64;  // device indices the per-device state covers
+constexpr int kMaxBlocks = 6000; // key/query blocks of one block-sparse problem
+
+// Runs fn() (returning cudaError_t) once per device index for each call site
+// (each lambda type has its own state), thread-safe; a failed fn() is retried
+// on the next call.  Used for per-device function attributes.
+template <typename F>
+cudaError_t once_per_device(int dev, F fn) {
+  static std::atomic<bool> done[kMaxDevices] = {};
+  static std::mutex mu;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+  const cudaError_t e = fn();
+  if (e == cudaSuccess) done[dev].store(true, std::memory_order_release);
+  return e;
+}
 
 // RoPE (rope.cu)
 cudaError_t launch_rope(void* q, void* k, const mmdit_tensor_desc& d, const DevLayout& L,
@@ -75,6 +110,14 @@ int launch_cross(const void* qv, const void* kv, const void* vv, const void* qa,
                  const void* va, void* o_video, void* o_audio, const mmdit_tensor_desc& video,
                  const mmdit_tensor_desc& audio, float scale, int splits, int kv_per_split,
                  float* part_o, float* part_ml, cudaStream_t s);
+// Split of the video keys for the audio-query direction of the cross
+// attention (mmdit_api.cu): audio query tiles of 256 rows, `splits` key ranges
+// of kv_per_split tokens (a multiple of 128), and the partial-result sizes.
+struct CrossPlan {
+  int n_qtiles_a, splits, kv_per_split, nq_pad;
+  size_t part_o_bytes, part_ml_bytes;
+};
+CrossPlan plan_cross(const mmdit_tensor_desc* video, const mmdit_tensor_desc* audio);
 int attn_rows_per_cta(int q_tiles);  // query rows one CTA covers
 int attn_store_cols(int q_tiles);    // channels per output store box
 cudaError_t launch_split_combine(const float* part_o, const float* part_ml, __nv_bfloat16* o,
@@ -84,10 +127,7 @@ cudaError_t launch_split_combine(const float* part_o, const float* part_ml, __nv
 // block-sparse attention: query blocks per CTA group are bounded by the rows
 // of the kernel shape used (kSparseQTiles 128-row Q tiles) and 8 blocks per
 // Q tile (membership masks are 16 bits wide)
-#ifndef MMDIT_SPARSE_QTILES
-#define MMDIT_SPARSE_QTILES 2
-#endif
-constexpr int kSparseQTiles = MMDIT_SPARSE_QTILES;
+constexpr int kSparseQTiles = 2;
 constexpr int kGroupTokens = 128 * kSparseQTiles;
 constexpr int kGroupBlocks = 8 * kSparseQTiles;
 

@@ -145,6 +145,7 @@ int mmdit_masked_joint_attn(const void* q, const void* k, const void* v, void* o
                             const mmdit_tensor_desc* desc, const mmdit_layout* layout,
                             float scale, const uint8_t* mask, int64_t mask_elems,
                             void* workspace, size_t ws_bytes, mmdit_stream_t stream) {
+  MMDIT_NVTX("mmdit_masked_joint_attn");
   int rc = check_desc(desc, "masked_joint");
   if (rc) return rc;
   if (desc->dtype != MMDIT_BF16) return fail(MMDIT_EUNSUPPORTED, "masked_joint: bf16 only");

@@ -193,8 +193,8 @@ int sparse_layout(const mmdit_layout* L, const mmdit_tensor_desc* d, int& T, int
   H = L->seg[0].H;
   W = L->seg[0].W;
   const long long nb = (long long)((T + 3) / 4) * ((H + 3) / 4) * ((W + 3) / 4);
-  if (nb > 6000)
-    return fail(MMDIT_EUNSUPPORTED, "%lld blocks; at most 6000 are supported", nb);
+  if (nb > kMaxBlocks)
+    return fail(MMDIT_EUNSUPPORTED, "%lld blocks; at most %d are supported", nb, kMaxBlocks);
   nblk = (int)nb;
   return MMDIT_OK;
 }
@@ -222,11 +222,6 @@ int host_group_count(int T, int H, int W, int nblk) {
   return g + (nb > 0 ? 1 : 0);
 }
 
-struct CrossPlan {
-  int n_qtiles_a, splits, kv_per_split, nq_pad;
-  size_t part_o_bytes, part_ml_bytes;
-};
-
 // Split of the video keys for the audio-query direction: enough splits that
 // the (few) audio query tiles x heads x batch fill one wave of the B200's 148
 // SMs, each split a whole number of 128-key tiles.  One wave of long items
@@ -236,10 +231,7 @@ constexpr int kCrossTargetCtas = 148;
 
 // Q tiles per CTA of video queries over a short key sequence (audio, text):
 // one tile, two CTAs per SM (measured faster than two tiles with resident K/V).
-#ifndef MMDIT_SHORT_KV_QTILES
-#define MMDIT_SHORT_KV_QTILES 1
-#endif
-constexpr int kShortKvQTiles = MMDIT_SHORT_KV_QTILES;
+constexpr int kShortKvQTiles = 1;
 
 // Q tiles per CTA of the dense joint attention: two, one CTA per SM.
 constexpr int kJointQTiles = 2;
@@ -337,15 +329,21 @@ int launch_cross(const void* qv, const void* kv, const void* vv, const void* qa,
 }
 
 int* device_error_flag() {
-  static int* cache[64] = {};
+  static std::atomic<int*> cache[kMaxDevices] = {};
+  static std::mutex mu;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (cache[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_error_word) != cudaSuccess) return nullptr;
-    cache[dev] = static_cast<int*>(p);
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  int* p = cache[dev].load(std::memory_order_acquire);
+  if (p != nullptr) return p;
+  std::lock_guard<std::mutex> lock(mu);
+  p = cache[dev].load(std::memory_order_relaxed);
+  if (p == nullptr) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_device_error_word) != cudaSuccess) return nullptr;
+    p = static_cast<int*>(a);
+    cache[dev].store(p, std::memory_order_release);
   }
-  return cache[dev];
+  return p;
 }
 
 }  // namespace mmdit
@@ -382,6 +380,7 @@ int mmdit_device_status(mmdit_stream_t stream) {
 
 int mmdit_rope_apply(void* q, void* k, const mmdit_tensor_desc* desc, const mmdit_layout* layout,
                      const mmdit_rope_params* rope, mmdit_stream_t stream) {
+  MMDIT_NVTX("mmdit_rope_apply");
   int rc = check_desc(desc, "rope");
   if (rc) return rc;
   if (q == nullptr && k == nullptr) return fail(MMDIT_EINVAL, "rope: q and k are both NULL");
@@ -401,6 +400,7 @@ int mmdit_joint_attn(const void* q, const void* k, const void* v, void* o, float
                      const mmdit_tensor_desc* desc, const mmdit_layout* layout, float scale,
                      const mmdit_rope_params* rope_q, const uint8_t* cond_mask, int64_t mask_elems,
                      void*, size_t, mmdit_stream_t stream) {
+  MMDIT_NVTX("mmdit_joint_attn");
   int rc = check_desc(desc, "joint_attn");
   if (rc) return rc;
   if (!q || !k || !v || !o) return fail(MMDIT_EINVAL, "joint_attn: q, k, v, o must be non-NULL");
@@ -486,6 +486,7 @@ int mmdit_av_cross_attn(const void* qv, const void* kv, const void* vv, const vo
                         const void* ka, const void* va, void* o_video, void* o_audio,
                         const mmdit_tensor_desc* video, const mmdit_tensor_desc* audio,
                         float scale, void* workspace, size_t ws_bytes, mmdit_stream_t stream) {
+  MMDIT_NVTX("mmdit_av_cross_attn");
   int rc;
   if ((rc = check_desc(video, "video")) || (rc = check_desc(audio, "audio"))) return rc;
   if (video->batch != audio->batch || video->heads != audio->heads ||
@@ -529,6 +530,7 @@ int mmdit_av_cross_attn(const void* qv, const void* kv, const void* vv, const vo
 int mmdit_text_cross_attn(const void* qv, const void* kt, const void* vt, void* o_video,
                           const mmdit_tensor_desc* video, const mmdit_tensor_desc* text,
                           float scale, mmdit_stream_t stream) {
+  MMDIT_NVTX("mmdit_text_cross_attn");
   int rc;
   if ((rc = check_desc(video, "video")) || (rc = check_desc(text, "text"))) return rc;
   if (video->batch != text->batch || video->heads != text->heads ||
@@ -573,6 +575,7 @@ int mmdit_block_select(const void* q, const void* k, const mmdit_tensor_desc* de
                        const mmdit_layout* layout, int top_k, float top_p, float scale, int cap,
                        int32_t* block_idx, int32_t* block_cnt, void* workspace, size_t ws_bytes,
                        mmdit_stream_t stream) {
+  MMDIT_NVTX("mmdit_block_select");
   int rc = check_desc(desc, "block_select");
   if (rc) return rc;
   if (desc->dtype != MMDIT_BF16) return fail(MMDIT_EUNSUPPORTED, "block_select: bf16 only");
@@ -615,6 +618,7 @@ int mmdit_sparse_attn(const void* q, const void* k, const void* v, void* o,
                       const mmdit_tensor_desc* desc, const mmdit_layout* layout,
                       const int32_t* block_idx, const int32_t* block_cnt, int cap, float scale,
                       void* workspace, size_t ws_bytes, mmdit_stream_t stream) {
+  MMDIT_NVTX("mmdit_sparse_attn");
   int rc = check_desc(desc, "sparse_attn");
   if (rc) return rc;
   if (desc->dtype != MMDIT_BF16) return fail(MMDIT_EUNSUPPORTED, "sparse_attn: bf16 only");

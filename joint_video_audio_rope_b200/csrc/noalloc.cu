@@ -61,6 +61,7 @@ extern "C" int mmdit_av_cross_attn_noalloc(const void* qv, const void* kv, const
                                            const mmdit_tensor_desc* video,
                                            const mmdit_tensor_desc* audio, float scale,
                                            mmdit_stream_t stream) {
+  MMDIT_NVTX("mmdit_av_cross_attn_noalloc");
   int rc;
   if ((rc = check_desc(video, "video")) || (rc = check_desc(audio, "audio"))) return rc;
   if (video->batch != audio->batch || video->heads != audio->heads ||
@@ -78,18 +79,17 @@ extern "C" int mmdit_av_cross_attn_noalloc(const void* qv, const void* kv, const
   if (!(scale > 0.f) || !isfinite(scale))
     return fail(MMDIT_EINVAL, "av_cross_noalloc: scale must be > 0");
 
-  // Split the video keys of the audio-query direction as the regular call
-  // does (<= 32 key tiles per split), then lower the split count until the
-  // partial results fit the fixed scratch array.
-  const int n_qtiles = (audio->n_tokens + 255) / 256;
-  const int nq_pad = n_qtiles * 256;
+  // Start from the split of the video keys that the regular call uses (one
+  // wave of audio-query items over the SMs), then lower the split count until
+  // the partial results fit the fixed scratch array.
+  const CrossPlan plan = plan_cross(video, audio);
   const int tiles = (video->n_tokens + 127) / 128;
-  const size_t rows_per_split = (size_t)audio->batch * audio->heads * nq_pad;
+  const size_t rows_per_split = (size_t)audio->batch * audio->heads * plan.nq_pad;
   auto bytes_for = [&](int splits) {
     return align256((size_t)splits * rows_per_split * 128 * sizeof(float)) +
            align256((size_t)splits * rows_per_split * 2 * sizeof(float));
   };
-  int splits = std::max(1, (tiles + 31) / 32);
+  int splits = plan.splits;
   while (splits > 1 && bytes_for(splits) > (size_t)MMDIT_NOALLOC_SCRATCH_BYTES) --splits;
   if (bytes_for(splits) > (size_t)MMDIT_NOALLOC_SCRATCH_BYTES)
     return fail(MMDIT_EINVAL,

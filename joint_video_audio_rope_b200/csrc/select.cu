@@ -415,8 +415,14 @@ cudaError_t launch_select_vpl(const float* qbar, const float* kbar, int B, int H
                               int top_k, float top_p, float scale, int cap, int32_t* idx,
                               int32_t* cnt, cudaStream_t s) {
   const size_t smem = select_smem_bytes(nblk);
-  cudaError_t e = cudaFuncSetAttribute(select_kernel<VPL>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // the attribute is raised to the largest size this library uses, once per device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess)
+    e = once_per_device(dev, [] {
+      return cudaFuncSetAttribute(select_kernel<VPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)select_smem_bytes(kMaxBlocks));
+    });
   if (e != cudaSuccess) return e;
   dim3 grid((nblk + kSelRows - 1) / kSelRows, H, B);
   select_kernel<VPL><<<grid, 256, smem, s>>>(qbar, kbar, H, nblk, top_k, top_p, scale, cap, idx,
@@ -452,11 +458,14 @@ cudaError_t launch_union(const int32_t* idx, const int32_t* cnt, int cap, const 
                          int Wg, uint4* ulist, int* ucnt, cudaStream_t s) {
   if (n_groups == 0) return cudaSuccess;
   const size_t smem = sizeof(uint32_t) * (size_t)nblk;
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-  }
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess)
+    e = once_per_device(dev, [] {
+      return cudaFuncSetAttribute(union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)(sizeof(uint32_t) * kMaxBlocks));
+    });
+  if (e != cudaSuccess) return e;
   union_kernel<<<dim3(n_groups, H, B), 256, smem, s>>>(idx, cnt, cap, groups, H, nblk, n_groups,
                                                        T, Hg, Wg, ulist, ucnt);
   return cudaGetLastError();

@@ -5,7 +5,10 @@ bench) and the fp64 oracle.  It holds configuration and random-number
 generation only -- none of the attention, RoPE, pooling or selection
 arithmetic.  Inputs are drawn in float32 from numpy's PCG64 with a fixed seed
 and, for bf16 workloads, rounded to bfloat16 (round to nearest even) once;
-the same bits go to the GPU and to the oracle.
+the same bits go to the GPU and to the oracle.  Tensors are drawn in chunks
+of tokens, each chunk from its own stream spawned from the workload seed, so
+that several threads can draw them and the values still depend on the seed
+alone.
 
 Layouts follow the sequence order [conditioning frames (t<0) | video | audio
 | text] of one batch item.  Audio tokens use the 21/218 temporal scale that
@@ -13,6 +16,7 @@ makes 218 audio tokens span 21 latent frames (SkyReels-V4 digest, novelty 5).
 """
 from __future__ import annotations
 
+import os
 from dataclasses import dataclass, field
 from typing import Dict, List, Optional, Tuple
 
@@ -218,29 +222,61 @@ def _mask(w: Workload, rng) -> np.ndarray:
     return m
 
 
-def generate(w: Workload) -> Dict[str, np.ndarray]:
+GEN_CHUNK_TOKENS = 2048  # tokens of one independently seeded generation chunk
+
+
+def _fill_chunk(out, name_idx, w, seed_seq, t0, t1, std, bump):
+    """Draw tokens [t0, t1) of one tensor from its own PCG64 stream (child
+    `seed_seq` of the workload seed), scale, add the planted bump, round."""
+    rng = np.random.Generator(np.random.PCG64(seed_seq))
+    x = rng.standard_normal((w.batch, t1 - t0, w.heads, w.head_dim), dtype=np.float32)
+    x *= np.float32(std)
+    if bump is not None and name_idx < 2:
+        x += bump[None, t0:t1, None, None]
+    out[:, t0:t1] = f32_to_bf16_bits(x) if w.dtype == "bf16" else x
+
+
+def generate(w: Workload, threads: Optional[int] = None) -> Dict[str, np.ndarray]:
     """Q, K, V [B, N, heads, d] (+ mask).  bf16 workloads return uint16 bit
-    patterns under 'q','k','v'; f32 workloads return float32 arrays."""
-    rng = np.random.Generator(np.random.PCG64(w.seed))
-    shape = (w.batch, w.n_tokens, w.heads, w.head_dim)
-    out = {}
-    for name, std in (("q", w.qk_std), ("k", w.qk_std), ("v", w.v_std)):
-        x = rng.standard_normal(shape, dtype=np.float32)
-        x *= np.float32(std)
-        out[name] = x
+    patterns under 'q','k','v'; f32 workloads return float32 arrays.
+
+    Every tensor is drawn in chunks of GEN_CHUNK_TOKENS tokens (all batch
+    items, heads and channels of those tokens), each from its own PCG64
+    stream spawned from the workload seed (numpy SeedSequence), so the values
+    do not depend on how many threads draw them.  The planted regions and the
+    mask have streams of their own."""
+    root = np.random.SeedSequence(w.seed)
+    n = w.n_tokens
+    n_chunks = max(1, -(-n // GEN_CHUNK_TOKENS))
+    kids = root.spawn(3 * n_chunks + 2)
+    bump = None
     if w.planted_regions:
+        rng_b = np.random.Generator(np.random.PCG64(kids[3 * n_chunks]))
+        bump = np.zeros(n, np.float32)
         start = 0
         for s in w.segments:
             if s["kind"] == SEG_VIDEO:
-                bump = _planted_bump(s, w.planted_regions, w.planted_amp, rng)
-                for name in ("q", "k"):
-                    out[name][:, start:start + s["n_tokens"]] += bump[None, :, None, None]
+                bump[start:start + s["n_tokens"]] = _planted_bump(s, w.planted_regions,
+                                                                  w.planted_amp, rng_b)
             start += s["n_tokens"]
-    if w.dtype == "bf16":
-        for name in ("q", "k", "v"):
-            out[name] = f32_to_bf16_bits(out[name])
+    shape = (w.batch, n, w.heads, w.head_dim)
+    dt = np.uint16 if w.dtype == "bf16" else np.float32
+    out = {name: np.empty(shape, dt) for name in ("q", "k", "v")}
+    jobs = []
+    for ti, (name, std) in enumerate((("q", w.qk_std), ("k", w.qk_std), ("v", w.v_std))):
+        for c in range(n_chunks):
+            t0, t1 = c * GEN_CHUNK_TOKENS, min(n, (c + 1) * GEN_CHUNK_TOKENS)
+            jobs.append((out[name], ti, w, kids[ti * n_chunks + c], t0, t1, std, bump))
+    workers = threads or min(32, os.cpu_count() or 1)
+    if workers > 1 and len(jobs) > 1:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(workers) as ex:
+            list(ex.map(lambda j: _fill_chunk(*j), jobs))
+    else:
+        for j in jobs:
+            _fill_chunk(*j)
     if w.mask:
-        out["mask"] = _mask(w, rng)
+        out["mask"] = _mask(w, np.random.Generator(np.random.PCG64(kids[3 * n_chunks + 1])))
     return out
 
 

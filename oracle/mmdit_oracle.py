@@ -349,20 +349,17 @@ def pool(x: np.ndarray, blocks) -> np.ndarray:
     return out
 
 
-def select_row(qbar_i: np.ndarray, kbar: np.ndarray, top_k: int, top_p: float,
-               scale: float) -> np.ndarray:
-    """Attended key-block set of one query block ([PRISM] Method 3).
+def select_from_probs(P: np.ndarray, top_k: int, top_p: float) -> np.ndarray:
+    """The attended set S_i = Top-k(P_i, k) U Top-p(P_i, p) of one row of
+    block probabilities ([PRISM] Method 3).
 
-    P_i = softmax_j(qbar_i . kbar_j * scale).  Blocks are ordered by P
-    descending, ties by block id ascending.  Top-k takes the first
-    min(k, n) blocks; Top-p takes the shortest prefix whose cumulative
-    probability reaches p (the block that crosses p is included; if
-    rounding keeps the sum below p, every block).  S_i is their union,
+    Blocks are ordered by P descending, ties by block id ascending.  Top-k
+    takes the first min(k, n) blocks; Top-p takes the shortest prefix whose
+    cumulative probability reaches p (the block that crosses p is included;
+    if rounding keeps the sum below p, every block).  S_i is their union,
     returned in ascending block id.
     """
-    s = (kbar @ qbar_i) * scale
-    e = np.exp(s - s.max())
-    P = e / e.sum()
+    P = np.asarray(P, np.float64)
     n = P.shape[0]
     order = sorted(range(n), key=lambda j: (-P[j], j))
     n_k = min(top_k, n)
@@ -375,6 +372,36 @@ def select_row(qbar_i: np.ndarray, kbar: np.ndarray, top_k: int, top_p: float,
             break
     chosen = order[:max(n_k, n_p)]
     return np.asarray(sorted(chosen), dtype=np.int64)
+
+
+def select_row(qbar_i: np.ndarray, kbar: np.ndarray, top_k: int, top_p: float,
+               scale: float) -> np.ndarray:
+    """Attended key-block set of one query block ([PRISM] Method 3):
+    P_i = softmax_j(qbar_i . kbar_j * scale), then ``select_from_probs``."""
+    return select_from_probs(block_probs(qbar_i, kbar, scale), top_k, top_p)
+
+
+def select_rows(qbar: np.ndarray, kbar: np.ndarray, top_k: int, top_p: float,
+                scale: float) -> List[np.ndarray]:
+    """``select_row`` for every query block of one (batch, head), for many
+    rows at once: qbar [nq, d], kbar [nk, d] -> list of nq int arrays.
+
+    The same definition written with array steps: the block softmax of every
+    row, the ranking by a stable sort of -P (equal probabilities keep
+    ascending block ids), the running sum along the ranking, the first
+    position where it reaches p (every block if none), and the union with the
+    first min(k, n) ranked blocks, returned in ascending id.
+    """
+    s = (np.asarray(qbar, np.float64) @ np.asarray(kbar, np.float64).T) * scale
+    e = np.exp(s - s.max(axis=1, keepdims=True))
+    P = e / e.sum(axis=1, keepdims=True)
+    n = P.shape[1]
+    order = np.argsort(-P, axis=1, kind="stable")
+    csum = np.cumsum(np.take_along_axis(P, order, axis=1), axis=1)
+    reached = csum >= top_p
+    n_p = np.where(reached.any(axis=1), reached.argmax(axis=1) + 1, n)
+    n_sel = np.maximum(min(top_k, n), n_p)
+    return [np.sort(order[i, :n_sel[i]]).astype(np.int64) for i in range(P.shape[0])]
 
 
 def block_probs(qbar_i, kbar, scale):

@@ -67,25 +67,59 @@ def assert_close(got, ref, dtype: str, what: str = ""):
     return max_abs, rel
 
 
-def selection_matches(got: np.ndarray, ref: np.ndarray, P: np.ndarray, top_k: int, top_p: float,
-                      tol: float = 1e-6) -> bool:
-    """True if the GPU set equals the oracle set, or differs only in blocks
-    tied with the cutoff within fp32 resolution: a differing block j is
-    excused when |P_j - P_cut| <= tol * P_cut, where P_cut is the smallest
-    probability the oracle selected; the whole row is excused when the
-    oracle's cumulative sum at its top-p cutoff is within tol of p."""
-    g, r = set(got.tolist()), set(ref.tolist())
+def selection_verdict(got: np.ndarray, ref: np.ndarray, P: np.ndarray, top_k: int,
+                      top_p: float, tol: float = 1e-6) -> str:
+    """Classify a selected block set against the oracle's (Prism guide, Method
+    section 3: S_i = Top-k(P_i, k) U Top-p(P_i, p)).
+
+    Returns "exact" when the sets are equal, "tie" when they differ only in
+    the way fp32 rounding can legitimately move the cutoff, and "mismatch"
+    otherwise.  With the oracle's ranking (P descending, lower id first) and
+    n_k = min(k, n) and n_p the shortest prefix whose cumulative sum reaches
+    p, the selected size is m = max(n_k, n_p).  Two effects of fp32 are
+    allowed, and nothing else:
+
+    * the top-p crossing moves by one block when the cumulative sum that
+      decides it is within ``tol`` of p (n_p - 1 if the sum before the
+      crossing block is within tol of p, n_p + 1 if the sum including it is);
+    * at the boundary of a set of size m, blocks whose probability is within
+      ``tol`` (relative) of the m-th ranked probability may be swapped for
+      one another.
+
+    So for some allowed size m the GPU set must hold exactly m blocks, every
+    block ranked clearly above the m-th (P > P_m (1 + tol)), and no block
+    clearly below it (P < P_m (1 - tol)): the top-k blocks and every block
+    above the cutoff must match exactly.
+    """
+    g = set(np.asarray(got).tolist())
+    r = set(np.asarray(ref).tolist())
     if g == r:
-        return True
-    order = sorted(range(len(P)), key=lambda j: (-P[j], j))
-    n_sel = len(r)
-    p_cut = P[order[n_sel - 1]]
+        return "exact"
+    P = np.asarray(P, np.float64)
+    n = len(P)
+    if len(g) != len(np.asarray(got)) or any(j < 0 or j >= n for j in g):
+        return "mismatch"  # duplicates or ids out of range
+    order = sorted(range(n), key=lambda j: (-P[j], j))
     csum = np.cumsum(P[order])
-    n_k = min(top_k, len(P))
-    if n_sel > n_k:  # top-p decided the size
-        if abs(csum[n_sel - 1] - top_p) <= tol or (n_sel >= 2 and abs(csum[n_sel - 2] - top_p) <= tol):
-            return True
-    for j in g ^ r:
-        if abs(P[j] - p_cut) > tol * p_cut:
-            return False
-    return True
+    n_k = min(max(top_k, 0), n)
+    hit = np.nonzero(csum >= top_p)[0]
+    n_p = int(hit[0]) + 1 if len(hit) else n
+    sizes = {max(n_k, n_p)}
+    if n_p >= 2 and abs(csum[n_p - 2] - top_p) <= tol:
+        sizes.add(max(n_k, n_p - 1))
+    if n_p < n and abs(csum[n_p - 1] - top_p) <= tol:
+        sizes.add(max(n_k, n_p + 1))
+    for m in sizes:
+        if len(g) != m or m == 0:
+            continue
+        pm = P[order[m - 1]]
+        above = {j for j in range(n) if P[j] > pm * (1 + tol)}
+        below = {j for j in range(n) if P[j] < pm * (1 - tol)}
+        if above <= g and not (g & below):
+            return "tie"
+    return "mismatch"
+
+
+def selection_matches(got, ref, P, top_k: int, top_p: float, tol: float = 1e-6) -> bool:
+    """True unless ``selection_verdict`` says "mismatch"."""
+    return selection_verdict(got, ref, P, top_k, top_p, tol) != "mismatch"

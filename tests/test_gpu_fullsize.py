@@ -4,13 +4,16 @@ against the fp64 oracle on sampled outputs it can compute one by one (the
 text cross-attention, a call of its own, runs in the same dense step, and so
 does the mask-guided region-restricted attention on the workload with a mask).
 
-Sampled rows per (batch, head): seeded random query rows, the first and last
-rows of the sequence and of every segment (the edge tiles, conditioning
-frames, audio and text), and every audio row for the audio-query direction
+Sampled rows per (batch, head): 2,048 seeded random query rows, the first
+and last 128 rows of the sequence (the first and last query tiles), the first
+and last 16 rows of every segment (conditioning frames, video, audio, text),
+every audio and text row, and every audio row for the audio-query direction
 of the cross-attention.  Tolerances: bf16 max-abs 2e-2, relative-L2 5e-3.
-The block-sparse workload additionally checks selected block sets exactly
-(outside fp32 ties) on sampled query blocks of four heads, and the sparse
-output of every sampled block whose selection agrees with the oracle.
+The block-sparse workload checks the selected block set of every one of the
+3,060 query blocks of four heads (12,240 rows) exactly, outside fp32 ties at
+the cutoff (tests/_util.py ``selection_verdict``; the excused rows are
+counted, printed and bounded), and the sparse output of 2,048 sampled query
+rows (32 query blocks plus the edge blocks) of each of those heads.
 
 Between steps the path stores Q and K in bf16 (the RoPE step writes them in
 place), so the oracle's own RoPE output is rounded to bf16 before it feeds the
@@ -23,13 +26,16 @@ import pytest
 import oracle as O
 from joint_video_audio_rope_b200 import workloads as WL
 
-from _util import assert_close, bf16_round, oracle_layout, selection_matches
+from _util import assert_close, bf16_round, oracle_layout, selection_verdict
 
 pytestmark = pytest.mark.gpu
 
 torch = pytest.importorskip("torch")
 
-ROWS = 48  # random query rows per (batch, head)
+ROWS = 2048  # seeded random query rows per (batch, head)
+EDGE = 128   # rows at each end of the sequence (the first and last query tiles)
+SEG_EDGE = 16  # rows at each end of every segment
+MAX_EXCUSED = 0.005  # at most 0.5 % of the checked selection rows may differ at a tie
 
 
 @pytest.fixture(scope="module")
@@ -55,12 +61,23 @@ def _sample_rows(w, rng):
     start = 0
     for s in w.segments:
         e = start + s["n_tokens"]
-        rows.update(range(start, min(start + 3, e)))
-        rows.update(range(max(start, e - 3), e))
+        if s["kind"] != WL.SEG_VIDEO:
+            rows.update(range(start, e))  # every audio and text row
+        rows.update(range(start, min(start + SEG_EDGE, e)))
+        rows.update(range(max(start, e - SEG_EDGE), e))
         start = e
-    rows.update(range(0, 2))
-    rows.update(range(n - 2, n))
+    rows.update(range(0, min(EDGE, n)))
+    rows.update(range(max(0, n - EDGE), n))
     return np.array(sorted(rows))
+
+
+def _attn_rows(q, k, v, scale, chunk=512):
+    """The oracle's attention for the rows of q, a chunk of rows at a time
+    (rows are independent; this only bounds the score matrix in memory)."""
+    out = np.zeros((q.shape[0], v.shape[1]))
+    for i in range(0, q.shape[0], chunk):
+        out[i:i + chunk], _ = O.attn(q[i:i + chunk], k, v, scale)
+    return out
 
 
 def _run_dense_step(M, w, x):
@@ -123,7 +140,7 @@ def test_dense_workload_full_size(M, name):
         got_v = _f64(oc[b, rows])
         ref_o = np.zeros_like(got_o)
         for h in range(w.heads):
-            ref_o[:, h], _ = O.attn(qr[:, h], kk[:, h], vv[:, h], scale)
+            ref_o[:, h] = _attn_rows(qr[:, h], kk[:, h], vv[:, h], scale)
         assert_close(got_o, ref_o, "bf16", f"{name} joint b{b}")
         if om is not None:
             # masked rows are joint-attention rows; the others keep the fill
@@ -137,12 +154,12 @@ def test_dense_workload_full_size(M, name):
         sel = np.isin(rows, vr)
         ref_v = np.zeros((len(vr), w.heads, 128))
         for h in range(w.heads):
-            ref_v[:, h], _ = O.attn(qr[sel, h], kk[a0:a1, h], vv[a0:a1, h], scale)
+            ref_v[:, h] = _attn_rows(qr[sel, h], kk[a0:a1, h], vv[a0:a1, h], scale)
         assert_close(got_v[sel], ref_v, "bf16", f"{name} cross v<-a b{b}")
         # text cross: the same sampled video rows over the text keys
         ref_t = np.zeros((len(vr), w.heads, 128))
         for h in range(w.heads):
-            ref_t[:, h], _ = O.attn(qr[sel, h], kk[t0:t1, h], vv[t0:t1, h], scale)
+            ref_t[:, h] = _attn_rows(qr[sel, h], kk[t0:t1, h], vv[t0:t1, h], scale)
         assert_close(_f64(ot[b, vr]), ref_t, "bf16", f"{name} text cross b{b}")
         # cross: every audio row over the video keys
         qa = bf16_round(O.rope(WL.as_f64(x["q"][b, a0:a1], "bf16"), pos[a0:a1], w.theta))
@@ -190,8 +207,11 @@ def test_sparse_workload_full_size(M):
     idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
     got_o = o[0, v0:v1]
     p32 = float(np.float32(w.top_p))
-    blk_sample = np.unique(np.concatenate([rng.choice(nb, 24, replace=False),
-                                           [0, 1, nb - 2, nb - 1]]))  # incl. short t-slab
+    # sparse outputs: 32 random query blocks (2,048 rows) plus the first two
+    # and the last two blocks (the short last t-slab)
+    blk_sample = np.unique(np.concatenate([rng.choice(nb, 32, replace=False),
+                                           [0, 1, nb - 2, nb - 1]]))
+    excused = skipped = 0
     for h in heads:
         qh = O.rope(WL.as_f64(x["q"][0, v0:v1, h:h + 1], "bf16"), pos[v0:v1], w.theta)
         kh = O.rope(WL.as_f64(x["k"][0, v0:v1, h:h + 1], "bf16"), pos[v0:v1], w.theta)
@@ -199,28 +219,41 @@ def test_sparse_workload_full_size(M):
         assert_close(_f64(q[0, v0:v1, h]), qh[:, 0], "bf16", f"rope h{h}")
         qh, kh = bf16_round(qh), bf16_round(kh)
         qb, kb = O.pool(qh[None], blocks), O.pool(kh[None], blocks)
-        agree = 0
-        for i in blk_sample:
-            ref_sel = O.select_row(qb[0, 0, i], kb[0, 0], w.top_k, p32, scale)
+        # the exact set of every query block of this head
+        ref_all = O.select_rows(qb[0, 0], kb[0, 0], w.top_k, p32, scale)
+        for i in range(nb):
             got_sel = idx_h[0, h, i, :cnt_h[0, h, i]]
-            P = O.block_probs(qb[0, 0, i], kb[0, 0], scale)
-            assert selection_matches(got_sel, ref_sel, P, w.top_k, p32), f"select h{h} blk{i}"
-            if not np.array_equal(got_sel, ref_sel):
+            if np.array_equal(got_sel, ref_all[i]):
                 continue
-            agree += 1
+            P = O.block_probs(qb[0, 0, i], kb[0, 0], scale)
+            verdict = selection_verdict(got_sel, ref_all[i], P, w.top_k, p32)
+            assert verdict == "tie", f"select h{h} blk{i}: {verdict}"
+            excused += 1
+        for i in blk_sample:
+            ref_sel = ref_all[i]
+            if not np.array_equal(idx_h[0, h, i, :cnt_h[0, h, i]], ref_sel):
+                skipped += 1  # a tie row: its set was validated above
+                continue
             s0, nn = blocks[i]
             ref, _ = O.sparse_attn_rows(qh[None], kh[None], vh[None], blocks, ref_sel, scale, 0,
                                         0, i)
             assert_close(_f64(got_o[s0:s0 + nn, h]), ref, "bf16", f"sparse h{h} blk{i}")
-        assert agree >= 0.9 * len(blk_sample)
-    # dense cross-attention on sampled video rows and every audio row (2 heads)
+    n_rows = len(heads) * nb
+    print(f"\n1080p selection: {n_rows} rows checked exactly, {excused} excused at an fp32 "
+          f"tie; sparse outputs: {len(heads) * len(blk_sample)} blocks, {skipped} skipped")
+    assert excused <= MAX_EXCUSED * n_rows
+    assert skipped <= max(1, MAX_EXCUSED * len(heads) * len(blk_sample))
+    # dense cross-attention on 2,048 sampled video rows and every audio row,
+    # every head
     kk = bf16_round(O.rope(WL.as_f64(x["k"][0], "bf16"), pos, w.theta))
     vv = WL.as_f64(x["v"][0], "bf16")
-    rows = np.sort(rng.choice(v1, 32, replace=False))
+    rows = np.sort(rng.choice(v1, ROWS, replace=False))
     qr = bf16_round(O.rope(WL.as_f64(x["q"][0, rows], "bf16"), pos[rows], w.theta))
     qa = bf16_round(O.rope(WL.as_f64(x["q"][0, a0:a1], "bf16"), pos[a0:a1], w.theta))
-    for h in (3, 17):
-        rv, _ = O.attn(qr[:, h], kk[a0:a1, h], vv[a0:a1, h], scale)
-        assert_close(_f64(oc[0, rows, h]), rv, "bf16", f"cross v<-a h{h}")
-        ra, _ = O.attn(qa[:, h], kk[v0:v1, h], vv[v0:v1, h], scale)
-        assert_close(_f64(oc[0, a0:a1, h]), ra, "bf16", f"cross a<-v h{h}")
+    got_v, got_a = _f64(oc[0, rows]), _f64(oc[0, a0:a1])
+    ref_v, ref_a = np.zeros_like(got_v), np.zeros_like(got_a)
+    for h in range(w.heads):
+        ref_v[:, h] = _attn_rows(qr[:, h], kk[a0:a1, h], vv[a0:a1, h], scale)
+        ref_a[:, h] = _attn_rows(qa[:, h], kk[v0:v1, h], vv[v0:v1, h], scale, chunk=64)
+    assert_close(got_v, ref_v, "bf16", "cross v<-a")
+    assert_close(got_a, ref_a, "bf16", "cross a<-v")

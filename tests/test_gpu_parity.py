@@ -10,7 +10,7 @@ import pytest
 import oracle as O
 from joint_video_audio_rope_b200 import workloads as WL
 
-from _util import (assert_close, bf16_round, errors, oracle_layout, rope_bands, selection_matches,
+from _util import (assert_close, bf16_round, errors, oracle_layout, rope_bands, selection_verdict,
                    to_device, to_host_f64)
 
 pytestmark = pytest.mark.gpu
@@ -457,17 +457,23 @@ def test_block_select(M, case):
     blocks, qb, kb = _oracle_select(host, w)
     scale = 1 / math.sqrt(128)
     p32 = float(np.float32(w.top_p))
-    bad = 0
+    bad = excused = rows = 0
     for b in range(w.batch):
         for h in range(w.heads):
+            ref_all = O.select_rows(qb[b, h], kb[b, h], w.top_k, p32, scale)
             for i in range(len(blocks)):
                 ref = O.select_row(qb[b, h, i], kb[b, h], w.top_k, p32, scale)
+                assert np.array_equal(ref, ref_all[i])  # the two oracle forms agree
                 got = idx[b, h, i, :cnt[b, h, i]]
                 assert np.all(np.diff(got) > 0), "ascending, unique"
                 P = O.block_probs(qb[b, h, i], kb[b, h], scale)
-                if not selection_matches(got, ref, P, w.top_k, p32):
-                    bad += 1
+                verdict = selection_verdict(got, ref, P, w.top_k, p32)
+                bad += verdict == "mismatch"
+                excused += verdict == "tie"
+                rows += 1
+    print(f"\n{case}: {rows} selection rows, {excused} excused at an fp32 tie")
     assert bad == 0, f"{bad} rows differ beyond fp32 ties"
+    assert excused <= max(1, 0.005 * rows), f"{excused} of {rows} rows excused"
 
 
 def _upload_lists(sel, nb, w):
@@ -548,15 +554,23 @@ def test_select_then_sparse_end_to_end(M):
     blocks, qb, kb = _oracle_select(host, w)
     got = to_host_f64(o)
     scale = 1 / math.sqrt(128)
-    checked = 0
+    checked = skipped = 0
     for h in range(w.heads):
         for i, (s, n) in enumerate(blocks):
             ref_sel = O.select_row(qb[0, h, i], kb[0, h], w.top_k, float(np.float32(w.top_p)), scale)
             gsel = idx[0, h, i, :cnt[0, h, i]]
             if not np.array_equal(gsel, ref_sel):
-                continue  # tie rows are covered by test_block_select
+                # a row whose set differs at an fp32 tie (validated by
+                # test_block_select); its output cannot be compared with the
+                # oracle's set, and is counted
+                P = O.block_probs(qb[0, h, i], kb[0, h], scale)
+                assert selection_verdict(gsel, ref_sel, P, w.top_k,
+                                         float(np.float32(w.top_p))) == "tie"
+                skipped += 1
+                continue
             ref, _ = O.sparse_attn_rows(host["q"], host["k"], host["v"], blocks, ref_sel, scale, 0,
                                         h, i)
             assert_close(got[0, s:s + n, h], ref, "bf16", f"e2e h{h} blk{i}")
             checked += 1
-    assert checked >= 0.95 * w.heads * len(blocks)
+    print(f"\nselect -> sparse: {checked} blocks compared, {skipped} skipped at an fp32 tie")
+    assert skipped <= max(1, 0.005 * w.heads * len(blocks))

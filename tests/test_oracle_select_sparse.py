@@ -70,6 +70,44 @@ def test_selection_brute_force(seed):
             assert sel == sorted(set(sel))
 
 
+@pytest.mark.parametrize("seed", range(6))
+def test_selection_rows_brute_force(seed):
+    """select_rows (array steps, every row of a head at once) against brute
+    force on tiny rows, including exactly tied scores."""
+    rng = np.random.default_rng(100 + seed)
+    n = int(rng.integers(2, 8))
+    qbar = rng.standard_normal((5, 8))
+    kbar = rng.standard_normal((n, 8))
+    if seed % 2:
+        kbar[1] = kbar[0]  # two key blocks with identical scores in every row
+    scale = 1 / math.sqrt(8)
+    for k in (0, 1, 3, n):
+        for p in (0.1, 0.5, 0.9, 0.99, 1.0):
+            sel = O.select_rows(qbar, kbar, k, p, scale)
+            for i in range(5):
+                P = O.block_probs(qbar[i], kbar, scale)
+                assert sel[i].tolist() in _brute_force(P, k, p)
+                if seed % 2:  # ties resolve to the lower id
+                    assert not (1 in sel[i] and 0 not in sel[i])
+
+
+def test_select_from_probs_golden_and_brute_force():
+    for line in open(os.path.join(GOLDEN, "hybrid_selection.txt")):
+        if not line.strip() or line.startswith("#"):
+            continue
+        probs, k, p, expect = [f.strip() for f in line.split("|")]
+        P = np.array([float(x) for x in probs.split()])
+        assert O.select_from_probs(P, int(k), float(p)).tolist() == \
+            [int(x) for x in expect.split()]
+    rng = np.random.default_rng(7)
+    for _ in range(20):
+        n = int(rng.integers(2, 9))
+        P = rng.dirichlet(np.ones(n))
+        for k in (0, 2):
+            for p in (0.3, 0.8):
+                assert O.select_from_probs(P, k, p).tolist() in _brute_force(P, k, p)
+
+
 def test_selection_degenerate_cases():
     rng = np.random.default_rng(1)
     qbar, kbar = rng.standard_normal(16), rng.standard_normal((37, 16))

@@ -32,10 +32,10 @@ def M():
     return mmdit
 
 
-def _inputs(seed):
+def _inputs(seed, grid=(21, 14, 16), heads=4):
     # 21x14x16 = 4704 video tokens = 37 key tiles: the audio-query direction is
-    # split in two, so the partial results really go through the scratch array
-    w = WL.Workload("noalloc", [WL.video(21, 14, 16), WL.audio(218)], batch=2, heads=4,
+    # split, so the partial results really go through the scratch array
+    w = WL.Workload("noalloc", [WL.video(*grid), WL.audio(218)], batch=2, heads=heads,
                     head_dim=128, dtype="bf16", seed=seed, qk_std=WL.INV_SQRT_128,
                     v_std=WL.INV_SQRT_128)
     x = WL.generate(w)
@@ -89,6 +89,21 @@ def test_noalloc_matches_workspace_entry_on_two_calls(M):
         ref = _run_workspace(M, w, dev)
         got = _run_noalloc(M, w, dev)
         _compare(got, ref, f"call {call + 1}")
+
+
+def test_noalloc_lowers_the_split_count_to_fit(M):
+    # batch 2 x 16 heads x 256 padded audio rows over 12,500 video tokens: the
+    # workspace call splits the video keys five ways (one wave of 160 items),
+    # whose partial results (~21 MB) exceed the fixed 16 MiB array, so the
+    # allocation-free call has to fall back to fewer, longer splits (three)
+    w, dev = _inputs(33, grid=(25, 20, 25), heads=16)
+    v0, v1 = w.video_range()
+    a0, a1 = w.audio_range()
+    dv, da = M.desc_of(dev["q"][:, v0:v1]), M.desc_of(dev["q"][:, a0:a1])
+    assert M.av_cross_attn_workspace_size(dv, da) > M.NOALLOC_SCRATCH_BYTES
+    ref = _run_workspace(M, w, dev)
+    got = _run_noalloc(M, w, dev)
+    _compare(got, ref, "reduced split")
 
 
 def test_noalloc_rejects_problems_beyond_the_scratch(M):
