@@ -102,7 +102,7 @@ def dense_step_flops(w: WL.Workload) -> dict:
 LATENT_CHANNELS = 16
 
 # Workloads timed after the headline one, each reported under "per_config".
-PER_CONFIG = ("480p", "720p", "720p_cond_b2", "1080p_sparse")
+PER_CONFIG = ("480p", "720p", "720p_cond_b2", "1080p_sparse", "1080p_adaptive")
 
 # DRAM bytes per launch of the dominant kernel from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only while the kernel
@@ -332,8 +332,31 @@ class Layer:
         self.dv, self.da = M.desc_of(q[:, v0:v1]), M.desc_of(q[:, a0:a1])
         ws_cross = M.av_cross_attn_workspace_size(self.dv, self.da)
         self.sparse = w.sparse
+        self.adaptive = w.adaptive
         ws_sel = ws_sp = 0
-        if self.sparse:
+        if self.adaptive:
+            # Prism content-adaptive blocks: plan from V and the previous
+            # step's A->V output norms, Q/K/V moved to the adaptive order,
+            # selection and sparse attention over the plan's block table, O
+            # moved back to raster order
+            seg = next(s for s in w.segments if s["kind"] == WL.SEG_VIDEO)
+            self.grid = (seg["T"], seg["H"], seg["W"])
+            T, H, W = self.grid
+            self.nz, self.nb = M.adaptive_num_zones(T, H, W), M.adaptive_max_blocks(T, H, W)
+            self.zones = torch.empty((w.batch, self.nz, 4), dtype=torch.int32, device=dev)
+            self.blocks = torch.empty((w.batch, self.nb, 2), dtype=torch.int32, device=dev)
+            self.nblk = torch.empty((w.batch,), dtype=torch.int32, device=dev)
+            self.norms = torch.zeros((w.batch, v1 - v0), dtype=torch.float32, device=dev)
+            # permuted copies with the strides of the video slice of q
+            self.perm = [torch.empty_like(q)[:, v0:v1] for _ in range(4)]
+            self.idx = torch.empty((w.batch, w.heads, self.nb, self.nb), dtype=torch.int32,
+                                   device=dev)
+            self.cnt = torch.empty((w.batch, w.heads, self.nb), dtype=torch.int32, device=dev)
+            ws_cross = M.av_cross_attn_norms_workspace_size(self.dv, self.da)
+            ws_sel = max(M.adaptive_plan_workspace_size(self.dv, T, H, W),
+                         M.block_select_table_workspace_size(self.dv, self.nb))
+            ws_sp = M.sparse_attn_table_workspace_size(self.dv, self.nb)
+        elif self.sparse:
             self.vlay = M.make_layout([s for s in w.segments if s["kind"] == WL.SEG_VIDEO])
             self.nb = M.num_blocks(self.vlay)
             self.idx = torch.empty((w.batch, w.heads, self.nb, self.nb), dtype=torch.int32,
@@ -342,9 +365,15 @@ class Layer:
             ws_sel = M.block_select_workspace_size(self.dv, self.vlay)
             ws_sp = M.sparse_attn_workspace_size(self.dv, self.vlay, self.nb)
         self.ws = torch.empty(max(ws_cross, ws_sel, ws_sp, 256), dtype=torch.uint8, device=dev)
-        # launches of this library's kernels per step: RoPE 1; joint 1 or
-        # pooling + selection 2 and groups + union + sparse attention 3; cross 3
-        self.launches = 1 + (5 if self.sparse else 1) + 3
+        # launches of this library's kernels per step: RoPE 1; joint 1, or
+        # table + pooling + scores + selection 4 and table + groups + union +
+        # schedule + sparse attention 5, or (adaptive) plan 2 + permute 1 +
+        # pooling + scores + selection 3 + groups + union + schedule + sparse
+        # attention 4 + permute back 1; cross 3 (+1 for the output norms)
+        if self.adaptive:
+            self.launches = 1 + 2 + 1 + 3 + 4 + 1 + 4
+        else:
+            self.launches = 1 + (9 if self.sparse else 1) + 3
 
     def step(self, stream, ev=None):
         M, w = self.M, self.w
@@ -355,6 +384,33 @@ class Layer:
         M.rope_apply(q, k, self.desc, self.lay, self.rope, stream)
         if ev is not None:
             ev[1].record(stream)
+        if self.adaptive:
+            T, H, W = self.grid
+            pq, pk, pv, po = self.perm
+            n = self.ws.numel()
+            M.adaptive_plan(v[:, v0:v1], self.norms, self.dv, T, H, W, self.zones, self.blocks,
+                            self.nblk, self.nb, self.ws, n, stream=stream)
+            M.adaptive_permute([q[:, v0:v1], k[:, v0:v1], v[:, v0:v1]], [pq, pk, pv], self.dv, T, H,
+                               W, self.zones, stream=stream)
+            M.block_select_table(pq, pk, self.dv, self.blocks, self.nblk, self.nb, w.top_k,
+                                 w.top_p, self.scale, self.nb, self.idx, self.cnt, self.ws, n,
+                                 stream)
+            if ev is not None:
+                ev[2].record(stream)
+            M.sparse_attn_table(pq, pk, pv, po, self.dv, self.blocks, self.nblk, self.nb,
+                                self.idx, self.cnt, self.nb, self.scale, self.ws, n, stream)
+            M.adaptive_permute([po], [o[:, v0:v1]], self.dv, T, H, W, self.zones, inverse=True,
+                               stream=stream)
+            if ev is not None:
+                ev[3].record(stream)
+            # this step's A->V output norms guide the next step's plan (the
+            # one-layer lag of the guidance)
+            M.av_cross_attn_norms(q[:, v0:v1], k[:, v0:v1], v[:, v0:v1], q[:, a0:a1], k[:, a0:a1],
+                                  v[:, a0:a1], oc[:, v0:v1], oc[:, a0:a1], self.dv, self.da,
+                                  self.scale, self.norms, self.ws, n, stream)
+            if ev is not None:
+                ev[4].record(stream)
+            return
         if self.sparse:
             M.block_select(q[:, v0:v1], k[:, v0:v1], self.dv, self.vlay, w.top_k, w.top_p,
                            self.scale, self.nb, self.idx, self.cnt, self.ws, self.ws.numel(),
@@ -377,17 +433,21 @@ class Layer:
             ev[4].record(stream)
 
 
-def selected_pair_flops(w, idx_h, cnt_h):
+def selected_pair_flops(w, idx_h, cnt_h, blen=None):
     """Algorithmic flops of block-sparse attention: 4 d per selected
-    (query token, key token) pair, summed over every (batch, head, block)."""
+    (query token, key token) pair, summed over every (batch, head, block).
+    blen [B, nblocks]: block lengths (default: the 4x4x4 blocks of the grid)."""
     seg = w.segments[0]
-    nb = idx_h.shape[2]
-    blen = np.array([_block_len(seg["T"], seg["H"], seg["W"], b) for b in range(nb)], np.int64)
+    if blen is None:
+        nb = idx_h.shape[2]
+        one = np.array([_block_len(seg["T"], seg["H"], seg["W"], b) for b in range(nb)], np.int64)
+        blen = np.tile(one, (w.batch, 1))
     pairs = 0
     for b in range(w.batch):
+        lb = np.asarray(blen[b], np.int64)
         for h in range(w.heads):
-            for i in range(nb):
-                pairs += blen[i] * blen[idx_h[b, h, i, :cnt_h[b, h, i]]].sum()
+            for i in range(len(lb)):
+                pairs += lb[i] * lb[idx_h[b, h, i, :cnt_h[b, h, i]]].sum()
     return 4.0 * pairs * w.head_dim
 
 
@@ -472,8 +532,22 @@ def measure_workload(M, w, args, dev, stream, world, peaks, sampler=None):
     res = {}
     if L.sparse:
         idx_h, cnt_h = L.idx.cpu().numpy(), L.cnt.cpu().numpy()
-        flops = {"joint": selected_pair_flops(w, idx_h, cnt_h), "cross": flops["cross"]}
-        res["block_density"] = round(float(cnt_h.mean() / L.nb), 4)
+        blen = None
+        if L.adaptive:
+            nblk = L.nblk.cpu().numpy()
+            tab = L.blocks.cpu().numpy()
+            blen = [tab[b, :nblk[b], 1] for b in range(w.batch)]
+            cnt_h = cnt_h[:, :, :int(nblk.max())]
+            zs = L.zones.cpu().numpy()[..., 0].ravel()
+            res["adaptive"] = {"zones": int(L.nz), "blocks": int(nblk.sum()),
+                               "volumes": {"64": int((zs < 7).sum()),
+                                           "128": int(((zs >= 7) & (zs < 13)).sum()),
+                                           "256": int((zs >= 13).sum())}}
+            res["block_density"] = round(float(np.mean([cnt_h[b].mean() / nblk[b]
+                                                        for b in range(w.batch)])), 4)
+        else:
+            res["block_density"] = round(float(cnt_h.mean() / L.nb), 4)
+        flops = {"joint": selected_pair_flops(w, idx_h, cnt_h, blen), "cross": flops["cross"]}
         del idx_h
     step_flops = flops["joint"] + flops["cross"]
     dom = "sparse" if L.sparse else "joint"
@@ -490,7 +564,8 @@ def measure_workload(M, w, args, dev, stream, world, peaks, sampler=None):
                      "peak": peak, "frac": round(achieved / peak, 4),
                      "peak_source": f"{peak_key} (timed region {region_ms / 1e3:.2f} s)"},
         "cross_frac": round(flops["cross"] / (part_ms["cross"] / 1e3) / 1e12 / peak, 4),
-        "step": "rope+select+sparse+cross" if L.sparse else "rope+joint+cross",
+        "step": ("rope+plan+permute+select+sparse+unpermute+cross_norms" if L.adaptive else
+                 "rope+select+sparse+cross" if L.sparse else "rope+joint+cross"),
         "launches_per_step": L.launches,
     })
     return res, L, x, window, step_flops

@@ -57,7 +57,9 @@ typedef enum {
   MMDIT_EUNSUPPORTED = 2, /* dtype / head_dim / architecture not supported     */
   MMDIT_EWORKSPACE = 3,   /* workspace missing or smaller than the size query  */
   MMDIT_ECUDA = 4,        /* a CUDA runtime/driver call failed                 */
-  MMDIT_ETIMEOUT = 5      /* a bounded device-side wait ran out                */
+  MMDIT_ETIMEOUT = 5,     /* a bounded device-side wait ran out                */
+  MMDIT_EDEVCHECK = 6     /* a device-side index check failed (builds with the
+                             device checks only; the access was skipped)        */
 } mmdit_status;
 
 enum { MMDIT_BF16 = 0, MMDIT_F32 = 1 };
@@ -339,6 +341,139 @@ MMDIT_API int mmdit_sparse_attn(const void* q, const void* k, const void* v, voi
                       mmdit_stream_t stream);
 MMDIT_API size_t mmdit_sparse_attn_workspace_size(const mmdit_tensor_desc* desc,
                                         const mmdit_layout* layout, int cap);
+
+/*
+ * mmdit_av_cross_attn_norms -- mmdit_av_cross_attn plus the output norm of
+ *   every video token of the video-query (audio -> video) direction:
+ *     video_norm[b, n] = || o_video[b, n, :, :] ||_2  over all heads and channels
+ *   (the norms a_{t,h,w} the Prism guide's Method section 1 caches from one
+ *   layer to guide the content-adaptive block shapes of the next; computed
+ *   from the fp32 output rows before their bf16 rounding, summed over heads in
+ *   a fixed order).  Other arguments as mmdit_av_cross_attn (bf16 only);
+ *   video_norm : device float [B, N_video].
+ *   workspace  : mmdit_av_cross_attn_norms_workspace_size bytes, 256-byte
+ *                aligned (the cross-attention partials + per-head norms).
+ *   Errors : EINVAL, EUNSUPPORTED, EWORKSPACE, ECUDA.
+ */
+MMDIT_API int mmdit_av_cross_attn_norms(const void* qv, const void* kv, const void* vv,
+                                        const void* qa, const void* ka, const void* va,
+                                        void* o_video, void* o_audio,
+                                        const mmdit_tensor_desc* video,
+                                        const mmdit_tensor_desc* audio, float scale,
+                                        float* video_norm, void* workspace, size_t ws_bytes,
+                                        mmdit_stream_t stream);
+MMDIT_API size_t mmdit_av_cross_attn_norms_workspace_size(const mmdit_tensor_desc* video,
+                                                          const mmdit_tensor_desc* audio);
+
+/*
+ * Content-adaptive block shapes (Prism guide, Key ideas and Method sections
+ * 1-2).  A raster-order video (T x H x W tokens per batch item) is cut into
+ * 8 x 8 x 8 macro-zones (short at the far edges).  Per zone m, from the value
+ * features V (all heads and channels, D = heads x 128):
+ *   sigma^2_{v,d}(m) = (1/D) sum_c (1/Z_d) sum_i (Vbar^(d)_{m,i,c} - mu^(d)_{m,c})^2
+ * (Vbar^(d)_{m,i}: mean of V over the zone's tokens with index i along axis
+ * d; mu^(d): the mean of those), r_{v,d} = sigma^2_{v,d} / sum_d' sigma^2_{v,d'};
+ * from the A->V cross-attention output norms a of the preceding layer,
+ * abar(m) = the zone mean of a / the largest zone mean, and vhat_{a,d}(m) =
+ * the directional variance of a normalised like r;
+ *   g_d(m) = r_{v,d}(m) + abar(m) vhat_{a,d}(m) + eps.
+ * The density rho(m) = sum_d sigma^2_{v,d}(m) / its largest value over the
+ * zones picks the block volume B(m) = 64 (rho >= tau_128), 128 (rho >=
+ * tau_256) or 256; the block shape is the candidate of that volume nearest in
+ * log2 space to l*_d = -1/2 log2 g_d + 1/3 (log2 B + 1/2 sum_d' log2 g_d').
+ * Candidates: edges 2, 4 or 8 with product B, 16 shapes, numbered
+ *   0..6   (B = 64):  (2,4,8) (2,8,4) (4,2,8) (4,4,4) (4,8,2) (8,2,4) (8,4,2)
+ *   7..12  (B = 128): (2,8,8) (4,4,8) (4,8,4) (8,2,8) (8,4,4) (8,8,2)
+ *   13..15 (B = 256): (4,8,8) (8,4,8) (8,8,4)
+ * as (b_T, b_H, b_W); distance ties go to the lower number.  A zone is cut
+ * into blocks of its shape (clipped at the zone edge).  Adaptive storage
+ * order: zones in raster order, each zone's blocks in raster order, each
+ * block's tokens in (t, h, w) raster order -- every block is one contiguous
+ * run of tokens, so the block-table calls below attend over it directly.
+ * The choices the guide leaves open (the 16 shapes, rho, the normalisations
+ * of abar and vhat, eps, short zones) are the readings stated above.
+ */
+typedef struct {
+  float tau_128;  /* rho threshold of B = 64 vs 128 (0.5) */
+  float tau_256;  /* rho threshold of B = 128 vs 256 (0.25) */
+  float eps;      /* epsilon of g_d (1e-6) */
+} mmdit_adaptive_params;
+
+/* Macro-zones of a T x H x W video, and the block-table capacity a plan of it
+ * may need (8 per zone: the finest volume, 64 tokens, in a full zone). */
+MMDIT_API int mmdit_adaptive_num_zones(int T, int H, int W);
+MMDIT_API int mmdit_adaptive_max_blocks(int T, int H, int W);
+
+/*
+ * mmdit_adaptive_plan -- the content-adaptive partition of every batch item.
+ *   v          : device bf16 [B, N, heads, 128], N = T*H*W, raster order (the
+ *                value features of the layer)
+ *   a_norm     : NULL (no audio guidance: abar = 0), or device float [B, N]:
+ *                the A->V output norms of the preceding layer (as written by
+ *                mmdit_av_cross_attn_norms), raster order
+ *   params     : NULL for (0.5, 0.25, 1e-6), else 0 <= tau_256 <= tau_128 <= 1
+ *                and eps > 0
+ *   zones      : device int32 [B, n_zones, 4], 16-byte aligned: per zone
+ *                {shape number 0..15, first storage position, first block,
+ *                blocks}
+ *   blocks     : device int32 [B, max_blocks, 2]: {start, length} of every
+ *                block in the adaptive storage order; n_blocks: device int32
+ *                [B] (entries past n_blocks[b] are not written)
+ *   max_blocks : >= mmdit_adaptive_max_blocks(T, H, W), <= 6000
+ *   workspace  : mmdit_adaptive_plan_workspace_size bytes, 256-byte aligned
+ *   The statistics are fp32 sums of the bf16 values; the plan arithmetic is
+ *   fp64.  Errors : EINVAL, EUNSUPPORTED, EWORKSPACE, ECUDA.
+ */
+MMDIT_API int mmdit_adaptive_plan(const void* v, const float* a_norm,
+                                  const mmdit_tensor_desc* desc, int T, int H, int W,
+                                  const mmdit_adaptive_params* params, int32_t* zones,
+                                  int32_t* blocks, int32_t* n_blocks, int max_blocks,
+                                  void* workspace, size_t ws_bytes, mmdit_stream_t stream);
+MMDIT_API size_t mmdit_adaptive_plan_workspace_size(const mmdit_tensor_desc* desc, int T, int H,
+                                                    int W);
+
+/*
+ * mmdit_adaptive_permute -- moves token rows between raster order and the
+ *   adaptive storage order of a plan: inverse = 0 writes dst[s(t,h,w)] =
+ *   src[(t H + h) W + w], inverse = 1 the reverse.  Up to three tensors (e.g.
+ *   Q, K, V) in one call; src[i] and dst[i] are device [B, N, heads, 128] bf16
+ *   described by `desc` (N = T*H*W), dst[i] may not alias src[i].  zones is a
+ *   plan's zone table.  Errors : EINVAL, EUNSUPPORTED, ECUDA.
+ */
+MMDIT_API int mmdit_adaptive_permute(const void* const* src, void* const* dst, int n_tensors,
+                                     const mmdit_tensor_desc* desc, int T, int H, int W,
+                                     const int32_t* zones, int inverse, mmdit_stream_t stream);
+
+/*
+ * mmdit_block_select_table / mmdit_sparse_attn_table -- mmdit_block_select and
+ *   mmdit_sparse_attn over the blocks of a block table (Prism guide, Method
+ *   section 3) instead of the 4x4x4 blocks of a grid: per batch item b the
+ *   blocks are blocks[b, i] = {start, length}, i < n_blocks[b] (device int32,
+ *   as written by mmdit_adaptive_plan), consecutive runs of 1..256 tokens of
+ *   q, k, v, o, which hold the video in that block storage order.  Block ids
+ *   index the table; block_idx is [B, heads, max_blocks, cap], block_cnt
+ *   [B, heads, max_blocks], cap >= max_blocks.  Selection and attention are
+ *   those of the 4x4x4 calls (pooled means over each block's tokens, P_i,
+ *   S_i = TopK U TopP, attention of every token of query block i over the
+ *   tokens of S_i).  A table entry outside [0, N) or longer than 256 tokens
+ *   is treated as an empty block.
+ *   Errors : EINVAL, EUNSUPPORTED, EWORKSPACE, ECUDA.
+ */
+MMDIT_API int mmdit_block_select_table(const void* q, const void* k, const mmdit_tensor_desc* desc,
+                                       const int32_t* blocks, const int32_t* n_blocks,
+                                       int max_blocks, int top_k, float top_p, float scale,
+                                       int cap, int32_t* block_idx, int32_t* block_cnt,
+                                       void* workspace, size_t ws_bytes, mmdit_stream_t stream);
+MMDIT_API size_t mmdit_block_select_table_workspace_size(const mmdit_tensor_desc* desc,
+                                                         int max_blocks);
+MMDIT_API int mmdit_sparse_attn_table(const void* q, const void* k, const void* v, void* o,
+                                      const mmdit_tensor_desc* desc, const int32_t* blocks,
+                                      const int32_t* n_blocks, int max_blocks,
+                                      const int32_t* block_idx, const int32_t* block_cnt, int cap,
+                                      float scale, void* workspace, size_t ws_bytes,
+                                      mmdit_stream_t stream);
+MMDIT_API size_t mmdit_sparse_attn_table_workspace_size(const mmdit_tensor_desc* desc,
+                                                        int max_blocks);
 
 /* Number of 4x4x4 blocks of the single BLOCK444 video segment of `layout`
  * (0 if the layout is not a single such segment). */

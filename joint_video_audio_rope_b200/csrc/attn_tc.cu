@@ -110,6 +110,7 @@ struct Work {
   int kv_lo, kv_hi;  // dense: key range
   int nkv;      // number of 128-row key tiles
   long long ubase;   // sparse: offset of the merged list
+  int ucount;        // sparse: entries of the merged list (two per key tile)
   int g_first, g_nblk;
 };
 
@@ -134,16 +135,32 @@ __device__ __forceinline__ ItemPos item_pos(const AttnProblem& pr, int item) {
 // The work items of this CTA: blockIdx.x and, in persistent launches, every
 // gridDim.x-th item after it.  The stride's digits are found once, so a step
 // is digit-wise addition with carry instead of four divisions; the walk ends
-// when the batch digit reaches B (item >= n_qtiles * n_splits * H * B).
-template <bool PERSIST>
+// when the batch digit reaches B (item >= n_qtiles * n_splits * H * B).  With
+// an item order (sparse mode) the CTA walks positions blockIdx.x,
+// blockIdx.x + gridDim.x, ... of that list instead, up to its length.
+template <bool PERSIST, bool ORDER>
 struct ItemWalk {
   ItemPos cur, stride;
+  int pos, n_ord;  // ordered walk: position in pr.order and the list length
   __device__ __forceinline__ explicit ItemWalk(const AttnProblem& pr)
-      : cur(item_pos(pr, (int)blockIdx.x)), stride(item_pos(pr, PERSIST ? (int)gridDim.x : 0)) {}
+      : cur(item_pos(pr, (int)blockIdx.x)), stride(item_pos(pr, PERSIST ? (int)gridDim.x : 0)),
+        pos((int)blockIdx.x), n_ord(0) {
+    if (ORDER) {
+      n_ord = *pr.n_order;
+      if (pos < n_ord) cur = item_pos(pr, pr.order[pos]);
+      else cur.b = pr.B;
+    }
+  }
   __device__ __forceinline__ bool more(const AttnProblem& pr) const { return cur.b < pr.B; }
   __device__ __forceinline__ void next(const AttnProblem& pr) {
     if (!PERSIST) {
       cur.b = pr.B;
+      return;
+    }
+    if (ORDER) {
+      pos += (int)gridDim.x;
+      if (pos < n_ord) cur = item_pos(pr, pr.order[pos]);
+      else cur.b = pr.B;
       return;
     }
     const int q = cur.qtile + stride.qtile;
@@ -159,6 +176,9 @@ struct ItemWalk {
   }
 };
 
+// SPARSE: the block-sparse mode (query groups, merged key lists); the mode is
+// a template parameter so that the dense launches carry none of its code.
+template <bool SPARSE>
 __device__ __forceinline__ Work decode_work(const AttnParams& P, const ItemPos& pos, int rows) {
   Work w;
   const AttnProblem& pr = P.prob;
@@ -166,7 +186,7 @@ __device__ __forceinline__ Work decode_work(const AttnParams& P, const ItemPos& 
   w.split = pos.split;
   w.h = pos.h;
   w.b = pos.b;
-  if (pr.mode == kModeDense) {
+  if (!SPARSE) {
     const int nq = pr.q_count != nullptr ? min(pr.Nq, pr.q_count[w.b]) : pr.Nq;
     w.q0 = w.qtile * rows;
     w.q_valid = min(rows, nq - w.q0);
@@ -175,9 +195,12 @@ __device__ __forceinline__ Work decode_work(const AttnParams& P, const ItemPos& 
     // an item past the valid rows of its batch item computes nothing
     w.nkv = (w.kv_hi > w.kv_lo && w.q_valid > 0) ? (w.kv_hi - w.kv_lo + 127) / 128 : 0;
     w.ubase = 0;
+    w.ucount = 0;
     w.g_first = w.g_nblk = 0;
   } else {
-    const int4 g = pr.groups[w.qtile];
+    // a group index past the batch item's group count is an empty item
+    const bool real = w.qtile < pr.n_groups[w.b];
+    const int4 g = real ? pr.groups[(long long)w.b * pr.n_qtiles + w.qtile] : make_int4(0, 0, 0, 0);
     w.g_first = g.x;
     w.g_nblk = g.y;
     w.q0 = g.z;
@@ -186,17 +209,18 @@ __device__ __forceinline__ Work decode_work(const AttnParams& P, const ItemPos& 
     w.kv_hi = pr.Nkv;
     const long long lid = ((long long)w.b * pr.H + w.h) * pr.n_qtiles + w.qtile;
     w.ubase = lid * pr.ucap;
-    const int cnt = pr.ucnt[lid];
-    w.nkv = (cnt + 1) / 2;
+    w.ucount = real ? min(max(pr.ucnt[lid], 0), pr.ucap) : 0;
+    w.nkv = (w.ucount + 1) / 2;
   }
   return w;
 }
 
 // Token start of the two 64-row halves of key tile j, and (sparse) the
 // merged-list entries they come from.
+template <bool SPARSE>
 __device__ __forceinline__ void kv_tile(const AttnProblem& pr, const Work& w, int j, int ucount,
                                         int& s0, int& s1) {
-  if (pr.mode == kModeDense) {
+  if (!SPARSE) {
     s0 = w.kv_lo + j * 128;
     s1 = s0 + 64;
   } else {
@@ -271,7 +295,9 @@ __device__ void rope_row_smem(uint8_t* q_tile, int r, int tok, const DevLayout& 
 // once, so no cross-item state is live).  PERSIST = true: each CTA walks items
 // blockIdx.x, blockIdx.x + gridDim.x, ... keeping TMEM and barriers alive, and
 // the next item's Q load and QK overlap the current item's epilogue.
-template <int QT, int ST, bool PERSIST>
+// ORDER: block-sparse mode, persistent CTAs walking the work items in the
+// order of pr.order (longest merged list first).
+template <int QT, int ST, bool PERSIST, bool ORDER>
 __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks)
     attn_tc_kernel(const __grid_constant__ AttnParams P) {
   using C = Cfg<QT, ST>;
@@ -330,14 +356,14 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
       bool ok = true;
       int ld = 0;  // ring loads issued so far (all items)
       int it = 0;  // items of this CTA so far
-      for (ItemWalk<PERSIST> wk(P.prob); wk.more(P.prob) && ok; wk.next(P.prob), ++it) {
-        const Work w = decode_work(P, wk.cur, C::kRows);
+      for (ItemWalk<PERSIST, ORDER> wk(P.prob); wk.more(P.prob) && ok; wk.next(P.prob), ++it) {
+        const Work w = decode_work<ORDER>(P, wk.cur, C::kRows);
         const AttnProblem& pr = P.prob;
         if (it == 0) {
           tma_prefetch_desc(&pr.tmQ);
           tma_prefetch_desc(&pr.tmK);
           tma_prefetch_desc(&pr.tmV);
-          if (pr.mode == kModeDense && pr.o != nullptr && pr.part_o == nullptr)
+          if (!ORDER && pr.o != nullptr && pr.part_o == nullptr)
             tma_prefetch_desc(&pr.tmO);
         }
         for (int t = 0; t < QT && ok; ++t) {
@@ -347,12 +373,10 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
           tma_tile(sbase + kQOff + t * kTileBytes, &pr.tmQ, bar(B_QFULL + t), w.h, w.b, s0,
                    s0 + 64);
         }
-        const int ucount = pr.mode == kModeSparse
-                               ? pr.ucnt[((long long)w.b * pr.H + w.h) * pr.n_qtiles + w.qtile]
-                               : 0;
+        const int ucount = w.ucount;
         for (int j = 0; j < w.nkv && ok; ++j) {
           int s0, s1;
-          kv_tile(pr, w, j, ucount, s0, s1);
+          kv_tile<ORDER>(pr, w, j, ucount, s0, s1);
           for (int kind = 0; kind < 2; ++kind, ++ld) {
             const int slot = ld % kStages;
             if (!(ok = mbar_wait(bar(B_KVEMPTY + slot), ((ld / kStages) & 1) ^ 1, err))) break;
@@ -385,8 +409,8 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
       int cs = 0;   // ring loads consumed so far (all items)
       int pt = 0;   // key tiles processed so far (P barrier phases)
       int it = 0;
-      for (ItemWalk<PERSIST> wk(P.prob); wk.more(P.prob) && ok; wk.next(P.prob), ++it) {
-        const Work w = decode_work(P, wk.cur, C::kRows);
+      for (ItemWalk<PERSIST, ORDER> wk(P.prob); wk.more(P.prob) && ok; wk.next(P.prob), ++it) {
+        const Work w = decode_work<ORDER>(P, wk.cur, C::kRows);
         const AttnProblem& pr = P.prob;
         const int nkv = w.nkv;
         const int qbar = pr.rope_q ? B_QREADY : B_QFULL;
@@ -465,8 +489,8 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
     bool ok = !skip;
     int st = 0;  // S tiles consumed so far (all items)
     int it = 0;
-    for (ItemWalk<PERSIST> wk(P.prob); wk.more(P.prob) && ok; wk.next(P.prob), ++it) {
-      const Work w = decode_work(P, wk.cur, C::kRows);
+    for (ItemWalk<PERSIST, ORDER> wk(P.prob); wk.more(P.prob) && ok; wk.next(P.prob), ++it) {
+      const Work w = decode_work<ORDER>(P, wk.cur, C::kRows);
       const AttnProblem& pr = P.prob;
       const int nkv = w.nkv;
 
@@ -482,19 +506,19 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
       // sparse mode: which query block of the group this row belongs to
       int qb = 0;
       int ucount = 0;
-      if (pr.mode == kModeSparse) {
+      if (ORDER) {
         int acc = 0;
         qb = -1;  // rows past the group: member of nothing
+        const int2* tb = pr.tab + (long long)w.b * pr.tab_cap + w.g_first;
         for (int i = 0; i < w.g_nblk; ++i) {
-          int bst, blen;
-          block_extent(pr.vT, pr.vH, pr.vW, w.g_first + i, bst, blen);
+          const int blen = tb[i].y;
           if (row < acc + blen) {
             qb = i;
             break;
           }
           acc += blen;
         }
-        ucount = pr.ucnt[((long long)w.b * pr.H + w.h) * pr.n_qtiles + w.qtile];
+        ucount = w.ucount;
       }
 
       float m_used = -INFINITY, l = 0.f;
@@ -503,7 +527,7 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
         // (independent of S, so computed before waiting for it)
         int len0, len1;
         uint32_t seg0 = 0xFu, seg1 = 0xFu;  // valid 16-row segments of each half
-        if (pr.mode == kModeDense) {
+        if (!ORDER) {
           const int s0 = w.kv_lo + j * 128;
           len0 = max(0, min(64, w.kv_hi - s0));
           len1 = max(0, min(64, w.kv_hi - s0 - 64));
@@ -658,7 +682,18 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
           pr.part_ml[prow * 2 + 0] = (m_used == -INFINITY) ? -INFINITY : m_used * sl2;
           pr.part_ml[prow * 2 + 1] = l;
         }
-      } else if (pr.mode == kModeDense) {
+      } else if (!ORDER) {
+        if (pr.row_sq != nullptr && valid_row) {
+          // squared L2 norm of the normalised row (the A->V output norms
+          // that guide the content-adaptive block shapes)
+          float ss = 0.f;
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            const float x = __uint_as_float(ov(c)) * inv;
+            ss = fmaf(x, x, ss);
+          }
+          pr.row_sq[((long long)w.b * pr.Nq + qrow) * pr.H + w.h] = ss;
+        }
         // normalised bf16 O through the TMA engine: each round packs
         // kStageCols channels of the warp's 32 rows into the warp's staging
         // buffer and one lane issues a bulk tensor store of that box; the
@@ -799,7 +834,7 @@ __global__ void __launch_bounds__(256) split_combine_kernel(const float* __restr
                             lane * 4) = pk;
 }
 
-template <int QT, int ST, bool PERSIST>
+template <int QT, int ST, bool PERSIST, bool ORDER = false>
 cudaError_t launch_shape(const AttnParams& p, cudaStream_t s) {
   using C = Cfg<QT, ST>;
   int dev = 0;
@@ -807,7 +842,7 @@ cudaError_t launch_shape(const AttnParams& p, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   // the dynamic shared-memory limit is a per-device function attribute
   e = once_per_device(dev, [] {
-    return cudaFuncSetAttribute(attn_tc_kernel<QT, ST, PERSIST>,
+    return cudaFuncSetAttribute(attn_tc_kernel<QT, ST, PERSIST, ORDER>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   });
   if (e != cudaSuccess) return e;
@@ -821,7 +856,7 @@ cudaError_t launch_shape(const AttnParams& p, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     grid = std::min(items, sms * C::kMinBlocks);
   }
-  attn_tc_kernel<QT, ST, PERSIST><<<grid, C::kThreads, C::kSmemBytes, s>>>(p);
+  attn_tc_kernel<QT, ST, PERSIST, ORDER><<<grid, C::kThreads, C::kSmemBytes, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -834,6 +869,11 @@ int attn_store_cols(int q_tiles) {
 int attn_rows_per_cta(int q_tiles) { return 128 * q_tiles; }
 
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
+  if (p.prob.order != nullptr) {
+    // an item order is walked by persistent CTAs (block-sparse attention)
+    if (p.q_tiles != 2 || !p.persistent) return cudaErrorInvalidValue;
+    return launch_shape<2, 4, true, true>(p, s);
+  }
   if (p.q_tiles == 1)
     return p.persistent ? launch_shape<1, 2, true>(p, s) : launch_shape<1, 2, false>(p, s);
   return p.persistent ? launch_shape<2, 4, true>(p, s) : launch_shape<2, 4, false>(p, s);

@@ -85,6 +85,22 @@ __device__ __forceinline__ void token_position(const DevLayout& L, int n, float&
   }
 }
 
+// Device-side index checks of the debug build (MMDIT_DEVICE_CHECKS): a failed
+// check records MMDIT_EDEVCHECK in the library's device error word (the first
+// error recorded stays) and the code goes on to skip or clamp the access, as
+// every build does; nothing traps.  In the regular build the check compiles
+// to nothing.
+#ifdef MMDIT_DEVICE_CHECKS
+#define MMDIT_DCHECK(cond, err)                                         \
+  do {                                                                  \
+    if (!(cond)) atomicCAS((err), 0, (int)MMDIT_EDEVCHECK);             \
+  } while (0)
+#else
+#define MMDIT_DCHECK(cond, err) \
+  do {                          \
+  } while (0)
+#endif
+
 // Start token and length of 4x4x4 block `b` of a block-major T x H x W grid.
 __device__ __forceinline__ void block_extent(int T, int H, int W, int b, int& start,
                                              int& len) {

@@ -78,15 +78,23 @@ struct AttnProblem {
   int kv_per_split;           // tokens per split, multiple of 128
   int ctas;                   // work items: n_qtiles * H * B * n_splits
   int mode;                   // AttnMode
-  // sparse mode: the query groups and the merged key-block lists
-  const int4* groups;         // per group: {first block, n blocks, start token, n tokens}
-  const uint4* ulist;         // [B][H][n_groups][ucap]: {start, len, seg masks 0|1, seg masks 2|3}
-  const int* ucnt;            // [B][H][n_groups]
+  // sparse mode: the query groups and the merged key lists (n_qtiles = the
+  // groups' capacity per batch item), the block table, and the order of the
+  // work items (ids (b H + h) n_qtiles + g, longest list first)
+  const int4* groups;         // [B][n_qtiles]: {first block, n blocks, start token, n tokens}
+  const int* n_groups;        // [B]
+  const uint4* ulist;         // [B][H][n_qtiles][ucap]: {start, len, seg masks 0|1, seg masks 2|3}
+  const int* ucnt;            // [B][H][n_qtiles]
   int ucap;
-  int vT, vH, vW;             // block-major video grid (sparse mode)
+  const int2* tab;            // [B][tab_cap] {start, length} of every block
+  int tab_cap;
+  const int* order;           // [*n_order] item ids; nullptr: items in index order
+  const int* n_order;
   int rope_q;                 // rotate Q tiles in shared memory after loading
   const int* q_count;         // dense mode, optional: valid query rows per batch item
                               // (device; rows from q_count[b] on are not computed)
+  float* row_sq;              // dense mode, optional: [B][Nq][H] squared L2 norm of every
+                              // normalised output row (fp32, before the bf16 rounding)
 };
 
 // One attention problem per launch: every field of `prob` sits at a fixed
@@ -106,10 +114,17 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s);
 // Both directions of the audio<->video cross-attention on one stream: audio
 // queries over the video keys (split-KV partials into part_o / part_ml), video
 // queries over the audio keys, then the merge of the partials.
+// With row_sq and video_norm non-NULL, the video-query launch also writes the
+// squared norm of every (token, head) output row into row_sq [B][Nv][H] and
+// video_norm [B][Nv] receives the L2 norm of each video token's output over
+// all heads (launch_cross_norms).
 int launch_cross(const void* qv, const void* kv, const void* vv, const void* qa, const void* ka,
                  const void* va, void* o_video, void* o_audio, const mmdit_tensor_desc& video,
                  const mmdit_tensor_desc& audio, float scale, int splits, int kv_per_split,
-                 float* part_o, float* part_ml, cudaStream_t s);
+                 float* part_o, float* part_ml, cudaStream_t s, float* row_sq = nullptr,
+                 float* video_norm = nullptr);
+cudaError_t launch_cross_norms(const float* sq, int heads, long long n_rows, float* a,
+                               cudaStream_t s);
 // Split of the video keys for the audio-query direction of the cross
 // attention (mmdit_api.cu): audio query tiles of 256 rows, `splits` key ranges
 // of kv_per_split tokens (a multiple of 128), and the partial-result sizes.
@@ -130,19 +145,28 @@ cudaError_t launch_split_combine(const float* part_o, const float* part_ml, __nv
 constexpr int kSparseQTiles = 2;
 constexpr int kGroupTokens = 128 * kSparseQTiles;
 constexpr int kGroupBlocks = 8 * kSparseQTiles;
+constexpr int kMaxBlockTokens = 256;  // longest block of any block table
 
-// block selection (select.cu)
+// block selection and the sparse-attention preparation (select.cu).  Block
+// tables: per batch item `maxb` int2 {start token, length} in storage order
+// and a block count; pooled means [B][H][maxb][128]; scores [B][H][maxb][ld].
+cudaError_t launch_grid_table(int T, int H, int W, int nblk, int B, int maxb, int2* tab,
+                              int* tab_n, cudaStream_t s);
+size_t select_scores_ld(int maxb);
 cudaError_t launch_pool(const __nv_bfloat16* q, const __nv_bfloat16* k, const mmdit_tensor_desc& d,
-                        int T, int H, int W, int nblk, float* qbar, float* kbar, cudaStream_t s);
-cudaError_t launch_select(const float* qbar, const float* kbar, int B, int H, int nblk, int top_k,
-                          float top_p, float scale, int cap, int32_t* idx, int32_t* cnt,
-                          cudaStream_t s);
-size_t select_smem_bytes(int nblk);
-cudaError_t launch_groups(int T, int H, int W, int nblk, int4* groups, int* n_groups,
-                          cudaStream_t s);
-cudaError_t launch_union(const int32_t* idx, const int32_t* cnt, int cap, const int4* groups,
-                         int n_groups_max, const int* n_groups, int B, int H, int nblk, int T,
-                         int Hg, int Wg, uint4* ulist, int* ucnt, cudaStream_t s);
+                        const int2* tab, const int* tab_n, int maxb, float* qbar, float* kbar,
+                        int* err, cudaStream_t s);
+cudaError_t launch_select(const float* qbar, const float* kbar, const int* tab_n, int B, int H,
+                          int maxb, int top_k, float top_p, float scale, int cap, float* S,
+                          int32_t* idx, int32_t* cnt, int* err, cudaStream_t s);
+cudaError_t launch_groups(const int2* tab, const int* tab_n, int B, int maxb, int N, int maxg,
+                          int4* groups, int* n_groups, int* err, cudaStream_t s);
+cudaError_t launch_union(const int32_t* idx, const int32_t* cnt, int cap, const int2* tab,
+                         const int* tab_n, int maxb, int N, const int4* groups,
+                         const int* n_groups, int maxg, int B, int H, int ucap, uint4* ulist,
+                         int* ucnt, int* err, cudaStream_t s);
+cudaError_t launch_schedule(const int* ucnt, const int* n_groups, int maxg, int B, int H,
+                            int ucap, int* order, int* n_order, cudaStream_t s);
 
 // helpers (mmdit_api.cu)
 int* device_error_flag();  // device address of this device's error word

@@ -182,46 +182,6 @@ int check_sm100() {
   return MMDIT_OK;
 }
 
-// single BLOCK444 video segment -> grid and block count
-int sparse_layout(const mmdit_layout* L, const mmdit_tensor_desc* d, int& T, int& H, int& W,
-                  int& nblk) {
-  int rc = check_layout(L, d->n_tokens);
-  if (rc) return rc;
-  if (L->n_seg != 1 || L->seg[0].kind != MMDIT_SEG_VIDEO || L->seg[0].order != MMDIT_ORDER_BLOCK444)
-    return fail(MMDIT_EINVAL, "block-sparse calls need exactly one BLOCK444 video segment");
-  T = L->seg[0].T;
-  H = L->seg[0].H;
-  W = L->seg[0].W;
-  const long long nb = (long long)((T + 3) / 4) * ((H + 3) / 4) * ((W + 3) / 4);
-  if (nb > kMaxBlocks)
-    return fail(MMDIT_EUNSUPPORTED, "%lld blocks; at most %d are supported", nb, kMaxBlocks);
-  nblk = (int)nb;
-  return MMDIT_OK;
-}
-
-int host_block_len(int T, int H, int W, int b) {
-  const int nhb = (H + 3) / 4, nwb = (W + 3) / 4;
-  const int tb = b / (nhb * nwb), r = b % (nhb * nwb), hb = r / nwb, wb = r % nwb;
-  return std::min(4, T - 4 * tb) * std::min(4, H - 4 * hb) * std::min(4, W - 4 * wb);
-}
-
-// greedy grouping of query blocks (<= kGroupTokens tokens, <= kGroupBlocks
-// blocks); the device groups_kernel applies the same rule and writes the table.
-int host_group_count(int T, int H, int W, int nblk) {
-  int g = 0, nb = 0, tokens = 0;
-  for (int b = 0; b < nblk; ++b) {
-    const int len = host_block_len(T, H, W, b);
-    if (nb == kGroupBlocks || tokens + len > kGroupTokens) {
-      ++g;
-      nb = 0;
-      tokens = 0;
-    }
-    ++nb;
-    tokens += len;
-  }
-  return g + (nb > 0 ? 1 : 0);
-}
-
 // Split of the video keys for the audio-query direction: enough splits that
 // the (few) audio query tiles x heads x batch fill one wave of the B200's 148
 // SMs, each split a whole number of 128-key tiles.  One wave of long items
@@ -287,7 +247,8 @@ int short_kv_params(AttnParams& p, const void* q, const void* k, const void* v, 
 int launch_cross(const void* qv, const void* kv, const void* vv, const void* qa, const void* ka,
                  const void* va, void* o_video, void* o_audio, const mmdit_tensor_desc& video,
                  const mmdit_tensor_desc& audio, float scale, int splits, int kv_per_split,
-                 float* part_o, float* part_ml, cudaStream_t s) {
+                 float* part_o, float* part_ml, cudaStream_t s, float* row_sq,
+                 float* video_norm) {
   int rc;
   int* err = device_error_flag();
   if (err == nullptr) return fail(MMDIT_ECUDA, "device error flag unavailable");
@@ -319,12 +280,16 @@ int launch_cross(const void* qv, const void* kv, const void* vv, const void* qa,
   AttnParams pv{};
   if ((rc = short_kv_params(pv, qv, ka, va, o_video, video, audio, scale, err, "video", "audio")))
     return rc;
+  pv.prob.row_sq = video_norm != nullptr ? row_sq : nullptr;
   cudaError_t e = launch_attn_tc(pa, s);
   if (e == cudaSuccess) e = launch_attn_tc(pv, s);
   if (e == cudaSuccess)
     e = launch_split_combine(part_o, part_ml, (__nv_bfloat16*)o_audio, audio.stride_tok,
                              audio.stride_batch, splits, audio.batch, audio.heads, audio.n_tokens,
                              a2v.n_qtiles * 256, s);
+  if (e == cudaSuccess && video_norm != nullptr)
+    e = launch_cross_norms(row_sq, video.heads, (long long)video.batch * video.n_tokens,
+                           video_norm, s);
   return e == cudaSuccess ? MMDIT_OK : cuda_fail(e, "av_cross launch");
 }
 
@@ -355,14 +320,6 @@ extern "C" {
 const char* mmdit_last_error(void) { return t_last_error.c_str(); }
 
 const char* mmdit_version(void) { return "mmdit-av-attn 0.1.0 (sm_100a)"; }
-
-int mmdit_num_blocks(const mmdit_layout* L) {
-  if (L == nullptr || L->n_seg != 1 || L->seg[0].kind != MMDIT_SEG_VIDEO ||
-      L->seg[0].order != MMDIT_ORDER_BLOCK444 || L->seg[0].T < 1 || L->seg[0].H < 1 ||
-      L->seg[0].W < 1)
-    return 0;
-  return ((L->seg[0].T + 3) / 4) * ((L->seg[0].H + 3) / 4) * ((L->seg[0].W + 3) / 4);
-}
 
 int mmdit_device_status(mmdit_stream_t stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
@@ -527,6 +484,49 @@ int mmdit_av_cross_attn(const void* qv, const void* kv, const void* vv, const vo
                       reinterpret_cast<float*>(static_cast<char*>(workspace) + c.part_o_bytes), s);
 }
 
+size_t mmdit_av_cross_attn_norms_workspace_size(const mmdit_tensor_desc* video,
+                                                const mmdit_tensor_desc* audio) {
+  const size_t base = mmdit_av_cross_attn_workspace_size(video, audio);
+  if (base == 0) return 0;
+  return base + align256(sizeof(float) * (size_t)video->batch * video->n_tokens * video->heads);
+}
+
+int mmdit_av_cross_attn_norms(const void* qv, const void* kv, const void* vv, const void* qa,
+                              const void* ka, const void* va, void* o_video, void* o_audio,
+                              const mmdit_tensor_desc* video, const mmdit_tensor_desc* audio,
+                              float scale, float* video_norm, void* workspace, size_t ws_bytes,
+                              mmdit_stream_t stream) {
+  MMDIT_NVTX("mmdit_av_cross_attn_norms");
+  int rc;
+  if ((rc = check_desc(video, "video")) || (rc = check_desc(audio, "audio"))) return rc;
+  if (video->batch != audio->batch || video->heads != audio->heads ||
+      video->head_dim != audio->head_dim || video->dtype != audio->dtype)
+    return fail(MMDIT_EINVAL, "av_cross_norms: video and audio descriptors disagree");
+  if (video->dtype != MMDIT_BF16) return fail(MMDIT_EUNSUPPORTED, "av_cross_norms: bf16 only");
+  const void* ptrs[8] = {qv, kv, vv, qa, ka, va, o_video, o_audio};
+  for (const void* p : ptrs) {
+    if (p == nullptr) return fail(MMDIT_EINVAL, "av_cross_norms: every tensor must be non-NULL");
+    if (!aligned16(p)) return fail(MMDIT_EINVAL, "av_cross_norms: tensors must be 16-byte aligned");
+  }
+  if (video_norm == nullptr || (reinterpret_cast<uintptr_t>(video_norm) & 3u))
+    return fail(MMDIT_EINVAL, "av_cross_norms: video_norm must be an aligned device float array");
+  if (video->n_tokens < 1 || audio->n_tokens < 1)
+    return fail(MMDIT_EINVAL, "av_cross_norms: both streams need at least one token");
+  if (!(scale > 0.f) || !isfinite(scale)) return fail(MMDIT_EINVAL, "av_cross_norms: scale must be > 0");
+  const CrossPlan c = plan_cross(video, audio);
+  const size_t need = mmdit_av_cross_attn_norms_workspace_size(video, audio);
+  if (workspace == nullptr || ws_bytes < need)
+    return fail(MMDIT_EWORKSPACE, "av_cross_norms: workspace needs %zu bytes", need);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(MMDIT_EINVAL, "av_cross_norms: workspace must be 256-byte aligned");
+  if ((rc = check_sm100())) return rc;
+  char* ws = static_cast<char*>(workspace);
+  return launch_cross(qv, kv, vv, qa, ka, va, o_video, o_audio, *video, *audio, scale, c.splits,
+                      c.kv_per_split, reinterpret_cast<float*>(ws),
+                      reinterpret_cast<float*>(ws + c.part_o_bytes), (cudaStream_t)stream,
+                      reinterpret_cast<float*>(ws + c.part_o_bytes + c.part_ml_bytes), video_norm);
+}
+
 int mmdit_text_cross_attn(const void* qv, const void* kt, const void* vt, void* o_video,
                           const mmdit_tensor_desc* video, const mmdit_tensor_desc* text,
                           float scale, mmdit_stream_t stream) {
@@ -563,124 +563,6 @@ int mmdit_text_cross_attn(const void* qv, const void* kt, const void* vt, void* 
     return rc;
   cudaError_t e = launch_attn_tc(p, s);
   return e == cudaSuccess ? MMDIT_OK : cuda_fail(e, "text_cross launch");
-}
-
-size_t mmdit_block_select_workspace_size(const mmdit_tensor_desc* desc, const mmdit_layout* layout) {
-  int T, H, W, nblk;
-  if (check_desc(desc, "block_select") || sparse_layout(layout, desc, T, H, W, nblk)) return 0;
-  return 2 * align256((size_t)desc->batch * desc->heads * nblk * 128 * sizeof(float));
-}
-
-int mmdit_block_select(const void* q, const void* k, const mmdit_tensor_desc* desc,
-                       const mmdit_layout* layout, int top_k, float top_p, float scale, int cap,
-                       int32_t* block_idx, int32_t* block_cnt, void* workspace, size_t ws_bytes,
-                       mmdit_stream_t stream) {
-  MMDIT_NVTX("mmdit_block_select");
-  int rc = check_desc(desc, "block_select");
-  if (rc) return rc;
-  if (desc->dtype != MMDIT_BF16) return fail(MMDIT_EUNSUPPORTED, "block_select: bf16 only");
-  if (!q || !k || !block_idx || !block_cnt)
-    return fail(MMDIT_EINVAL, "block_select: q, k, block_idx, block_cnt must be non-NULL");
-  if (!aligned16(q) || !aligned16(k)) return fail(MMDIT_EINVAL, "block_select: 16-byte alignment");
-  int T, H, W, nblk;
-  if ((rc = sparse_layout(layout, desc, T, H, W, nblk))) return rc;
-  if (cap < nblk) return fail(MMDIT_EINVAL, "block_select: cap %d < number of blocks %d", cap, nblk);
-  if (top_k < 0) return fail(MMDIT_EINVAL, "block_select: top_k < 0");
-  if (!(top_p >= 0.f && top_p <= 1.f)) return fail(MMDIT_EINVAL, "block_select: top_p outside [0, 1]");
-  if (!(scale > 0.f) || !isfinite(scale)) return fail(MMDIT_EINVAL, "block_select: scale must be > 0");
-  const size_t half = align256((size_t)desc->batch * desc->heads * nblk * 128 * sizeof(float));
-  if (workspace == nullptr || ws_bytes < 2 * half)
-    return fail(MMDIT_EWORKSPACE, "block_select: workspace needs %zu bytes", 2 * half);
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    return fail(MMDIT_EINVAL, "block_select: workspace must be 256-byte aligned");
-  float* qbar = static_cast<float*>(workspace);
-  float* kbar = reinterpret_cast<float*>(static_cast<char*>(workspace) + half);
-  cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = launch_pool((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, *desc, T, H, W,
-                              nblk, qbar, kbar, s);
-  if (e == cudaSuccess)
-    e = launch_select(qbar, kbar, desc->batch, desc->heads, nblk, top_k, top_p, scale, cap,
-                      block_idx, block_cnt, s);
-  return e == cudaSuccess ? MMDIT_OK : cuda_fail(e, "block_select launch");
-}
-
-size_t mmdit_sparse_attn_workspace_size(const mmdit_tensor_desc* desc, const mmdit_layout* layout,
-                                        int) {
-  int T, H, W, nblk;
-  if (check_desc(desc, "sparse_attn") || sparse_layout(layout, desc, T, H, W, nblk)) return 0;
-  const int ng = host_group_count(T, H, W, nblk);
-  const size_t lists = (size_t)desc->batch * desc->heads * ng;
-  return align256(sizeof(int4) * ng) + align256(lists * nblk * sizeof(uint4)) +
-         align256(lists * sizeof(int));
-}
-
-int mmdit_sparse_attn(const void* q, const void* k, const void* v, void* o,
-                      const mmdit_tensor_desc* desc, const mmdit_layout* layout,
-                      const int32_t* block_idx, const int32_t* block_cnt, int cap, float scale,
-                      void* workspace, size_t ws_bytes, mmdit_stream_t stream) {
-  MMDIT_NVTX("mmdit_sparse_attn");
-  int rc = check_desc(desc, "sparse_attn");
-  if (rc) return rc;
-  if (desc->dtype != MMDIT_BF16) return fail(MMDIT_EUNSUPPORTED, "sparse_attn: bf16 only");
-  if (!q || !k || !v || !o || !block_idx || !block_cnt)
-    return fail(MMDIT_EINVAL, "sparse_attn: every pointer must be non-NULL");
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
-    return fail(MMDIT_EINVAL, "sparse_attn: 16-byte alignment");
-  if (o == q || o == k || o == v) return fail(MMDIT_EINVAL, "sparse_attn: o aliases an input");
-  int T, H, W, nblk;
-  if ((rc = sparse_layout(layout, desc, T, H, W, nblk))) return rc;
-  if (cap < nblk) return fail(MMDIT_EINVAL, "sparse_attn: cap %d < number of blocks %d", cap, nblk);
-  if (!(scale > 0.f) || !isfinite(scale)) return fail(MMDIT_EINVAL, "sparse_attn: scale must be > 0");
-  const int ng = host_group_count(T, H, W, nblk);
-  const size_t lists = (size_t)desc->batch * desc->heads * ng;
-  const size_t g_bytes = align256(sizeof(int4) * ng);
-  const size_t l_bytes = align256(lists * nblk * sizeof(uint4));
-  const size_t c_bytes = align256(lists * sizeof(int));
-  if (workspace == nullptr || ws_bytes < g_bytes + l_bytes + c_bytes)
-    return fail(MMDIT_EWORKSPACE, "sparse_attn: workspace needs %zu bytes", g_bytes + l_bytes + c_bytes);
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    return fail(MMDIT_EINVAL, "sparse_attn: workspace must be 256-byte aligned");
-  if ((rc = check_sm100())) return rc;
-  char* ws = static_cast<char*>(workspace);
-  int4* groups = reinterpret_cast<int4*>(ws);
-  uint4* ulist = reinterpret_cast<uint4*>(ws + g_bytes);
-  int* ucnt = reinterpret_cast<int*>(ws + g_bytes + l_bytes);
-  cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = launch_groups(T, H, W, nblk, groups, nullptr, s);
-  if (e == cudaSuccess)
-    e = launch_union(block_idx, block_cnt, cap, groups, ng, nullptr, desc->batch, desc->heads, nblk,
-                     T, H, W, ulist, ucnt, s);
-  if (e != cudaSuccess) return cuda_fail(e, "sparse_attn prep launch");
-  AttnParams p{};
-  AttnProblem& pr = p.prob;
-  if ((rc = make_map(&pr.tmQ, q, *desc, desc->n_tokens, "q")) ||
-      (rc = make_map(&pr.tmK, k, *desc, desc->n_tokens, "k")) ||
-      (rc = make_map(&pr.tmV, v, *desc, desc->n_tokens, "v")))
-    return rc;
-  pr.o = (__nv_bfloat16*)o;
-  pr.o_st = desc->stride_tok;
-  pr.o_sb = desc->stride_batch;
-  pr.Nq = pr.Nkv = desc->n_tokens;
-  pr.H = desc->heads;
-  pr.B = desc->batch;
-  pr.n_qtiles = ng;
-  pr.n_splits = 1;
-  pr.kv_per_split = 0;
-  pr.ctas = ng * pr.H * pr.B;
-  pr.mode = kModeSparse;
-  p.q_tiles = kSparseQTiles;
-  pr.groups = groups;
-  pr.ulist = ulist;
-  pr.ucnt = ucnt;
-  pr.ucap = nblk;
-  pr.vT = T;
-  pr.vH = H;
-  pr.vW = W;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.err = device_error_flag();
-  if (p.err == nullptr) return fail(MMDIT_ECUDA, "device error flag unavailable");
-  e = launch_attn_tc(p, s);
-  return e == cudaSuccess ? MMDIT_OK : cuda_fail(e, "sparse attn launch");
 }
 
 }  // extern "C"

@@ -24,7 +24,7 @@ if not os.path.exists(LIB_PATH):
                       "`python -m joint_video_audio_rope_b200.build`")
 _lib = C.CDLL(LIB_PATH)
 
-OK, EINVAL, EUNSUPPORTED, EWORKSPACE, ECUDA, ETIMEOUT = range(6)
+OK, EINVAL, EUNSUPPORTED, EWORKSPACE, ECUDA, ETIMEOUT, EDEVCHECK = range(7)
 BF16, F32 = 0, 1
 SEG_VIDEO, SEG_AUDIO, SEG_TEXT = 0, 1, 2
 ORDER_RASTER, ORDER_BLOCK444 = 0, 1
@@ -49,6 +49,10 @@ class TensorDesc(C.Structure):
 class RopeParams(C.Structure):
     _fields_ = [("theta", C.c_float), ("dim_t", C.c_int32), ("dim_h", C.c_int32),
                 ("dim_w", C.c_int32)]
+
+
+class AdaptiveParams(C.Structure):
+    _fields_ = [("tau_128", C.c_float), ("tau_256", C.c_float), ("eps", C.c_float)]
 
 
 _P = C.c_void_p
@@ -81,6 +85,23 @@ _SIGS = {
                                     C.c_size_t, _P]),
     "mmdit_sparse_attn_workspace_size": (C.c_size_t, [_D, _L, C.c_int]),
     "mmdit_num_blocks": (C.c_int, [_L]),
+    "mmdit_av_cross_attn_norms": (C.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _D, _D, C.c_float,
+                                            _P, _P, C.c_size_t, _P]),
+    "mmdit_av_cross_attn_norms_workspace_size": (C.c_size_t, [_D, _D]),
+    "mmdit_adaptive_num_zones": (C.c_int, [C.c_int, C.c_int, C.c_int]),
+    "mmdit_adaptive_max_blocks": (C.c_int, [C.c_int, C.c_int, C.c_int]),
+    "mmdit_adaptive_plan": (C.c_int, [_P, _P, _D, C.c_int, C.c_int, C.c_int,
+                                      C.POINTER(AdaptiveParams), _P, _P, _P, C.c_int, _P,
+                                      C.c_size_t, _P]),
+    "mmdit_adaptive_plan_workspace_size": (C.c_size_t, [_D, C.c_int, C.c_int, C.c_int]),
+    "mmdit_adaptive_permute": (C.c_int, [C.POINTER(C.c_void_p), C.POINTER(C.c_void_p), C.c_int,
+                                         _D, C.c_int, C.c_int, C.c_int, _P, C.c_int, _P]),
+    "mmdit_block_select_table": (C.c_int, [_P, _P, _D, _P, _P, C.c_int, C.c_int, C.c_float,
+                                           C.c_float, C.c_int, _P, _P, _P, C.c_size_t, _P]),
+    "mmdit_block_select_table_workspace_size": (C.c_size_t, [_D, C.c_int]),
+    "mmdit_sparse_attn_table": (C.c_int, [_P, _P, _P, _P, _D, _P, _P, C.c_int, _P, _P, C.c_int,
+                                          C.c_float, _P, C.c_size_t, _P]),
+    "mmdit_sparse_attn_table_workspace_size": (C.c_size_t, [_D, C.c_int]),
     "mmdit_device_status": (C.c_int, [_P]),
     "mmdit_selftest_wait_timeout": (C.c_int, [C.c_int, _P, _P]),
     "mmdit_last_error": (C.c_char_p, []),
@@ -288,6 +309,84 @@ def sparse_attn(q, k, v, o, desc: TensorDesc, layout: Layout, block_idx, block_c
 
 def sparse_attn_workspace_size(desc: TensorDesc, layout: Layout, cap: int) -> int:
     return _lib.mmdit_sparse_attn_workspace_size(C.byref(desc), C.byref(layout), cap)
+
+
+def av_cross_attn_norms(qv, kv, vv, qa, ka, va, o_video, o_audio, video: TensorDesc,
+                        audio: TensorDesc, scale: float, video_norm, workspace=None,
+                        ws_bytes: int = 0, stream=None) -> None:
+    """av_cross_attn plus video_norm[b, n] = ||o_video[b, n]||_2 over all heads
+    (float [B, N_video]); workspace from av_cross_attn_norms_workspace_size."""
+    _check(_lib.mmdit_av_cross_attn_norms(_ptr(qv), _ptr(kv), _ptr(vv), _ptr(qa), _ptr(ka),
+                                          _ptr(va), _ptr(o_video), _ptr(o_audio), C.byref(video),
+                                          C.byref(audio), scale, _ptr(video_norm),
+                                          _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def av_cross_attn_norms_workspace_size(video: TensorDesc, audio: TensorDesc) -> int:
+    return _lib.mmdit_av_cross_attn_norms_workspace_size(C.byref(video), C.byref(audio))
+
+
+def adaptive_params(tau_128: float = 0.5, tau_256: float = 0.25, eps: float = 1e-6):
+    return AdaptiveParams(tau_128, tau_256, eps)
+
+
+def adaptive_num_zones(T: int, H: int, W: int) -> int:
+    return _lib.mmdit_adaptive_num_zones(T, H, W)
+
+
+def adaptive_max_blocks(T: int, H: int, W: int) -> int:
+    return _lib.mmdit_adaptive_max_blocks(T, H, W)
+
+
+def adaptive_plan_workspace_size(desc: TensorDesc, T: int, H: int, W: int) -> int:
+    return _lib.mmdit_adaptive_plan_workspace_size(C.byref(desc), T, H, W)
+
+
+def adaptive_plan(v, a_norm, desc: TensorDesc, T: int, H: int, W: int, zones, blocks, n_blocks,
+                  max_blocks: int, workspace=None, ws_bytes: int = 0,
+                  params: Optional[AdaptiveParams] = None, stream=None) -> None:
+    """Content-adaptive blocks of a raster video: zones int32 [B, n_zones, 4],
+    blocks int32 [B, max_blocks, 2], n_blocks int32 [B] (device)."""
+    _check(_lib.mmdit_adaptive_plan(_ptr(v), _ptr(a_norm), C.byref(desc), T, H, W, _ref(params),
+                                    _ptr(zones), _ptr(blocks), _ptr(n_blocks), max_blocks,
+                                    _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def adaptive_permute(srcs, dsts, desc: TensorDesc, T: int, H: int, W: int, zones,
+                     inverse: bool = False, stream=None) -> None:
+    """Raster -> adaptive storage order (inverse: back) of 1..3 tensors."""
+    n = len(srcs)
+    m = max(n, len(dsts), 1)
+    src = (C.c_void_p * m)(*[_ptr(x) for x in srcs])
+    dst = (C.c_void_p * m)(*[_ptr(x) for x in dsts])
+    _check(_lib.mmdit_adaptive_permute(src, dst, n, C.byref(desc), T, H, W, _ptr(zones),
+                                       1 if inverse else 0, _stream(stream)))
+
+
+def block_select_table(q, k, desc: TensorDesc, blocks, n_blocks, max_blocks: int, top_k: int,
+                       top_p: float, scale: float, cap: int, block_idx, block_cnt, workspace=None,
+                       ws_bytes: int = 0, stream=None) -> None:
+    _check(_lib.mmdit_block_select_table(_ptr(q), _ptr(k), C.byref(desc), _ptr(blocks),
+                                         _ptr(n_blocks), max_blocks, top_k, top_p, scale, cap,
+                                         _ptr(block_idx), _ptr(block_cnt), _ptr(workspace),
+                                         ws_bytes, _stream(stream)))
+
+
+def block_select_table_workspace_size(desc: TensorDesc, max_blocks: int) -> int:
+    return _lib.mmdit_block_select_table_workspace_size(C.byref(desc), max_blocks)
+
+
+def sparse_attn_table(q, k, v, o, desc: TensorDesc, blocks, n_blocks, max_blocks: int, block_idx,
+                      block_cnt, cap: int, scale: float, workspace=None, ws_bytes: int = 0,
+                      stream=None) -> None:
+    _check(_lib.mmdit_sparse_attn_table(_ptr(q), _ptr(k), _ptr(v), _ptr(o), C.byref(desc),
+                                        _ptr(blocks), _ptr(n_blocks), max_blocks, _ptr(block_idx),
+                                        _ptr(block_cnt), cap, scale, _ptr(workspace), ws_bytes,
+                                        _stream(stream)))
+
+
+def sparse_attn_table_workspace_size(desc: TensorDesc, max_blocks: int) -> int:
+    return _lib.mmdit_sparse_attn_table_workspace_size(C.byref(desc), max_blocks)
 
 
 def num_blocks(layout: Layout) -> int:

@@ -61,6 +61,8 @@ class Workload:
     top_p: float = 0.9
     theta: float = 10000.0
     extra: Dict = field(default_factory=dict)
+    plant_v: bool = False        # add the planted regions to V as well
+    adaptive: bool = False       # content-adaptive blocks (raster video, planned per step)
 
     @property
     def n_tokens(self) -> int:
@@ -125,6 +127,14 @@ WORKLOADS: Dict[str, Workload] = {
         "1080p_sparse", [video(21, 68, 120, order=ORDER_BLOCK444), audio(218)],
         batch=1, heads=24, head_dim=128, dtype="bf16", seed=4,
         qk_std=1.0, v_std=1.0, planted_regions=8, planted_amp=2.0, sparse=True),
+    # the 1080p layer with Prism's content-adaptive blocks: raster video whose
+    # values V carry the planted regions too (the zones' directional variance
+    # decides block volumes and shapes)
+    "1080p_adaptive": Workload(
+        "1080p_adaptive", [video(21, 68, 120), audio(218)],
+        batch=1, heads=24, head_dim=128, dtype="bf16", seed=6,
+        qk_std=1.0, v_std=1.0, planted_regions=8, planted_amp=2.0, sparse=True,
+        plant_v=True, adaptive=True),
     # a quarter of the 1080p grid (17 x 30 -> 17 x 15 blocks per frame slab):
     # the same structure at a size an ncu capture can hold (~2 GB on device)
     "1080p_sparse_quarter": Workload(
@@ -153,7 +163,7 @@ def reduced(name: str, T: int, H: int, W: int, n_audio: Optional[int] = None,
     return Workload(f"{name}_reduced_{T}x{H}x{W}", segs, batch or w.batch, heads,
                     w.head_dim, w.dtype, w.seed + seed_offset, w.qk_std, w.v_std,
                     w.planted_regions, w.planted_amp, w.mask, w.sparse, w.top_k,
-                    w.top_p, w.theta)
+                    w.top_p, w.theta, plant_v=w.plant_v, adaptive=w.adaptive)
 
 
 # ---------------------------------------------------------------------------
@@ -231,7 +241,7 @@ def _fill_chunk(out, name_idx, w, seed_seq, t0, t1, std, bump):
     rng = np.random.Generator(np.random.PCG64(seed_seq))
     x = rng.standard_normal((w.batch, t1 - t0, w.heads, w.head_dim), dtype=np.float32)
     x *= np.float32(std)
-    if bump is not None and name_idx < 2:
+    if bump is not None and (name_idx < 2 or w.plant_v):
         x += bump[None, t0:t1, None, None]
     out[:, t0:t1] = f32_to_bf16_bits(x) if w.dtype == "bf16" else x
 

@@ -27,7 +27,11 @@ reader can check it against the sources by eye:
     generation" -- reading guide of arXiv 2610.05416, Method section 3
     (mean-pooled key blocks, block probabilities P_i, and the attended set
     S_i = Top-k(P_i, k) U Top-p(P_i, p)); scope rule in the Method preamble
-    (only video self-attention is sparsified, cross-attention stays dense).
+    (only video self-attention is sparsified, cross-attention stays dense);
+    Key ideas and Method sections 1-2 (8x8x8 macro-zones, the dual-guidance
+    variation indicator g_d, block volumes B in {64, 128, 256} from a density
+    rho against tau_128 = 0.5 and tau_256 = 0.25, and the block shape nearest
+    to the optimal log-edges l*_d among 16 candidates).
 
 Readings where the sources are silent are stated at each function; the
 complete list is kept with the design notes of the repository.
@@ -446,3 +450,200 @@ def sparse_attn(q, k, v, blocks, sel, scale):
                 o[b, s0:s0 + n, h], _ = sparse_attn_rows(q, k, v, blocks, sel[b][h][i],
                                                          scale, b, h, i)
     return o
+
+
+# ---------------------------------------------------------------------------
+# Prism content-adaptive block shapes ([PRISM] Key ideas; Method 1 and 2)
+# ---------------------------------------------------------------------------
+
+ZONE = (8, 8, 8)          # Z_T x Z_H x Z_W macro-zone ([PRISM] Key ideas)
+TAU_128 = 0.5             # density threshold below which B(m) = 128 ([PRISM] Method 2)
+TAU_256 = 0.25            # density threshold below which B(m) = 256
+EPS_G = 1e-6              # the epsilon of g_d (reading: a small constant)
+VOLUMES = (64, 128, 256)  # B(m)
+
+
+def shape_candidates(volume: int) -> List[Tuple[int, int, int]]:
+    """The candidate block shapes C_B of one volume ([PRISM] Key ideas: 16
+    shapes over the volumes {64, 128, 256}).
+
+    Reading: the edges (b_T, b_H, b_W) are powers of two from 2 to the zone
+    edge 8 with product B; that gives 7 + 6 + 3 = 16 shapes, the count the
+    guide states.  Listed in ascending lexicographic order of the edges, the
+    order that breaks distance ties."""
+    out = []
+    for bt in (2, 4, 8):
+        for bh in (2, 4, 8):
+            for bw in (2, 4, 8):
+                if bt * bh * bw == volume:
+                    out.append((bt, bh, bw))
+    return out
+
+
+def macro_zones(T: int, H: int, W: int, zone=ZONE):
+    """Macro-zones of a T x H x W token volume ([PRISM] Key ideas), in
+    (zt, zh, zw) raster order, as (t0, h0, w0, et, eh, ew).  Reading: zones on
+    the far edge of an axis that the zone edge does not divide are short
+    (they hold only the real tokens)."""
+    out = []
+    for t0 in range(0, T, zone[0]):
+        for h0 in range(0, H, zone[1]):
+            for w0 in range(0, W, zone[2]):
+                out.append((t0, h0, w0, min(zone[0], T - t0), min(zone[1], H - h0),
+                            min(zone[2], W - w0)))
+    return out
+
+
+def directional_variance(x: np.ndarray) -> np.ndarray:
+    """sigma^2_d of one zone for d = T, H, W ([PRISM] Method 1).
+
+    x [Z_T, Z_H, Z_W, D]: the zone's features.  For axis d, the slice means
+    xbar^(d)_i average x over the zone's tokens with index i along d (the
+    other two axes); mu^(d) is the mean of those slice means over i; and
+    sigma^2_d = (1/D) sum_c (1/Z_d) sum_i (xbar^(d)_{i,c} - mu^(d)_c)^2."""
+    x = np.asarray(x, np.float64)
+    D = x.shape[3]
+    out = np.zeros(3)
+    for d in range(3):
+        other = tuple(a for a in range(3) if a != d)
+        xbar = x.mean(axis=other)             # [Z_d, D]
+        mu = xbar.mean(axis=0)                # [D]
+        out[d] = ((xbar - mu[None, :]) ** 2).mean(axis=0).sum() / D
+    return out
+
+
+def _ratio(sig: np.ndarray) -> np.ndarray:
+    """sigma^2_d / sum_d' sigma^2_d'; all zero when the sum is zero (reading)."""
+    tot = sig.sum()
+    return sig / tot if tot > 0 else np.zeros(3)
+
+
+def zone_indicators(v: np.ndarray, a: np.ndarray | None, T: int, H: int, W: int,
+                    eps: float = EPS_G):
+    """The dual-guidance indicator of every macro-zone ([PRISM] Method 1).
+
+    v : [T, H, W, D] value features of one video (D = heads x head_dim)
+    a : [T, H, W] or None: the A->V cross-attention output norms
+        a_{t,h,w} = ||h_{t,h,w}||_2 cached from the preceding layer; None
+        means no audio guidance (abar = 0).
+    Per zone m:
+      r_{v,d}(m)   = sigma^2_{v,d}(m) / sum_d' sigma^2_{v,d'}(m)
+      vhat_{a,d}(m) = sigma^2_{a,d}(m) / sum_d' sigma^2_{a,d'}(m)  (reading:
+                      the directional variance of the norms, normalised like r)
+      abar(m)      = mean of a over the zone / max over zones of that mean
+                      (reading: the coupling strength, normalised to [0, 1])
+      g_d(m)       = r_{v,d}(m) + abar(m) * vhat_{a,d}(m) + eps
+      rho(m)       = sum_d sigma^2_{v,d}(m) / max over zones of that sum
+                      (reading: the normalised spatio-temporal information
+                      density of Method 2)
+    Returns (zones, g [nz, 3], rho [nz], abar [nz])."""
+    zones = macro_zones(T, H, W)
+    nz = len(zones)
+    sig_v = np.zeros((nz, 3))
+    sig_a = np.zeros((nz, 3))
+    a_mean = np.zeros(nz)
+    for m, (t0, h0, w0, et, eh, ew) in enumerate(zones):
+        sig_v[m] = directional_variance(v[t0:t0 + et, h0:h0 + eh, w0:w0 + ew])
+        if a is not None:
+            az = np.asarray(a, np.float64)[t0:t0 + et, h0:h0 + eh, w0:w0 + ew]
+            sig_a[m] = directional_variance(az[..., None])
+            a_mean[m] = az.mean()
+    amax = a_mean.max() if nz else 0.0
+    abar = a_mean / amax if amax > 0 else np.zeros(nz)
+    tot = sig_v.sum(axis=1)
+    tmax = tot.max() if nz else 0.0
+    rho = tot / tmax if tmax > 0 else np.zeros(nz)
+    g = np.zeros((nz, 3))
+    for m in range(nz):
+        g[m] = _ratio(sig_v[m]) + abar[m] * _ratio(sig_a[m]) + eps
+    return zones, g, rho, abar
+
+
+def block_volume(rho: float) -> int:
+    """B(m) from the density rho(m) against tau_128 = 0.5 and tau_256 = 0.25
+    ([PRISM] Method 2).  Reading: dense zones keep the finest blocks --
+    B = 64 for rho >= tau_128, 128 for tau_256 <= rho < tau_128, 256 below."""
+    if rho >= TAU_128:
+        return 64
+    if rho >= TAU_256:
+        return 128
+    return 256
+
+
+def optimal_log_edges(g: np.ndarray, volume: int) -> np.ndarray:
+    """l*_d = -1/2 log2 g_d + 1/3 (S + 1/2 sum_d' log2 g_d'), S = log2 B(m):
+    the minimiser of sum_d g_d (b_d^2 - 1) subject to prod_d b_d = B(m), in
+    log2 space (b*_d proportional to g_d^(-1/2)) ([PRISM] Method 2)."""
+    lg = np.log2(np.asarray(g, np.float64))
+    S = math.log2(volume)
+    return -0.5 * lg + (S + 0.5 * lg.sum()) / 3.0
+
+
+def choose_shape(g: np.ndarray, volume: int) -> Tuple[int, int, int]:
+    """The candidate of C_B(m) at the smallest Euclidean distance from l*
+    in log2 space ([PRISM] Method 2); ties go to the earlier candidate."""
+    ls = optimal_log_edges(g, volume)
+    best, best_d = None, None
+    for c in shape_candidates(volume):
+        d = sum((math.log2(c[i]) - ls[i]) ** 2 for i in range(3))
+        if best_d is None or d < best_d:
+            best, best_d = c, d
+    return best
+
+
+def zone_blocks(zone, shape):
+    """Blocks of one zone cut with `shape`: (t0, h0, w0, et, eh, ew) in (bt,
+    bh, bw) raster order, clipped to the zone's real extent."""
+    t0, h0, w0, et, eh, ew = zone
+    out = []
+    for bt in range(0, et, shape[0]):
+        for bh in range(0, eh, shape[1]):
+            for bw in range(0, ew, shape[2]):
+                out.append((t0 + bt, h0 + bh, w0 + bw, min(shape[0], et - bt),
+                            min(shape[1], eh - bh), min(shape[2], ew - bw)))
+    return out
+
+
+def adaptive_layout(T: int, H: int, W: int, zones, shapes):
+    """Storage order of the content-adaptive blocks (reading: zones in
+    raster order, each zone's blocks in raster order, each block's tokens in
+    (t, h, w) raster order, so every block is one contiguous run of tokens).
+
+    Returns (perm, blocks): perm[s] is the raster index (t H + h) W + w of
+    the token stored at position s, and blocks the (start, length) of every
+    block in storage order."""
+    perm, blocks = [], []
+    for zone, shape in zip(zones, shapes):
+        for (t0, h0, w0, et, eh, ew) in zone_blocks(zone, shape):
+            blocks.append((len(perm), et * eh * ew))
+            for t in range(t0, t0 + et):
+                for h in range(h0, h0 + eh):
+                    for w in range(w0, w0 + ew):
+                        perm.append((t * H + h) * W + w)
+    return np.asarray(perm, np.int64), blocks
+
+
+def adaptive_plan(v: np.ndarray, a: np.ndarray | None, T: int, H: int, W: int,
+                  eps: float = EPS_G):
+    """The whole content-adaptive partition of one video ([PRISM] Method 1
+    and 2): indicator per zone, volume B(m), shape s*(m), storage order.
+
+    v [N, heads, d] (raster order, N = T H W); a [N] or None.
+    Returns dict(zones, g, rho, abar, volumes, shapes, perm, blocks)."""
+    v = np.asarray(v, np.float64)
+    vg = v.reshape(T, H, W, -1)
+    ag = None if a is None else np.asarray(a, np.float64).reshape(T, H, W)
+    zones, g, rho, abar = zone_indicators(vg, ag, T, H, W, eps)
+    volumes = [block_volume(r) for r in rho]
+    shapes = [choose_shape(g[m], volumes[m]) for m in range(len(zones))]
+    perm, blocks = adaptive_layout(T, H, W, zones, shapes)
+    return dict(zones=zones, g=g, rho=rho, abar=abar, volumes=volumes, shapes=shapes,
+                perm=perm, blocks=blocks)
+
+
+def cross_output_norms(o_video: np.ndarray) -> np.ndarray:
+    """a_{t,h,w} = ||h_{t,h,w}||_2: the L2 norm of every video token's A->V
+    cross-attention output over all heads and channels ([PRISM] Method 1;
+    cached for the next layer).  o_video [B, N, heads, d] -> [B, N]."""
+    o = np.asarray(o_video, np.float64)
+    return np.sqrt((o.reshape(o.shape[0], o.shape[1], -1) ** 2).sum(axis=2))

@@ -129,7 +129,9 @@ def test_block_counts_and_select_validation():
     assert M.num_blocks(_layout()) == 0  # raster: not a block-sparse layout
     d = _desc(n_tokens=171360, heads=24)
     ws = M.block_select_workspace_size(d, L)
-    assert ws == 2 * ((24 * 3060 * 128 * 4 + 255) // 256 * 256)
+    a = lambda n: (n + 255) // 256 * 256
+    # block table, its count, pooled Q and K means, fp32 block scores
+    assert ws == a(3060 * 8) + a(4) + 2 * a(24 * 3060 * 128 * 4) + a(24 * 3060 * 3060 * 4)
     assert _rc(M.block_select, FAKE, FAKE, d, L, 32, 0.9, 0.088, 3059, FAKE, FAKE, FAKE, ws) == M.EINVAL
     assert "cap" in M.last_error()
     assert _rc(M.block_select, FAKE, FAKE, d, L, 32, 1.5, 0.088, 3060, FAKE, FAKE, FAKE, ws) == M.EINVAL
@@ -223,3 +225,55 @@ def test_batch_limits_of_row_grids():
     d, lay = _desc(batch=65536), _cond_layout()
     assert f(FAKE, FAKE * 2, FAKE * 3, FAKE * 4, C.byref(d), C.byref(lay), C.c_float(0.1),
              FAKE * 5, 65536 * 80, 0x100000, 1 << 40, None) == M.EINVAL
+
+
+def test_adaptive_and_table_calls_validate_arguments():
+    T, H, W = 21, 68, 120
+    assert M.adaptive_num_zones(T, H, W) == 3 * 9 * 15
+    assert M.adaptive_max_blocks(T, H, W) == 8 * 405
+    assert M.adaptive_num_zones(0, 4, 4) == 0
+    d = _desc(n_tokens=T * H * W, heads=24)
+    mb = M.adaptive_max_blocks(T, H, W)
+    n = M.adaptive_plan_workspace_size(d, T, H, W)
+    assert n > 0 and M.adaptive_plan_workspace_size(d, T, H, W - 1) == 0
+    plan = lambda *a, **k: _rc(M.adaptive_plan, *a, **k)
+    assert plan(FAKE, None, d, T, H, W + 1, FAKE, FAKE, FAKE, mb, FAKE, n) == M.EINVAL
+    assert plan(FAKE, None, d, T, H, W, FAKE, FAKE, FAKE, mb - 1, FAKE, n) == M.EINVAL
+    assert plan(FAKE, None, d, T, H, W, FAKE, FAKE, FAKE, mb, FAKE, n - 1) == M.EWORKSPACE
+    assert plan(FAKE, None, d, T, H, W, FAKE + 8, FAKE, FAKE, mb, FAKE, n) == M.EINVAL  # zones align
+    bad = M.adaptive_params(0.2, 0.5, 1e-6)  # tau_256 > tau_128
+    assert plan(FAKE, None, d, T, H, W, FAKE, FAKE, FAKE, mb, FAKE, n, bad) == M.EINVAL
+    assert plan(FAKE, None, _desc(n_tokens=T * H * W, heads=24, dtype=M.F32), T, H, W, FAKE, FAKE,
+                FAKE, mb, FAKE, n) == M.EUNSUPPORTED
+    perm = lambda *a: _rc(M.adaptive_permute, *a)
+    assert perm([FAKE], [FAKE], d, T, H, W, FAKE) == M.EINVAL             # dst aliases src
+    assert perm([FAKE] * 4, [FAKE * 2] * 4, d, T, H, W, FAKE) == M.EINVAL  # at most three
+    assert perm([FAKE], [FAKE * 2], d, T, H, W, None) == M.EINVAL
+    # block-table selection / sparse attention
+    ns = M.block_select_table_workspace_size(d, mb)
+    assert ns > 0 and M.block_select_table_workspace_size(d, 7000) == 0
+    sel = lambda *a: _rc(M.block_select_table, *a)
+    assert sel(FAKE, FAKE, d, FAKE, FAKE, mb, 32, 0.9, 0.088, mb - 1, FAKE, FAKE, FAKE, ns) == M.EINVAL
+    assert sel(FAKE, FAKE, d, FAKE, FAKE, 7000, 32, 0.9, 0.088, 7000, FAKE, FAKE, FAKE, ns) == M.EINVAL
+    assert sel(FAKE, FAKE, d, None, FAKE, mb, 32, 0.9, 0.088, mb, FAKE, FAKE, FAKE, ns) == M.EINVAL
+    assert sel(FAKE, FAKE, d, FAKE, FAKE, mb, 32, 0.9, 0.088, mb, FAKE, FAKE, FAKE, ns - 1) == M.EWORKSPACE
+    nsp = M.sparse_attn_table_workspace_size(d, mb)
+    assert nsp > 0
+    sp = lambda *a: _rc(M.sparse_attn_table, *a)
+    args = [FAKE, FAKE + 4096, FAKE + 8192, FAKE + 12288]
+    assert sp(*args, d, FAKE, FAKE, mb, FAKE, FAKE, mb - 1, 0.088, FAKE, nsp) == M.EINVAL
+    assert sp(*args, d, FAKE + 4, FAKE, mb, FAKE, FAKE, mb, 0.088, FAKE, nsp) == M.EINVAL  # align
+    assert sp(*args, d, FAKE, FAKE, mb, FAKE, FAKE, mb, 0.088, FAKE, nsp - 1) == M.EWORKSPACE
+    assert sp(FAKE, FAKE, FAKE, FAKE, d, FAKE, FAKE, mb, FAKE, FAKE, mb, 0.088, FAKE, nsp) == M.EINVAL
+
+
+def test_cross_norms_validation():
+    dv, da = _desc(n_tokens=4096), _desc(n_tokens=218)
+    n = M.av_cross_attn_norms_workspace_size(dv, da)
+    assert n == M.av_cross_attn_workspace_size(dv, da) + (4096 * 2 * 4 + 255) // 256 * 256
+    ptrs = [FAKE + 4096 * i for i in range(8)]
+    f = lambda *a: _rc(M.av_cross_attn_norms, *a)
+    assert f(*ptrs, dv, da, 0.088, None, FAKE, n) == M.EINVAL
+    assert f(*ptrs, dv, da, 0.088, FAKE + 2, FAKE, n) == M.EINVAL
+    assert f(*ptrs, dv, da, 0.088, FAKE, FAKE, n - 1) == M.EWORKSPACE
+    assert f(*ptrs, dv, _desc(n_tokens=218, heads=3), 0.088, FAKE, FAKE, n) == M.EINVAL

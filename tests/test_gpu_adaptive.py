@@ -1,0 +1,382 @@
+"""GPU parity of Prism's content-adaptive blocks (Prism guide, Key ideas and
+Method sections 1-3) against the fp64 oracle, through the C ABI:
+
+* the A->V cross-attention output norms (mmdit_av_cross_attn_norms);
+* the plan (mmdit_adaptive_plan): every zone's shape number, storage start,
+  first block and block count, and the block table, exactly -- a zone whose
+  decision the oracle finds within 1e-5 of a threshold or of a distance tie
+  is the only allowed difference, and is counted;
+* the raster <-> adaptive permutation (bit-exact) on the oracle's plan;
+* selection and sparse attention over a block table (the oracle's table);
+* the whole chain plan -> permute -> select -> sparse -> permute back, on
+  the reduced case and on the full 1080p layer (sampled blocks).
+
+The GPU statistics are fp32 sums of the bf16 values and the plan arithmetic
+is fp64; the oracle is fp64 throughout on the same bf16 values."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle as O
+from joint_video_audio_rope_b200 import workloads as WL
+
+from _util import assert_close, selection_verdict
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+SHAPES = [c for B in O.VOLUMES for c in O.shape_candidates(B)]
+SCALE = 1 / math.sqrt(128)
+
+
+@pytest.fixture(scope="module")
+def M():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from joint_video_audio_rope_b200 import build
+    build.build()
+    from joint_video_audio_rope_b200 import mmdit
+    return mmdit
+
+
+def _up(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def _f64(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def _video(w, x, name):
+    v0, v1 = w.video_range()
+    return np.ascontiguousarray(x[name][:, v0:v1])
+
+
+def _grid(w):
+    s = w.segments[0]
+    return s["T"], s["H"], s["W"]
+
+
+def _tables(plan, max_blocks):
+    """The oracle plan as the C ABI's zone and block tables (one batch item)."""
+    nz = len(plan["zones"])
+    zones = np.zeros((1, nz, 4), np.int32)
+    start = first = 0
+    for m, (zone, shape) in enumerate(zip(plan["zones"], plan["shapes"])):
+        nb = len(O.zone_blocks(zone, shape))
+        zones[0, m] = (SHAPES.index(shape), start, first, nb)
+        start += zone[3] * zone[4] * zone[5]
+        first += nb
+    blocks = np.zeros((1, max_blocks, 2), np.int32)
+    blocks[0, :len(plan["blocks"])] = np.asarray(plan["blocks"], np.int32)
+    return zones, blocks, np.array([len(plan["blocks"])], np.int32)
+
+
+def _margins(plan):
+    """Per zone, how far the oracle's decision is from flipping: the density's
+    distance to the nearest threshold and the gap between the two nearest
+    candidate shapes of the chosen volume."""
+    out = []
+    for m in range(len(plan["zones"])):
+        rho = plan["rho"][m]
+        vm = min(abs(rho - O.TAU_128), abs(rho - O.TAU_256))
+        ls = O.optimal_log_edges(plan["g"][m], plan["volumes"][m])
+        d = sorted(sum((math.log2(c[i]) - ls[i]) ** 2 for i in range(3))
+                   for c in O.shape_candidates(plan["volumes"][m]))
+        out.append(min(vm, d[1] - d[0] if len(d) > 1 else 1.0))
+    return np.array(out)
+
+
+def _plan_gpu(M, w, vb, a_norm):
+    T, H, W = _grid(w)
+    v = _up(vb)
+    d = M.desc_of(v)
+    nz, mb = M.adaptive_num_zones(T, H, W), M.adaptive_max_blocks(T, H, W)
+    zones = torch.full((1, nz, 4), -1, dtype=torch.int32, device="cuda")
+    blocks = torch.full((1, mb, 2), -1, dtype=torch.int32, device="cuda")
+    nblk = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    n = M.adaptive_plan_workspace_size(d, T, H, W)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    a = None if a_norm is None else torch.from_numpy(a_norm.astype(np.float32)).cuda()
+    M.adaptive_plan(v, a, d, T, H, W, zones, blocks, nblk, mb, ws, n)
+    torch.cuda.synchronize()
+    assert M.device_status() == M.OK
+    return zones.cpu().numpy(), blocks.cpu().numpy(), nblk.cpu().numpy(), mb
+
+
+def _check_plan(plan, zones_g, blocks_g, nblk_g, mb, what):
+    zones_o, blocks_o, nblk_o = _tables(plan, mb)
+    margin = _margins(plan)
+    differ = np.nonzero(np.any(zones_g[0, :, :1] != zones_o[0, :, :1], axis=1))[0]
+    for m in differ:
+        assert margin[m] < 1e-5, (f"{what}: zone {m} shape {zones_g[0, m, 0]} vs oracle "
+                                  f"{zones_o[0, m, 0]} (margin {margin[m]:.2e})")
+    print(f"\n{what}: {len(plan['zones'])} zones, {len(differ)} excused at a near-tie; "
+          f"volumes {np.bincount(np.searchsorted([64, 128, 256], plan['volumes']), minlength=3)}")
+    if len(differ) == 0:
+        assert np.array_equal(zones_g, zones_o), what
+        assert nblk_g[0] == nblk_o[0]
+        assert np.array_equal(blocks_g[0, :nblk_o[0]], blocks_o[0, :nblk_o[0]]), what
+    return len(differ) == 0
+
+
+def _a_norm(T, H, W, seed):
+    """A positive, spatially varying stand-in for the norms a (an input)."""
+    rng = np.random.default_rng(seed)
+    t, h, w = np.meshgrid(np.arange(T), np.arange(H), np.arange(W), indexing="ij")
+    base = 1.0 + 0.8 * np.exp(-((w - W / 3) / (W / 6)) ** 2) * np.exp(-((t - T / 2) / 3.0) ** 2)
+    return (base + 0.05 * np.abs(rng.standard_normal((T, H, W)))).reshape(1, -1).astype(np.float32)
+
+
+REDUCED = dict(T=21, H=34, W=40, heads=4)
+
+
+def _reduced():
+    return WL.reduced("1080p_adaptive", REDUCED["T"], REDUCED["H"], REDUCED["W"],
+                      n_audio=37, heads=REDUCED["heads"])
+
+
+@pytest.mark.parametrize("with_audio", [False, True])
+def test_plan_matches_oracle(M, with_audio):
+    w = _reduced()
+    x = WL.generate(w)
+    T, H, W = _grid(w)
+    vb = _video(w, x, "v")
+    a = _a_norm(T, H, W, 3) if with_audio else None
+    zones_g, blocks_g, nblk_g, mb = _plan_gpu(M, w, vb, a)
+    plan = O.adaptive_plan(WL.as_f64(vb[0], "bf16"), None if a is None else a[0].astype(np.float64),
+                           T, H, W)
+    assert _check_plan(plan, zones_g, blocks_g, nblk_g, mb, f"plan audio={with_audio}")
+    assert len(set(plan["volumes"])) == 3  # the case exercises every volume
+
+
+def test_plan_edge_cases(M):
+    # a flat V (no variation anywhere) on a grid smaller than one zone: rho = 0
+    # gives B = 256; g is isotropic, so the three shapes of that volume tie
+    # (the margin is 0 and any of them may win); the zone is one block
+    w = WL.Workload("flat", [WL.video(5, 6, 7)], 1, 2, 128, "bf16", 1, 1.0, 1.0)
+    vb = np.full((1, 5 * 6 * 7, 2, 128), WL.f32_to_bf16_bits(np.float32(0.5)), np.uint16)
+    zones_g, blocks_g, nblk_g, mb = _plan_gpu(M, w, vb, None)
+    assert zones_g.shape[1] == 1 and zones_g[0, 0, 0] in (13, 14, 15) and nblk_g[0] == 1
+    assert tuple(blocks_g[0, 0]) == (0, 210) and tuple(zones_g[0, 0, 1:]) == (0, 0, 1)
+    # one zone varying strongly along t and weakly along h (no tie): B = 64
+    # (rho = 1) and the oracle's shape, exactly
+    t = np.arange(5, dtype=np.float32)[:, None, None]
+    hh = np.arange(6, dtype=np.float32)[None, :, None]
+    g = np.broadcast_to(0.3 * t + 0.05 * hh, (5, 6, 7)).reshape(-1)
+    vb2 = np.repeat(WL.f32_to_bf16_bits(g)[None, :, None, None], 2, axis=2).repeat(128, axis=3)
+    zones_g, blocks_g, nblk_g, mb = _plan_gpu(M, w, vb2, None)
+    plan = O.adaptive_plan(WL.as_f64(vb2[0], "bf16"), None, 5, 6, 7)
+    assert plan["volumes"] == [64] and plan["shapes"][0][0] == 2
+    assert _check_plan(plan, zones_g, blocks_g, nblk_g, mb, "one zone")
+
+
+def test_permute_is_the_oracle_order(M):
+    w = _reduced()
+    x = WL.generate(w)
+    T, H, W = _grid(w)
+    vb = _video(w, x, "v")
+    plan = O.adaptive_plan(WL.as_f64(vb[0], "bf16"), None, T, H, W)
+    zones_o, _, _ = _tables(plan, M.adaptive_max_blocks(T, H, W))
+    src = [_up(_video(w, x, n)) for n in ("q", "k", "v")]
+    dst = [torch.empty_like(t) for t in src]
+    d = M.desc_of(src[0])
+    z = torch.from_numpy(zones_o).cuda()
+    M.adaptive_permute(src, dst, d, T, H, W, z)
+    back = [torch.empty_like(t) for t in src]
+    M.adaptive_permute(dst, back, d, T, H, W, z, inverse=True)
+    torch.cuda.synchronize()
+    perm = plan["perm"]
+    for i, n in enumerate(("q", "k", "v")):
+        ref = _video(w, x, n)[:, perm]
+        got = dst[i].cpu().view(torch.int16).numpy().view(np.uint16)
+        assert np.array_equal(got, ref), n
+        assert torch.equal(back[i], src[i]), n
+
+
+def _permuted(w, x, plan):
+    return {n: np.ascontiguousarray(_video(w, x, n)[:, plan["perm"]]) for n in ("q", "k", "v")}
+
+
+def test_table_select_and_sparse_on_the_oracle_plan(M):
+    w = _reduced()
+    x = WL.generate(w)
+    T, H, W = _grid(w)
+    plan = O.adaptive_plan(WL.as_f64(_video(w, x, "v")[0], "bf16"), None, T, H, W)
+    mb = M.adaptive_max_blocks(T, H, W)
+    _, blocks_o, nblk_o = _tables(plan, mb)
+    px = _permuted(w, x, plan)
+    dev = {n: _up(px[n]) for n in px}
+    d = M.desc_of(dev["q"])
+    blocks_t = torch.from_numpy(blocks_o).cuda()
+    nblk_t = torch.from_numpy(nblk_o).cuda()
+    idx = torch.full((1, w.heads, mb, mb), -1, dtype=torch.int32, device="cuda")
+    cnt = torch.full((1, w.heads, mb), -1, dtype=torch.int32, device="cuda")
+    n = M.block_select_table_workspace_size(d, mb)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    M.block_select_table(dev["q"], dev["k"], d, blocks_t, nblk_t, mb, w.top_k, w.top_p, SCALE, mb,
+                         idx, cnt, ws, n)
+    torch.cuda.synchronize()
+    assert M.device_status() == M.OK
+    hq, hk, hv = (WL.as_f64(px[c], "bf16") for c in ("q", "k", "v"))
+    blocks = plan["blocks"]
+    qb, kb = O.pool(hq, blocks), O.pool(hk, blocks)
+    p32 = float(np.float32(w.top_p))
+    idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
+    excused = 0
+    sel = [[None] * w.heads]
+    for h in range(w.heads):
+        ref_all = O.select_rows(qb[0, h], kb[0, h], w.top_k, p32, SCALE)
+        sel[0][h] = ref_all
+        for i in range(len(blocks)):
+            got = idx_h[0, h, i, :cnt_h[0, h, i]]
+            if np.array_equal(got, ref_all[i]):
+                continue
+            v = selection_verdict(got, ref_all[i], O.block_probs(qb[0, h, i], kb[0, h], SCALE),
+                                  w.top_k, p32)
+            assert v == "tie", f"select h{h} blk{i}: {v}"
+            excused += 1
+    rows = w.heads * len(blocks)
+    print(f"\ntable selection: {rows} rows, {excused} excused at an fp32 tie")
+    assert excused <= max(1, 0.005 * rows)
+    # sparse attention over the table with the oracle's selection
+    idx_o = np.full((1, w.heads, mb, mb), -1, np.int32)
+    cnt_o = np.zeros((1, w.heads, mb), np.int32)
+    for h in range(w.heads):
+        for i, s in enumerate(sel[0][h]):
+            idx_o[0, h, i, :len(s)] = s
+            cnt_o[0, h, i] = len(s)
+    o = torch.full_like(dev["q"], float("nan"))
+    n2 = M.sparse_attn_table_workspace_size(d, mb)
+    ws2 = torch.empty(n2, dtype=torch.uint8, device="cuda")
+    M.sparse_attn_table(dev["q"], dev["k"], dev["v"], o, d, blocks_t, nblk_t, mb,
+                        torch.from_numpy(idx_o).cuda(), torch.from_numpy(cnt_o).cuda(), mb, SCALE,
+                        ws2, n2)
+    torch.cuda.synchronize()
+    assert M.device_status() == M.OK
+    ref = O.sparse_attn(hq, hk, hv, blocks, sel, SCALE)
+    assert_close(_f64(o), ref, "bf16", "sparse over the adaptive table")
+    # every block selected: dense attention
+    all_idx = np.tile(np.arange(mb, dtype=np.int32), (1, w.heads, mb, 1))
+    all_cnt = np.full((1, w.heads, mb), len(blocks), np.int32)
+    M.sparse_attn_table(dev["q"], dev["k"], dev["v"], o, d, blocks_t, nblk_t, mb,
+                        torch.from_numpy(all_idx).cuda(), torch.from_numpy(all_cnt).cuda(), mb,
+                        SCALE, ws2, n2)
+    torch.cuda.synchronize()
+    dense, _ = O.joint_attn(hq, hk, hv, SCALE)
+    assert_close(_f64(o), dense, "bf16", "all adaptive blocks = dense")
+
+
+def test_cross_attention_output_norms(M):
+    w = WL.reduced("480p", 3, 10, 12, n_audio=50, n_text=4, heads=3)
+    x = WL.generate(w)
+    q, k, v = _up(x["q"]), _up(x["k"]), _up(x["v"])
+    v0, v1 = w.video_range()
+    a0, a1 = w.audio_range()
+    oc = torch.full_like(q, float("nan"))
+    dv, da = M.desc_of(q[:, v0:v1]), M.desc_of(q[:, a0:a1])
+    n = M.av_cross_attn_norms_workspace_size(dv, da)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    norms = torch.full((1, v1 - v0), float("nan"), device="cuda")
+    M.av_cross_attn_norms(q[:, v0:v1], k[:, v0:v1], v[:, v0:v1], q[:, a0:a1], k[:, a0:a1],
+                          v[:, a0:a1], oc[:, v0:v1], oc[:, a0:a1], dv, da, SCALE, norms, ws, n)
+    torch.cuda.synchronize()
+    assert M.device_status() == M.OK
+    hq, hk, hv = (WL.as_f64(x[c], "bf16") for c in ("q", "k", "v"))
+    ref_v, ref_a = O.av_cross_attn(hq[:, v0:v1], hk[:, v0:v1], hv[:, v0:v1], hq[:, a0:a1],
+                                   hk[:, a0:a1], hv[:, a0:a1], SCALE)
+    assert_close(_f64(oc[:, v0:v1]), ref_v, "bf16", "cross v<-a")
+    assert_close(_f64(oc[:, a0:a1]), ref_a, "bf16", "cross a<-v")
+    assert_close(norms.cpu().numpy().astype(np.float64), O.cross_output_norms(ref_v), "bf16",
+                 "A->V output norms")
+
+
+def _chain_gpu(M, w, x, a_norm):
+    """plan -> permute Q, K, V -> table selection -> table sparse attention ->
+    permute O back, all on the GPU."""
+    T, H, W = _grid(w)
+    qv, kv, vv = (_up(_video(w, x, n)) for n in ("q", "k", "v"))
+    d = M.desc_of(qv)
+    nz, mb = M.adaptive_num_zones(T, H, W), M.adaptive_max_blocks(T, H, W)
+    zones = torch.empty((1, nz, 4), dtype=torch.int32, device="cuda")
+    blocks = torch.empty((1, mb, 2), dtype=torch.int32, device="cuda")
+    nblk = torch.empty((1,), dtype=torch.int32, device="cuda")
+    n = max(M.adaptive_plan_workspace_size(d, T, H, W), M.block_select_table_workspace_size(d, mb),
+            M.sparse_attn_table_workspace_size(d, mb))
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    a = None if a_norm is None else torch.from_numpy(a_norm).cuda()
+    M.adaptive_plan(vv, a, d, T, H, W, zones, blocks, nblk, mb, ws, n)
+    pq, pk, pv = (torch.empty_like(t) for t in (qv, kv, vv))
+    M.adaptive_permute([qv, kv, vv], [pq, pk, pv], d, T, H, W, zones)
+    idx = torch.empty((1, w.heads, mb, mb), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((1, w.heads, mb), dtype=torch.int32, device="cuda")
+    M.block_select_table(pq, pk, d, blocks, nblk, mb, w.top_k, w.top_p, SCALE, mb, idx, cnt, ws, n)
+    po = torch.empty_like(pq)
+    M.sparse_attn_table(pq, pk, pv, po, d, blocks, nblk, mb, idx, cnt, mb, SCALE, ws, n)
+    o = torch.empty_like(pq)
+    M.adaptive_permute([po], [o], d, T, H, W, zones, inverse=True)
+    torch.cuda.synchronize()
+    assert M.device_status() == M.OK
+    return (zones.cpu().numpy(), blocks.cpu().numpy(), nblk.cpu().numpy(), mb, idx.cpu().numpy(),
+            cnt.cpu().numpy(), o)
+
+
+def _check_chain(w, x, a_norm, res, heads, blk_sample, what):
+    T, H, W = _grid(w)
+    zones_g, blocks_g, nblk_g, mb, idx_h, cnt_h, o = res
+    plan = O.adaptive_plan(WL.as_f64(_video(w, x, "v")[0], "bf16"),
+                           None if a_norm is None else a_norm[0].astype(np.float64), T, H, W)
+    assert _check_plan(plan, zones_g, blocks_g, nblk_g, mb, what), \
+        f"{what}: the plan differs at a near-tie; the chain cannot be compared"
+    px = _permuted(w, x, plan)
+    blocks = plan["blocks"]
+    p32 = float(np.float32(w.top_p))
+    got_o = o[0]
+    perm = plan["perm"]
+    excused = skipped = 0
+    for h in heads:
+        hq, hk, hv = (WL.as_f64(px[c][0, :, h:h + 1], "bf16") for c in ("q", "k", "v"))
+        qb, kb = O.pool(hq[None], blocks), O.pool(hk[None], blocks)
+        ref_all = O.select_rows(qb[0, 0], kb[0, 0], w.top_k, p32, SCALE)
+        for i in range(len(blocks)):
+            got = idx_h[0, h, i, :cnt_h[0, h, i]]
+            if not np.array_equal(got, ref_all[i]):
+                v = selection_verdict(got, ref_all[i], O.block_probs(qb[0, 0, i], kb[0, 0], SCALE),
+                                      w.top_k, p32)
+                assert v == "tie", f"{what} select h{h} blk{i}: {v}"
+                excused += 1
+        for i in (range(len(blocks)) if blk_sample is None else blk_sample):
+            if not np.array_equal(idx_h[0, h, i, :cnt_h[0, h, i]], ref_all[i]):
+                skipped += 1
+                continue
+            s0, nn = blocks[i]
+            ref, _ = O.sparse_attn_rows(hq[None], hk[None], hv[None], blocks, ref_all[i], SCALE,
+                                        0, 0, i)
+            # output rows in raster order: storage positions s0..s0+nn map to perm[s]
+            assert_close(_f64(got_o[perm[s0:s0 + nn], h]), ref, "bf16", f"{what} sparse h{h} blk{i}")
+    rows = len(heads) * len(blocks)
+    print(f"\n{what}: {rows} selection rows, {excused} excused, {skipped} sparse blocks skipped")
+    assert excused <= max(1, 0.005 * rows)
+    assert skipped <= max(1, 0.005 * rows)
+
+
+def test_chain_reduced(M):
+    w = _reduced()
+    x = WL.generate(w)
+    T, H, W = _grid(w)
+    a = _a_norm(T, H, W, 5)
+    res = _chain_gpu(M, w, x, a)
+    _check_chain(w, x, a, res, range(w.heads), None, "adaptive chain (reduced)")
+
+
+def test_chain_full_size_1080p(M):
+    w = WL.WORKLOADS["1080p_adaptive"]
+    x = WL.generate(w)
+    T, H, W = _grid(w)
+    a = _a_norm(T, H, W, 6)
+    res = _chain_gpu(M, w, x, a)
+    rng = np.random.default_rng(7)
+    nb = int(res[2][0])
+    sample = np.unique(np.concatenate([rng.choice(nb, 24, replace=False), [0, nb - 1]]))
+    _check_chain(w, x, a, res, [0, 11, 23], sample, "adaptive chain (1080p)")
