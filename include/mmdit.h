@@ -481,7 +481,9 @@ MMDIT_API int mmdit_num_blocks(const mmdit_layout* layout);
 
 /* Reads and clears the device error flag of the current device after
  * synchronising `stream`: MMDIT_OK, or MMDIT_ETIMEOUT if a bounded wait ran out
- * in a kernel since the last call, or MMDIT_ECUDA. */
+ * in a kernel since the last call, or MMDIT_EDEVCHECK if a device-side index
+ * check of the checked build failed, or MMDIT_ECUDA.  While the flag is set,
+ * the library's attention kernels skip their work. */
 MMDIT_API int mmdit_device_status(mmdit_stream_t stream);
 
 /* Diagnostic, no counterpart on the source pages: launches one warp that

@@ -1,6 +1,12 @@
 """Build the sm_100a shared library libmmdit.so in-tree with nvcc.
 
-    python -m joint_video_audio_rope_b200.build [--force] [--verbose]
+    python -m joint_video_audio_rope_b200.build [--force] [--verbose] [--device-checks]
+
+--device-checks builds the debug variant libmmdit_checked.so instead: kernels
+check the indices they read from caller data (block ids and counts, block
+tables) on the device and record MMDIT_EDEVCHECK in the device error word
+when one is out of range (read back by mmdit_device_status); nothing traps.
+Load it by pointing the binding at it (MMDIT_LIB=.../libmmdit_checked.so).
 
 Compiles every .cu file under csrc/ for sm_100a (-gencode
 arch=compute_100a,code=sm_100a) with -lineinfo and links them, with the CUDA
@@ -21,6 +27,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OUT = os.path.join(PKG, "libmmdit.so")
+OUT_CHECKED = os.path.join(PKG, "libmmdit_checked.so")
 BUILD = os.path.join(ROOT, "_build")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -39,23 +46,27 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(OUT):
+def _stale(out: str = OUT) -> bool:
+    if not os.path.exists(out):
         return True
-    t = os.path.getmtime(OUT)
+    t = os.path.getmtime(out)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h"))
     deps.append(os.path.join(ROOT, "include", "mmdit.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False) -> str:
-    if not force and not _stale():
-        return OUT
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False,
+          device_checks: bool = False) -> str:
+    out = OUT_CHECKED if device_checks else OUT
+    if not force and not _stale(out):
+        return out
+    bdir = os.path.join(BUILD, "checked") if device_checks else BUILD
+    os.makedirs(bdir, exist_ok=True)
+    defs = ["-DMMDIT_DEVICE_CHECKS"] if device_checks else []
     objs, cmds = [], []
     for src in sources():
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
-        cmd = [nvcc(), *ARCH, *FLAGS, "-c", src, "-o", obj]
+        obj = os.path.join(bdir, os.path.basename(src) + ".o")
+        cmd = [nvcc(), *ARCH, *FLAGS, *defs, "-c", src, "-o", obj]
         if ptxas_verbose:
             cmd += ["-Xptxas", "-v"]
         if verbose:
@@ -69,13 +80,13 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
             if r.stdout or r.stderr:
                 print(r.stdout + r.stderr, end="", flush=True)
             r.check_returncode()
-    tmp = OUT + ".tmp"
+    tmp = out + ".tmp"
     cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-Xcompiler", "-fPIC"]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, OUT)
-    return OUT
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":
@@ -83,6 +94,8 @@ if __name__ == "__main__":
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-verbose", action="store_true")
+    ap.add_argument("--device-checks", action="store_true")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.verbose, ptxas_verbose=a.ptxas_verbose))
+    print(build(force=a.force, verbose=a.verbose, ptxas_verbose=a.ptxas_verbose,
+                device_checks=a.device_checks))
     sys.exit(0)

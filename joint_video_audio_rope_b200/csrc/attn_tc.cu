@@ -573,10 +573,21 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
         }
         const bool masked = len0 < 64 || len1 < 64 || seg0 != 0xFu || seg1 != 0xFu;
         if (masked) {
+          // per 16-column segment: the valid columns are a prefix (the key
+          // run's length cuts at most one segment per half; a segment whose
+          // membership bit is clear has none), so a full segment costs one
+          // comparison and only a cut or cleared one touches its columns
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            if (c >= len0 || !((seg0 >> (c >> 4)) & 1u)) s[c] = -INFINITY;
-            if (c >= len1 || !((seg1 >> (c >> 4)) & 1u)) s[64 + c] = -INFINITY;
+          for (int g = 0; g < 8; ++g) {
+            const uint32_t segm = g < 4 ? seg0 : seg1;
+            const int len = g < 4 ? len0 : len1;
+            const int base = (g & 3) * 16;
+            const int lim = ((segm >> (g & 3)) & 1u) ? min(max(len - base, 0), 16) : 0;
+            if (lim < 16) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                if (i >= lim) s[(g >> 2) * 64 + base + i] = -INFINITY;
+            }
           }
         }
         const float mt = row_max128(s);
@@ -874,8 +885,8 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
     if (p.q_tiles != 2 || !p.persistent) return cudaErrorInvalidValue;
     return launch_shape<2, 4, true, true>(p, s);
   }
-  if (p.q_tiles == 1)
-    return p.persistent ? launch_shape<1, 2, true>(p, s) : launch_shape<1, 2, false>(p, s);
+  if (p.q_tiles == 1)  // one-tile CTAs are always persistent (short key sequences)
+    return p.persistent ? launch_shape<1, 2, true>(p, s) : cudaErrorInvalidValue;
   return p.persistent ? launch_shape<2, 4, true>(p, s) : launch_shape<2, 4, false>(p, s);
 }
 

@@ -111,6 +111,12 @@ struct AttnParams {
 };
 
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s);
+// Queries over at most kShortKeys keys (attn_short.cu): every key in one
+// N = 256 tile, single-pass softmax, K/V resident per (batch, head).  Uses the
+// fields of a dense persistent one-tile problem (tmQ, tmK, tmV, tmO with a
+// 32-channel store box, Nq, Nkv, H, B, row_sq).
+constexpr int kShortKeys = 256;
+cudaError_t launch_attn_short(const AttnParams& p, cudaStream_t s);
 // Both directions of the audio<->video cross-attention on one stream: audio
 // queries over the video keys (split-KV partials into part_o / part_ml), video
 // queries over the audio keys, then the merge of the partials.

@@ -282,7 +282,9 @@ int launch_cross(const void* qv, const void* kv, const void* vv, const void* qa,
     return rc;
   pv.prob.row_sq = video_norm != nullptr ? row_sq : nullptr;
   cudaError_t e = launch_attn_tc(pa, s);
-  if (e == cudaSuccess) e = launch_attn_tc(pv, s);
+  // video queries: every audio key in one tile when there are at most 256
+  if (e == cudaSuccess)
+    e = audio.n_tokens <= kShortKeys ? launch_attn_short(pv, s) : launch_attn_tc(pv, s);
   if (e == cudaSuccess)
     e = launch_split_combine(part_o, part_ml, (__nv_bfloat16*)o_audio, audio.stride_tok,
                              audio.stride_batch, splits, audio.batch, audio.heads, audio.n_tokens,
@@ -330,7 +332,9 @@ int mmdit_device_status(mmdit_stream_t stream) {
   if (v != 0) {
     const int zero = 0;
     cudaMemcpyToSymbol(g_device_error_word, &zero, sizeof(int));
-    return fail(v, "a bounded device wait ran out (status %d)", v);
+    return fail(v, v == MMDIT_EDEVCHECK ? "a device-side index check failed (status %d)"
+                                        : "a bounded device wait ran out (status %d)",
+                v);
   }
   return MMDIT_OK;
 }

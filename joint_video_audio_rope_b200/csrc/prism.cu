@@ -353,7 +353,8 @@ struct PermuteArgs {
 // heads * 128 bf16 in 16-byte vectors; strides in 16-byte units.
 __global__ void __launch_bounds__(256) permute_kernel(PermuteArgs pa, long long st, long long sb,
                                                       int row_u4, ZoneGrid zg,
-                                                      const int4* __restrict__ zones, int inverse) {
+                                                      const int4* __restrict__ zones, int inverse,
+                                                      int* err) {
   const int b = blockIdx.y;
   const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int N = zg.T * zg.H * zg.W;
@@ -361,6 +362,9 @@ __global__ void __launch_bounds__(256) permute_kernel(PermuteArgs pa, long long 
   const int lane = threadIdx.x & 31;
   const int t = r / (zg.H * zg.W), rem = r - t * zg.H * zg.W, h = rem / zg.W, w = rem - h * zg.W;
   const int s = storage_index(zg, zones + (long long)b * zg.count(), t, h, w);
+  // a zone table that is not a plan of this grid must not move rows outside it
+  MMDIT_DCHECK(s >= 0 && s < N, err);
+  if (s < 0 || s >= N) return;
   const long long from = b * sb + (long long)(inverse ? s : r) * st;
   const long long to = b * sb + (long long)(inverse ? r : s) * st;
   for (int x = 0; x < pa.n; ++x)
@@ -503,10 +507,12 @@ int mmdit_adaptive_permute(const void* const* src, void* const* dst, int n_tenso
   }
   if (desc->n_tokens == 0) return MMDIT_OK;
   if ((rc = check_sm100())) return rc;
+  int* err = device_error_flag();
+  if (err == nullptr) return fail(MMDIT_ECUDA, "device error flag unavailable");
   const ZoneGrid zg = zone_grid(T, H, W);
   permute_kernel<<<dim3((desc->n_tokens + 7) / 8, desc->batch), 256, 0, (cudaStream_t)stream>>>(
       pa, desc->stride_tok / 8, desc->stride_batch / 8, desc->heads * 16, zg,
-      reinterpret_cast<const int4*>(zones), inverse != 0);
+      reinterpret_cast<const int4*>(zones), inverse != 0, err);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? MMDIT_OK : cuda_fail(e, "adaptive_permute launch");
 }

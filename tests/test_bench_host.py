@@ -37,3 +37,22 @@ def test_traffic_reported_only_for_the_captured_source(monkeypatch):
     monkeypatch.setitem(bench.NCU_TRAFFIC, "480p", {"src": "0" * 16, "bytes": 123})
     assert bench.ncu_traffic("480p") is None
     assert bench.ncu_traffic("no such workload") is None
+
+
+def test_peak_follows_the_length_of_the_timed_region():
+    peaks = {"bf16_tflops": 1638.7, "bf16_tflops_sustained": 1372.3}
+    assert bench.pick_peak(peaks, 240.0) == (1638.7, "bf16_tflops")       # a burst
+    assert bench.pick_peak(peaks, 2970.0) == (1372.3, "bf16_tflops_sustained")
+    assert bench.pick_peak({}, 5000.0)[0] == bench.FALLBACK_PEAKS["bf16_tflops_sustained"]
+
+
+def test_selected_pair_flops_with_block_lengths():
+    import numpy as np
+    w = WL.WORKLOADS["1080p_adaptive"]
+    # two heads' worth: block lengths 64, 128, 256; rows select {0}, {0, 2}, {1}
+    w2 = WL.Workload("t", w.segments, 1, 2, 128, "bf16", 0, 1.0, 1.0)
+    idx = np.array([[[[0, -1, -1], [0, 2, -1], [1, -1, -1]]] * 2])
+    cnt = np.array([[[1, 2, 1]] * 2])
+    blen = [np.array([64, 128, 256])]
+    pairs = 64 * 64 + 128 * (64 + 256) + 256 * 128
+    assert bench.selected_pair_flops(w2, idx, cnt, blen) == 4.0 * 128 * 2 * pairs

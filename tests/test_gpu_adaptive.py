@@ -21,7 +21,7 @@ import pytest
 import oracle as O
 from joint_video_audio_rope_b200 import workloads as WL
 
-from _util import assert_close, selection_verdict
+from _util import assert_close, fp32_tie_tol, selection_verdict
 
 pytestmark = pytest.mark.gpu
 
@@ -234,7 +234,7 @@ def test_table_select_and_sparse_on_the_oracle_plan(M):
             if np.array_equal(got, ref_all[i]):
                 continue
             v = selection_verdict(got, ref_all[i], O.block_probs(qb[0, h, i], kb[0, h], SCALE),
-                                  w.top_k, p32)
+                                  w.top_k, p32, ltol=fp32_tie_tol(qb[0, h, i], kb[0, h], SCALE, 256))
             assert v == "tie", f"select h{h} blk{i}: {v}"
             excused += 1
     rows = w.heads * len(blocks)
@@ -343,7 +343,8 @@ def _check_chain(w, x, a_norm, res, heads, blk_sample, what):
             got = idx_h[0, h, i, :cnt_h[0, h, i]]
             if not np.array_equal(got, ref_all[i]):
                 v = selection_verdict(got, ref_all[i], O.block_probs(qb[0, 0, i], kb[0, 0], SCALE),
-                                      w.top_k, p32)
+                                      w.top_k, p32,
+                                      ltol=fp32_tie_tol(qb[0, 0, i], kb[0, 0], SCALE, 256))
                 assert v == "tie", f"{what} select h{h} blk{i}: {v}"
                 excused += 1
         for i in (range(len(blocks)) if blk_sample is None else blk_sample):

@@ -9,7 +9,7 @@ import numpy as np
 
 import oracle as O
 
-from _util import selection_matches, selection_verdict
+from _util import fp32_tie_tol, selection_matches, selection_verdict
 
 
 def _probs(n, seed):
@@ -98,3 +98,37 @@ def test_garbage_on_a_near_tied_row_is_rejected():
     assert selection_verdict(garbage, ref, P, 1, p) == "mismatch"
     missing_top = np.array(sorted(order[1:len(ref) + 1]))
     assert selection_verdict(missing_top, ref, P, 1, p) == "mismatch"
+
+
+def test_fp32_tie_band_from_the_score_error_bound():
+    # a row of near-uniform probabilities (a background query block): blocks
+    # whose log-probabilities differ by less than the fp32 error bound of the
+    # scores are ties; a wider gap is not
+    rng = np.random.default_rng(4)
+    d, n = 128, 50
+    qbar = rng.standard_normal(d) * 0.05
+    kbar = rng.standard_normal((n, d)) * 0.05
+    scale = 1 / np.sqrt(d)
+    ltol = fp32_tie_tol(qbar, kbar, scale, 64)
+    assert np.all(ltol > 0) and np.all(ltol < 1e-5)
+    # the bound: at least the d-term dot product's worst case
+    a = np.abs(kbar * qbar).sum(1) * scale
+    assert np.all(ltol >= 2.0 ** -24 * d * a)
+    s = (kbar @ qbar) * scale
+    P = np.exp(s - s.max())
+    P /= P.sum()
+    order = _ranked(P)
+    k = 10
+    a_, b_ = order[k - 1], order[k]
+    # place block b_ just below a_, within and then beyond the tie band
+    for factor, expect in ((0.5, "tie"), (3.0, "mismatch")):
+        Q = P.copy()
+        gap = factor * (ltol[a_] + ltol[b_])
+        Q[b_] = Q[a_] * np.exp(-gap)
+        ref = O.select_from_probs(Q, k, 0.0)
+        swapped = np.array(sorted(set(ref.tolist()) - {a_} | {b_}))
+        assert selection_verdict(swapped, ref, Q, k, 0.0, ltol=ltol) == expect
+    # far below the cutoff is never a tie
+    ref = O.select_from_probs(P, k, 0.0)
+    wrong = np.array(sorted(set(ref.tolist()) - {order[k - 1]} | {order[-1]}))
+    assert selection_verdict(wrong, ref, P, k, 0.0, ltol=ltol) == "mismatch"
