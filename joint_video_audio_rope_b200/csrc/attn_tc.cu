@@ -97,7 +97,9 @@ enum {
   B_OEMPTY = 20,  // 2: epilogue has read O out of TMEM (128 arrivals)
   B_MMADONE = 22, // 1: every MMA of the CTA done (teardown)
   B_PHALF = 23,   // 2: first 64 keys of the P tile written (128 arrivals)
-  B_COUNT = 25
+  B_EXPTOK = 25,  // 2: the other softmax warpgroup has finished its exponentials
+                  //    of its latest key tile (128 arrivals; two Q tiles only)
+  B_COUNT = 27
 };
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0, 0);  // Q, K: K-major
@@ -229,6 +231,36 @@ __device__ __forceinline__ void kv_tile(const AttnProblem& pr, const Work& w, in
   }
 }
 
+// Sparse mode: the query blocks (bits of the group) that selected any key
+// block of key tile j, from the membership masks of its two list entries.
+__device__ __forceinline__ uint32_t tile_members(const AttnProblem& pr, const Work& w, int j) {
+  const uint4 e0 = pr.ulist[w.ubase + 2 * j];
+  uint32_t m = e0.z | e0.w;
+  if (2 * j + 1 < w.ucount) {
+    const uint4 e1 = pr.ulist[w.ubase + 2 * j + 1];
+    m |= e1.z | e1.w;
+  }
+  return (m | (m >> 16)) & 0xFFFFu;
+}
+
+// Sparse mode: for each 128-row Q tile of the group, the query blocks whose
+// rows it holds (bit i = block i of the group).
+template <int QT>
+__device__ __forceinline__ void tile_blocks(const AttnProblem& pr, const Work& w,
+                                            uint32_t (&qm)[QT]) {
+  const int2* tb = pr.tab + (long long)w.b * pr.tab_cap + w.g_first;
+  int acc = 0;
+#pragma unroll
+  for (int t = 0; t < QT; ++t) qm[t] = 0u;
+  for (int i = 0; i < w.g_nblk; ++i) {
+    const int len = tb[i].y;
+#pragma unroll
+    for (int t = 0; t < QT; ++t)
+      if (acc < 128 * (t + 1) && acc + len > 128 * t) qm[t] |= 1u << i;
+    acc += len;
+  }
+}
+
 __device__ __forceinline__ void tma_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                          int h, int b, int s0, int s1) {
   tma_load_4d(dst, map, bar, 0, h, s0, b);
@@ -295,8 +327,8 @@ __device__ void rope_row_smem(uint8_t* q_tile, int r, int tok, const DevLayout& 
 // once, so no cross-item state is live).  PERSIST = true: each CTA walks items
 // blockIdx.x, blockIdx.x + gridDim.x, ... keeping TMEM and barriers alive, and
 // the next item's Q load and QK overlap the current item's epilogue.
-// ORDER: block-sparse mode, persistent CTAs walking the work items in the
-// order of pr.order (longest merged list first).
+// ORDER: block-sparse mode, persistent CTAs walking the work items listed in
+// pr.order (the items whose query group exists, in index order).
 template <int QT, int ST, bool PERSIST, bool ORDER>
 __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks)
     attn_tc_kernel(const __grid_constant__ AttnParams P) {
@@ -333,6 +365,8 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
       mbar_init(bar(B_KVEMPTY + s), 1);
     }
     mbar_init(bar(B_MMADONE), 1);
+    mbar_init(bar(B_EXPTOK), 128);
+    mbar_init(bar(B_EXPTOK + 1), 128);
     fence_mbar_init();
   }
   if (warp == C::kMmaWarp) {
@@ -420,13 +454,25 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
         auto v_slot = [&](int j) { return (cs + 2 * j + 1) % kStages; };
         auto ring_parity = [&](int i) { return ((cs + i) / kStages) & 1; };
         if (nkv > 0) {
+          // Sparse mode: a Q tile none of whose query blocks selected any key
+          // block of key tile j skips that tile's QK and PV (the barriers
+          // still complete, so both sides stay in phase); O_t is written by
+          // its first PV without accumulation.
+          uint32_t qm[QT];
+          if (ORDER) tile_blocks<QT>(pr, w, qm);
+          auto active = [&](uint32_t members, int t) { return !ORDER || (members & qm[t]) != 0u; };
+          bool o_init[QT];
+#pragma unroll
+          for (int t = 0; t < QT; ++t) o_init[t] = false;
+          uint32_t mem_j = ORDER ? tile_members(pr, w, 0) : ~0u;
           // prologue: S_t = Q_t K_0^T for every tile
           const int s_k0 = k_slot(0);
           if (!(ok = mbar_wait(bar(B_KVFULL + s_k0), ring_parity(0), err))) break;
           tc_fence_after();
 #pragma unroll
           for (int t = 0; t < QT; ++t) {
-            mma_qk(tmem + t * 128, sbase + kQOff + t * kTileBytes, sbase + kKVOff + s_k0 * kTileBytes);
+            if (active(mem_j, t))
+              mma_qk(tmem + t * 128, sbase + kQOff + t * kTileBytes, sbase + kKVOff + s_k0 * kTileBytes);
             tc_commit(bar(B_SFULL + t));
             if (nkv == 1) tc_commit(bar(B_QEMPTY + t));
           }
@@ -436,29 +482,36 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
             const uint32_t v_smem = sbase + kKVOff + sv * kTileBytes;
             const uint32_t k_smem = sbase + kKVOff + sk * kTileBytes;
             const bool more = j + 1 < nkv;
+            const uint32_t mem_next = (ORDER && more) ? tile_members(pr, w, j + 1) : ~0u;
             if (!(ok = mbar_wait(bar(B_KVFULL + sv), ring_parity(2 * j + 1), err))) break;
 #pragma unroll
             for (int t = 0; t < QT; ++t) {
+              const bool act = active(mem_j, t);
               if (!(ok = mbar_wait(bar(B_PHALF + t), (pt + j) & 1, err))) break;
               if (j == 0 && it > 0 && !(ok = mbar_wait(bar(B_OEMPTY + t), (it - 1) & 1, err)))
                 break;
               tc_fence_after();
-              mma_pv_part<0, 4>(tmem + QT * 128 + t * 128, tmem + t * 128, v_smem, j > 0);
+              if (act)
+                mma_pv_part<0, 4>(tmem + QT * 128 + t * 128, tmem + t * 128, v_smem, o_init[t]);
               if (!(ok = mbar_wait(bar(B_PFULL + t), (pt + j) & 1, err))) break;
               tc_fence_after();
-              mma_pv_part<4, 8>(tmem + QT * 128 + t * 128, tmem + t * 128, v_smem, true);
+              if (act) {
+                mma_pv_part<4, 8>(tmem + QT * 128 + t * 128, tmem + t * 128, v_smem, true);
+                o_init[t] = true;
+              }
               if (t == QT - 1) tc_commit(bar(B_KVEMPTY + sv));
               if (more) {
                 if (t == 0) {
                   if (!(ok = mbar_wait(bar(B_KVFULL + sk), ring_parity(2 * j + 2), err))) break;
                   tc_fence_after();
                 }
-                mma_qk(tmem + t * 128, sbase + kQOff + t * kTileBytes, k_smem);
+                if (active(mem_next, t)) mma_qk(tmem + t * 128, sbase + kQOff + t * kTileBytes, k_smem);
                 tc_commit(bar(B_SFULL + t));
                 if (j + 2 == nkv) tc_commit(bar(B_QEMPTY + t));
                 if (t == QT - 1) tc_commit(bar(B_KVEMPTY + sk));
               }
             }
+            mem_j = mem_next;
           }
           cs += 2 * nkv;
           pt += nkv;
@@ -485,6 +538,15 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
     const uint32_t o_addr = tmem + lane_off + QT * 128 + t * 128;
     const float sl2 = P.scale_log2;
     const float thresh = kRescaleLog2 / sl2;  // in raw score units
+    // Exponential turn of key tile number k (counted over all items) of this
+    // warpgroup: tile 0 waits for tile 1's (k-1)-th turn to end, tile 1 for
+    // tile 0's k-th (bounded waits: an error exit of one side ends the other).
+    auto exp_turn = [&](int k) -> bool {
+      if (t == 0 && k == 0) return true;
+      const uint32_t par = t == 0 ? (uint32_t)((k - 1) & 1) : (uint32_t)(k & 1);
+      const bool got = mbar_wait(bar(B_EXPTOK + t), par, err);
+      return !__any_sync(0xffffffffu, !got);
+    };
     const uint64_t sl2x2 = pack_f32x2(sl2, sl2);
     bool ok = !skip;
     int st = 0;  // S tiles consumed so far (all items)
@@ -520,6 +582,16 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
         }
         ucount = w.ucount;
       }
+      // sparse mode: the query blocks of this warpgroup's Q tile (a key tile
+      // none of them selected is skipped by the whole warpgroup, as by the
+      // MMA warp)
+      uint32_t tile_qm = ~0u;
+      if (ORDER) {
+        uint32_t qm[QT];
+        tile_blocks<QT>(pr, w, qm);
+        tile_qm = qm[t];
+      }
+      bool o_written = false;  // a PV of this item has written O_t
 
       float m_used = -INFINITY, l = 0.f;
       for (int j = 0; j < nkv; ++j, ++st) {
@@ -548,10 +620,35 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
             seg0 = seg1 = 0u;
           }
         }
+        bool tile_on = true;
+        if (ORDER) {
+          const uint4 f0 = pr.ulist[w.ubase + 2 * j];
+          uint32_t mm = f0.z | f0.w;
+          if (2 * j + 1 < ucount) {
+            const uint4 f1 = pr.ulist[w.ubase + 2 * j + 1];
+            mm |= f1.z | f1.w;
+          }
+          tile_on = (((mm | (mm >> 16)) & 0xFFFFu) & tile_qm) != 0u;
+        }
         ok = ok && mbar_wait(bar(B_SFULL + t), st & 1, err);
         if (__any_sync(0xffffffffu, !ok)) {
           ok = false;
           break;
+        }
+        if (!tile_on) {
+          // no QK was issued for this tile: release both P barriers at once
+          // and pass the exponential token on
+          tc_fence_before();
+          mbar_arrive(bar(B_PHALF + t));
+          mbar_arrive(bar(B_PFULL + t));
+          if (QT == 2) {
+            if (!exp_turn(st)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive(bar(B_EXPTOK + (t ^ 1)));
+          }
+          continue;
         }
         __syncwarp();
         tc_fence_after();
@@ -598,7 +695,7 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
           m_used = mt;
           l *= alpha;
         }
-        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        if (o_written && __any_sync(0xffffffffu, grow)) {
           // rescale the running O of this row (previous PV is complete: it was
           // issued before the QK whose completion released this S tile)
 #pragma unroll 1
@@ -614,6 +711,14 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
         }
         const float mref = (m_used == -INFINITY) ? 0.f : m_used * sl2;
         const uint64_t nm2 = pack_f32x2(-mref, -mref);
+        // The two softmax warpgroups take turns at the exponentials (tile 0's
+        // k-th key tile, tile 1's k-th, tile 0's (k+1)-th, ...), so that each
+        // runs with the SM's MUFU to itself while the tensor core works on
+        // the other Q tile, instead of both slowing each other down.
+        if (QT == 2 && !exp_turn(st)) {
+          ok = false;
+          break;
+        }
         // exponentials on the MUFU (ex2), arguments formed two at a time
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
@@ -637,6 +742,7 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
             mbar_arrive(bar(B_PHALF + t));
           }
         }
+        if (QT == 2) mbar_arrive(bar(B_EXPTOK + (t ^ 1)));  // the other tile's turn
         tmem_wait_st();
         {
           float a0, a1, b0, b1;
@@ -646,6 +752,7 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
         }
         tc_fence_before();
         mbar_arrive(bar(B_PFULL + t));
+        o_written = true;
       }
 
       // ---------------------------------------------------------- epilogue
@@ -663,7 +770,7 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
       // the MMA warp before any global store (the next item's first PV may
       // overwrite O while this warpgroup stores)
       uint32_t o0[32], o1[32], o2[32], o3[32];
-      if (nkv > 0) {
+      if (o_written) {
         tmem_ld32(o_addr, o0);
         tmem_ld32(o_addr + 32, o1);
         tmem_ld32(o_addr + 64, o2);

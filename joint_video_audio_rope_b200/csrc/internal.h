@@ -79,8 +79,8 @@ struct AttnProblem {
   int ctas;                   // work items: n_qtiles * H * B * n_splits
   int mode;                   // AttnMode
   // sparse mode: the query groups and the merged key lists (n_qtiles = the
-  // groups' capacity per batch item), the block table, and the order of the
-  // work items (ids (b H + h) n_qtiles + g, longest list first)
+  // groups' capacity per batch item), the block table, and the list of the
+  // work items that exist (ids (b H + h) n_qtiles + g, in index order)
   const int4* groups;         // [B][n_qtiles]: {first block, n blocks, start token, n tokens}
   const int* n_groups;        // [B]
   const uint4* ulist;         // [B][H][n_qtiles][ucap]: {start, len, seg masks 0|1, seg masks 2|3}
@@ -171,8 +171,8 @@ cudaError_t launch_union(const int32_t* idx, const int32_t* cnt, int cap, const 
                          const int* tab_n, int maxb, int N, const int4* groups,
                          const int* n_groups, int maxg, int B, int H, int ucap, uint4* ulist,
                          int* ucnt, int* err, cudaStream_t s);
-cudaError_t launch_schedule(const int* ucnt, const int* n_groups, int maxg, int B, int H,
-                            int ucap, int* order, int* n_order, cudaStream_t s);
+cudaError_t launch_schedule(const int* n_groups, int maxg, int B, int H, int* order,
+                            int* n_order, cudaStream_t s);
 
 // helpers (mmdit_api.cu)
 int* device_error_flag();  // device address of this device's error word

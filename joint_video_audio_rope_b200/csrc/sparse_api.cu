@@ -181,7 +181,7 @@ int run_sparse(const void* q, const void* k, const void* v, void* o, const mmdit
     e = launch_union(idx, cnt, cap, tab, tab_n, maxb, d.n_tokens, groups, n_groups, w.maxg,
                      d.batch, d.heads, w.ucap, ulist, ucnt, err, s);
   if (e == cudaSuccess)
-    e = launch_schedule(ucnt, n_groups, w.maxg, d.batch, d.heads, w.ucap, order, n_order, s);
+    e = launch_schedule(n_groups, w.maxg, d.batch, d.heads, order, n_order, s);
   if (e != cudaSuccess) return cuda_fail(e, "sparse_attn prep launch");
   int rc;
   AttnParams p{};

@@ -154,12 +154,16 @@ def test_plan_matches_oracle(M, with_audio):
 def test_plan_edge_cases(M):
     # a flat V (no variation anywhere) on a grid smaller than one zone: rho = 0
     # gives B = 256; g is isotropic, so the three shapes of that volume tie
-    # (the margin is 0 and any of them may win); the zone is one block
+    # (the margin is 0 and any of them may win); each of them cuts the
+    # 5 x 6 x 7 zone into two blocks (4 + 1 frames, 4 + 2 rows or 4 + 3 columns)
     w = WL.Workload("flat", [WL.video(5, 6, 7)], 1, 2, 128, "bf16", 1, 1.0, 1.0)
     vb = np.full((1, 5 * 6 * 7, 2, 128), WL.f32_to_bf16_bits(np.float32(0.5)), np.uint16)
     zones_g, blocks_g, nblk_g, mb = _plan_gpu(M, w, vb, None)
-    assert zones_g.shape[1] == 1 and zones_g[0, 0, 0] in (13, 14, 15) and nblk_g[0] == 1
-    assert tuple(blocks_g[0, 0]) == (0, 210) and tuple(zones_g[0, 0, 1:]) == (0, 0, 1)
+    assert zones_g.shape[1] == 1 and zones_g[0, 0, 0] in (13, 14, 15) and nblk_g[0] == 2
+    assert tuple(zones_g[0, 0, 1:]) == (0, 0, 2)
+    shape = SHAPES[zones_g[0, 0, 0]]
+    first = min(shape[0], 5) * min(shape[1], 6) * min(shape[2], 7)
+    assert tuple(blocks_g[0, 0]) == (0, first) and tuple(blocks_g[0, 1]) == (first, 210 - first)
     # one zone varying strongly along t and weakly along h (no tie): B = 64
     # (rho = 1) and the oracle's shape, exactly
     t = np.arange(5, dtype=np.float32)[:, None, None]
