@@ -97,9 +97,7 @@ enum {
   B_OEMPTY = 20,  // 2: epilogue has read O out of TMEM (128 arrivals)
   B_MMADONE = 22, // 1: every MMA of the CTA done (teardown)
   B_PHALF = 23,   // 2: first 64 keys of the P tile written (128 arrivals)
-  B_EXPTOK = 25,  // 2: the other softmax warpgroup has finished its exponentials
-                  //    of its latest key tile (128 arrivals; two Q tiles only)
-  B_COUNT = 27
+  B_COUNT = 25
 };
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0, 0);  // Q, K: K-major
@@ -344,6 +342,10 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
   const uint32_t bars = sbase + kBarOff;
   auto bar = [&](int i) { return bars + 8u * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + 8 * B_COUNT);
+  // sparse mode: per K/V ring slot, the query blocks that selected any key
+  // block of the key tile loaded there (written by the producer before the
+  // slot's TMA, read by the MMA warp after the slot's barrier completes)
+  volatile uint32_t* slot_members = reinterpret_cast<volatile uint32_t*>(smem + kBarOff + 8 * B_COUNT + 16);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* err = P.err;
@@ -365,8 +367,6 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
       mbar_init(bar(B_KVEMPTY + s), 1);
     }
     mbar_init(bar(B_MMADONE), 1);
-    mbar_init(bar(B_EXPTOK), 128);
-    mbar_init(bar(B_EXPTOK + 1), 128);
     fence_mbar_init();
   }
   if (warp == C::kMmaWarp) {
@@ -414,6 +414,7 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
           for (int kind = 0; kind < 2; ++kind, ++ld) {
             const int slot = ld % kStages;
             if (!(ok = mbar_wait(bar(B_KVEMPTY + slot), ((ld / kStages) & 1) ^ 1, err))) break;
+            if (ORDER && kind == 0) slot_members[slot] = tile_members(pr, w, j);
             mbar_expect_tx(bar(B_KVFULL + slot), kTileBytes);
             tma_tile(sbase + kKVOff + slot * kTileBytes, kind ? &pr.tmV : &pr.tmK,
                      bar(B_KVFULL + slot), w.h, w.b, s0, s1);
@@ -464,11 +465,11 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
           bool o_init[QT];
 #pragma unroll
           for (int t = 0; t < QT; ++t) o_init[t] = false;
-          uint32_t mem_j = ORDER ? tile_members(pr, w, 0) : ~0u;
           // prologue: S_t = Q_t K_0^T for every tile
           const int s_k0 = k_slot(0);
           if (!(ok = mbar_wait(bar(B_KVFULL + s_k0), ring_parity(0), err))) break;
           tc_fence_after();
+          uint32_t mem_j = ORDER ? slot_members[s_k0] : ~0u;
 #pragma unroll
           for (int t = 0; t < QT; ++t) {
             if (active(mem_j, t))
@@ -482,7 +483,7 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
             const uint32_t v_smem = sbase + kKVOff + sv * kTileBytes;
             const uint32_t k_smem = sbase + kKVOff + sk * kTileBytes;
             const bool more = j + 1 < nkv;
-            const uint32_t mem_next = (ORDER && more) ? tile_members(pr, w, j + 1) : ~0u;
+            uint32_t mem_next = ~0u;
             if (!(ok = mbar_wait(bar(B_KVFULL + sv), ring_parity(2 * j + 1), err))) break;
 #pragma unroll
             for (int t = 0; t < QT; ++t) {
@@ -504,6 +505,7 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
                 if (t == 0) {
                   if (!(ok = mbar_wait(bar(B_KVFULL + sk), ring_parity(2 * j + 2), err))) break;
                   tc_fence_after();
+                  if (ORDER) mem_next = slot_members[sk];
                 }
                 if (active(mem_next, t)) mma_qk(tmem + t * 128, sbase + kQOff + t * kTileBytes, k_smem);
                 tc_commit(bar(B_SFULL + t));
@@ -538,15 +540,7 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
     const uint32_t o_addr = tmem + lane_off + QT * 128 + t * 128;
     const float sl2 = P.scale_log2;
     const float thresh = kRescaleLog2 / sl2;  // in raw score units
-    // Exponential turn of key tile number k (counted over all items) of this
-    // warpgroup: tile 0 waits for tile 1's (k-1)-th turn to end, tile 1 for
-    // tile 0's k-th (bounded waits: an error exit of one side ends the other).
-    auto exp_turn = [&](int k) -> bool {
-      if (t == 0 && k == 0) return true;
-      const uint32_t par = t == 0 ? (uint32_t)((k - 1) & 1) : (uint32_t)(k & 1);
-      const bool got = mbar_wait(bar(B_EXPTOK + t), par, err);
-      return !__any_sync(0xffffffffu, !got);
-    };
+
     const uint64_t sl2x2 = pack_f32x2(sl2, sl2);
     bool ok = !skip;
     int st = 0;  // S tiles consumed so far (all items)
@@ -637,17 +631,9 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
         }
         if (!tile_on) {
           // no QK was issued for this tile: release both P barriers at once
-          // and pass the exponential token on
           tc_fence_before();
           mbar_arrive(bar(B_PHALF + t));
           mbar_arrive(bar(B_PFULL + t));
-          if (QT == 2) {
-            if (!exp_turn(st)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive(bar(B_EXPTOK + (t ^ 1)));
-          }
           continue;
         }
         __syncwarp();
@@ -711,14 +697,6 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
         }
         const float mref = (m_used == -INFINITY) ? 0.f : m_used * sl2;
         const uint64_t nm2 = pack_f32x2(-mref, -mref);
-        // The two softmax warpgroups take turns at the exponentials (tile 0's
-        // k-th key tile, tile 1's k-th, tile 0's (k+1)-th, ...), so that each
-        // runs with the SM's MUFU to itself while the tensor core works on
-        // the other Q tile, instead of both slowing each other down.
-        if (QT == 2 && !exp_turn(st)) {
-          ok = false;
-          break;
-        }
         // exponentials on the MUFU (ex2), arguments formed two at a time
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
@@ -742,7 +720,6 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
             mbar_arrive(bar(B_PHALF + t));
           }
         }
-        if (QT == 2) mbar_arrive(bar(B_EXPTOK + (t ^ 1)));  // the other tile's turn
         tmem_wait_st();
         {
           float a0, a1, b0, b1;
@@ -988,9 +965,11 @@ int attn_rows_per_cta(int q_tiles) { return 128 * q_tiles; }
 
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
   if (p.prob.order != nullptr) {
-    // an item order is walked by persistent CTAs (block-sparse attention)
-    if (p.q_tiles != 2 || !p.persistent) return cudaErrorInvalidValue;
-    return launch_shape<2, 4, true, true>(p, s);
+    // block-sparse attention over a list of work items: one CTA per listed
+    // item (grid = the list's capacity; CTAs past its length exit at once),
+    // or persistent CTAs walking the list
+    if (p.q_tiles != 2) return cudaErrorInvalidValue;
+    return p.persistent ? launch_shape<2, 4, true, true>(p, s) : launch_shape<2, 4, false, true>(p, s);
   }
   if (p.q_tiles == 1)  // one-tile CTAs are always persistent (short key sequences)
     return p.persistent ? launch_shape<1, 2, true>(p, s) : cudaErrorInvalidValue;

@@ -211,7 +211,7 @@ int run_sparse(const void* q, const void* k, const void* v, void* o, const mmdit
   pr.order = order;
   pr.n_order = n_order;
   p.q_tiles = kSparseQTiles;
-  p.persistent = 1;
+  p.persistent = 0;  // one CTA per listed item: the hardware balances the ragged lists
   p.scale_log2 = scale * 1.4426950408889634f;
   p.err = err;
   e = launch_attn_tc(p, s);
