@@ -45,7 +45,7 @@ constexpr int kOffK = 0;
 constexpr int kOffV = kOffK + kKVBytes;
 constexpr int kOffQ = kOffV + kKVBytes;
 constexpr int kOffStage = kOffQ + 2 * kQTileBytes;
-constexpr int kOffBar = kOffStage + 8 * kStageWarp;
+constexpr int kOffBar = kOffStage + 2 * 8 * kStageWarp;  // two staging buffers per warp
 constexpr int kSkSmem = kOffBar + 256 + 1024;
 // registers: launched at 168 per thread (384 x 168 = 64,512); the producer /
 // MMA warpgroup drops to 104 and the softmax warpgroups rise to 200
@@ -316,11 +316,13 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_short_kernel(const __grid_
       }
       const int wrow = row0 + (warp & 3) * 32;  // first row of this warp
       if (wrow < pr.Nq) {
-        uint8_t* stg = smem + kOffStage + warp * kStageWarp;
         const int sw = ((lane * kStageColsS * 2) >> 7) & 3;  // 64-byte swizzle of this lane's row
 #pragma unroll
         for (int rr = 0; rr < 128 / kStageColsS; ++rr) {
-          if (lane == 0) bulk_wait_read<0>();
+          // two staging buffers per warp: a round waits only for the store
+          // issued two rounds ago to have read its buffer
+          uint8_t* stg = smem + kOffStage + (2 * warp + (rr & 1)) * kStageWarp;
+          if (lane == 0) bulk_wait_read<1>();
           __syncwarp();
 #pragma unroll
           for (int chunk = 0; chunk < 4; ++chunk) {

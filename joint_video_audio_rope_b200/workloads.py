@@ -135,6 +135,12 @@ WORKLOADS: Dict[str, Workload] = {
         batch=1, heads=24, head_dim=128, dtype="bf16", seed=6,
         qk_std=1.0, v_std=1.0, planted_regions=8, planted_amp=2.0, sparse=True,
         plant_v=True, adaptive=True),
+    # the adaptive layer on a quarter of the 1080p grid (profiling size)
+    "1080p_adaptive_quarter": Workload(
+        "1080p_adaptive_quarter", [video(21, 34, 60), audio(218)],
+        batch=1, heads=24, head_dim=128, dtype="bf16", seed=7,
+        qk_std=1.0, v_std=1.0, planted_regions=8, planted_amp=2.0, sparse=True,
+        plant_v=True, adaptive=True),
     # a quarter of the 1080p grid (17 x 30 -> 17 x 15 blocks per frame slab):
     # the same structure at a size an ncu capture can hold (~2 GB on device)
     "1080p_sparse_quarter": Workload(
