@@ -169,45 +169,73 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_short_kernel(const __grid_
       if (kv_loads > 0) mbar_wait(bar(SB_KVFULL), (kv_loads - 1) & 1, err);
     } else if (warp == kSkMmaWarp && lane == 0 && !skip) {
       // ---------------------------------------------------------- MMA issuer
+      // Issue order QK_0(n), PV_1(n-1), QK_1(n), PV_0(n), QK_0(n+1), ...: the
+      // two tiles run half a period apart, so each softmax overlaps the other
+      // tile's PV, epilogue read and QK instead of the other softmax (they
+      // would share the MUFU).  QK_t(n) waits for its Q and for the epilogue
+      // of item n-1 to have read O_t out (S_t and O_t share TMEM columns).
       bool ok = true;
-      int cur_bh = -1, kv_loads = 0, n = 0;
-      for (int it = first; it < last && ok; ++it, ++n) {
-        const ShortWork w = short_item(it, pairs, pr.H);
-        const int bh = w.b * pr.H + w.h;
-        if (bh != cur_bh) {
-          if (kv_loads > 0) tc_commit(bar(SB_KVEMPTY));  // after every MMA of the old head
-          if (!(ok = mbar_wait(bar(SB_KVFULL), kv_loads & 1, err))) break;
-          cur_bh = bh;
-          ++kv_loads;
-        }
-        for (int t = 0; t < 2 && ok; ++t) {
-          const uint32_t s_tmem = tmem + 256 * t;
-          if (!(ok = mbar_wait(bar(SB_QFULL + t), n & 1, err))) break;
-          // S and O of this tile are free once the last item's epilogue read O
-          if (n > 0 && !(ok = mbar_wait(bar(SB_OEMPTY + t), (n - 1) & 1, err))) break;
-          tc_fence_after();
-          const uint32_t q = sbase + kOffQ + t * kQTileBytes;
+      int cur_bh = -1, kv_loads = 0;
+      const int n_items = last - first;
+      auto issue_qk = [&](int t, int n) -> bool {
+        if (!mbar_wait(bar(SB_QFULL + t), n & 1, err)) return false;
+        if (n > 0 && !mbar_wait(bar(SB_OEMPTY + t), (n - 1) & 1, err)) return false;
+        tc_fence_after();
+        const uint32_t q = sbase + kOffQ + t * kQTileBytes;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t qo = (kk >> 2) * kQHalf + (kk & 3) * 32;
-            const uint32_t ko = (kk >> 2) * kKVHalf + (kk & 3) * 32;
-            tc_mma_ss(s_tmem, smem_desc_sw128(q + qo, 16, 1024),
-                      smem_desc_sw128(sbase + kOffK + ko, 16, 1024), kIdescS, kk > 0);
-          }
-          tc_commit(bar(SB_SFULL + t));
-          tc_commit(bar(SB_QEMPTY + t));
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t qo = (kk >> 2) * kQHalf + (kk & 3) * 32;
+          const uint32_t ko = (kk >> 2) * kKVHalf + (kk & 3) * 32;
+          tc_mma_ss(tmem + 256 * t, smem_desc_sw128(q + qo, 16, 1024),
+                    smem_desc_sw128(sbase + kOffK + ko, 16, 1024), kIdescS, kk > 0);
         }
-        for (int t = 0; t < 2 && ok; ++t) {
-          const uint32_t s_tmem = tmem + 256 * t;
-          if (!(ok = mbar_wait(bar(SB_PFULL + t), n & 1, err))) break;
-          tc_fence_after();
-          for (int kk = 0; kk < n_ksteps; ++kk)
-            tc_mma_ts(s_tmem + 128, s_tmem + kk * 8,
-                      smem_desc_sw128(sbase + kOffV + kk * 2048, kKVHalf, 1024), kIdescO,
-                      kk > 0 ? 1u : 0u);
-          tc_commit(bar(SB_OFULL + t));
+        tc_commit(bar(SB_SFULL + t));
+        tc_commit(bar(SB_QEMPTY + t));
+        return true;
+      };
+      auto issue_pv = [&](int t, int n) -> bool {
+        if (!mbar_wait(bar(SB_PFULL + t), n & 1, err)) return false;
+        tc_fence_after();
+        const uint32_t s_tmem = tmem + 256 * t;
+        for (int kk = 0; kk < n_ksteps; ++kk)
+          tc_mma_ts(s_tmem + 128, s_tmem + kk * 8,
+                    smem_desc_sw128(sbase + kOffV + kk * 2048, kKVHalf, 1024), kIdescO,
+                    kk > 0 ? 1u : 0u);
+        tc_commit(bar(SB_OFULL + t));
+        return true;
+      };
+      // K/V of item n resident: when the head changes, every MMA issued so far
+      // (all of the old head's) completes before the producer reloads K/V
+      auto ensure_kv = [&](int n) -> bool {
+        const ShortWork w = short_item(first + n, pairs, pr.H);
+        const int bh = w.b * pr.H + w.h;
+        if (bh == cur_bh) return true;
+        if (kv_loads > 0) tc_commit(bar(SB_KVEMPTY));
+        if (!mbar_wait(bar(SB_KVFULL), kv_loads & 1, err)) return false;
+        cur_bh = bh;
+        ++kv_loads;
+        return true;
+      };
+      bool pv1_pending = false;  // PV_1 of the previous item not issued yet
+      if (n_items > 0) ok = ensure_kv(0) && issue_qk(0, 0);
+      for (int n = 0; n < n_items && ok; ++n) {
+        if (pv1_pending) {
+          if (!(ok = issue_pv(1, n - 1))) break;
+          pv1_pending = false;
+        }
+        if (!(ok = issue_qk(1, n))) break;
+        if (!(ok = issue_pv(0, n))) break;
+        pv1_pending = true;
+        if (n + 1 < n_items) {
+          const ShortWork wn = short_item(first + n + 1, pairs, pr.H);
+          if (wn.b * pr.H + wn.h != cur_bh) {  // the old K/V is still read by PV_1(n)
+            if (!(ok = issue_pv(1, n))) break;
+            pv1_pending = false;
+          }
+          if (!(ok = ensure_kv(n + 1) && issue_qk(0, n + 1))) break;
         }
       }
+      if (ok && pv1_pending) issue_pv(1, n_items - 1);
       tc_commit(bar(SB_DONE));
       mbar_wait(bar(SB_DONE), 0, err);
     }

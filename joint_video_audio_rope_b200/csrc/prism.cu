@@ -21,10 +21,11 @@
 // tokens in (t, h, w) raster order, so every block is one contiguous run.
 //
 // Kernels:
-//   zone_stats_kernel  one warp per (zone, head, batch): slice sums of its
-//                      head's 128 channels along t, h and w (fp32, lane =
-//                      4 channels) and the three centred variance sums; the
-//                      head-0 warp also takes the statistics of the norms a.
+//   zone_stats_kernel  one CTA per (zone, head, batch), one warp per t-slice:
+//                      slice sums of the head's 128 channels along t, h and w
+//                      (fp32, lane = 4 channels) and the three centred
+//                      variance sums; the head-0 CTA also takes the
+//                      statistics of the norms a.
 //   zone_plan_kernel   one CTA per batch item: the indicator, volume and shape
 //                      of every zone in fp64, the zone and block prefix sums,
 //                      the block table and the zone table.
@@ -91,38 +92,75 @@ __device__ __forceinline__ float centred(const float (&s)[NMAX], int n, float cn
   return v;
 }
 
+// Centred variance sum of `n` means m_i:  sum_i (m_i - mu)^2, mu = mean of m_i.
+template <int NMAX>
+__device__ __forceinline__ float centred_means(const float (&m)[NMAX], int n) {
+  float mu = 0.f;
+#pragma unroll
+  for (int i = 0; i < NMAX; ++i) mu += i < n ? m[i] : 0.f;
+  mu /= (float)n;
+  float v = 0.f;
+#pragma unroll
+  for (int i = 0; i < NMAX; ++i) {
+    const float d = m[i] - mu;
+    v += i < n ? d * d : 0.f;
+  }
+  return v;
+}
+
 // part[b][z][h][3] = sum over the head's channels of (1/Z_d) sum_i (slice mean
 // - mean)^2 along t, h, w;  ast[b][z][4] = the same three for the norms a (a
 // single channel) and the zone mean of a (zeros when a is NULL).
-__global__ void __launch_bounds__(128) zone_stats_kernel(
+// One CTA per (zone, head, batch), one warp per t-slice of the zone (lane =
+// 4 channels): each warp sums its slice, its slice's rows (h) and columns
+// (w); warp 0 combines the warps' partial h and w sums from shared memory.
+constexpr int kStatsThreads = 32 * kZone;
+constexpr int kStatsSmem = (int)sizeof(float) * (kZone * 128 + 2 * kZone * kZone * 128);
+
+__global__ void __launch_bounds__(kStatsThreads, 2) zone_stats_kernel(
     const __nv_bfloat16* __restrict__ v, long long st, long long sb, int heads, ZoneGrid zg,
     const float* __restrict__ a, float* __restrict__ part, float* __restrict__ ast) {
-  __shared__ float s_t[4][kZone][128];  // per warp: slice sums along t
+  extern __shared__ float s_dyn[];
+  float(*s_t)[128] = reinterpret_cast<float(*)[128]>(s_dyn);                  // [t] slice sums
+  float(*s_h)[kZone][128] = reinterpret_cast<float(*)[kZone][128]>(s_dyn + kZone * 128);  // [warp][h]
+  float(*s_w)[kZone][128] =
+      reinterpret_cast<float(*)[kZone][128]>(s_dyn + kZone * 128 + kZone * kZone * 128);  // [warp][w]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int z = blockIdx.x, b = blockIdx.z;
-  const int h = blockIdx.y * 4 + warp;
+  // heads are the fastest grid dimension: the CTAs of one zone run side by
+  // side and read whole token rows (every head's 256 bytes) together
+  const int h = blockIdx.x, z = blockIdx.y, b = blockIdx.z;
   const int nz = zg.count();
-  if (h >= heads) return;
   int t0, h0, w0, et, eh, ew;
   zg.zone(z, t0, h0, w0, et, eh, ew);
-  float sh[kZone][4], sw[kZone][4];
+  const int lt = warp;  // this warp's t-slice
+  float sh[kZone][4], sw[kZone][4], stt[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int i = 0; i < kZone; ++i)
 #pragma unroll
     for (int c = 0; c < 4; ++c) sh[i][c] = sw[i][c] = 0.f;
-  const __nv_bfloat16* base = v + (long long)b * sb + (long long)h * 128 + 4 * lane;
-  for (int lt = 0; lt < et; ++lt) {
-    float stt[4] = {0.f, 0.f, 0.f, 0.f};
+  if (lt < et) {
+    const __nv_bfloat16* base = v + (long long)b * sb + (long long)h * 128 + 4 * lane;
+    // the slice's 8 x 8 tokens in two halves of four rows (32 loads in flight)
 #pragma unroll
-    for (int lh = 0; lh < kZone; ++lh) {
-      if (lh >= eh) break;
-      const long long row = ((long long)(t0 + lt) * zg.H + (h0 + lh)) * zg.W + w0;
+    for (int half = 0; half < 2; ++half) {
+      uint2 raw[kZone / 2][kZone];
 #pragma unroll
-      for (int lw = 0; lw < kZone; ++lw) {
-        if (lw < ew) {
-          const uint2 raw = __ldg(reinterpret_cast<const uint2*>(base + (row + lw) * st));
-          const float2 x01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
-          const float2 x23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+      for (int i = 0; i < kZone / 2; ++i) {
+        const int lh = half * (kZone / 2) + i;
+        const long long row = ((long long)(t0 + lt) * zg.H + (h0 + lh)) * zg.W + w0;
+#pragma unroll
+        for (int lw = 0; lw < kZone; ++lw)
+          raw[i][lw] = (lh < eh && lw < ew)
+                           ? __ldg(reinterpret_cast<const uint2*>(base + (row + lw) * st))
+                           : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int i = 0; i < kZone / 2; ++i) {
+        const int lh = half * (kZone / 2) + i;
+#pragma unroll
+        for (int lw = 0; lw < kZone; ++lw) {
+          const float2 x01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[i][lw].x));
+          const float2 x23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[i][lw].y));
           const float x[4] = {x01.x, x01.y, x23.x, x23.y};
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -133,47 +171,84 @@ __global__ void __launch_bounds__(128) zone_stats_kernel(
         }
       }
     }
-#pragma unroll
-    for (int c = 0; c < 4; ++c) s_t[warp][lt][4 * lane + c] = stt[c];
   }
-  __syncwarp();
-  float vt = 0.f, vh = 0.f, vw = 0.f;
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
-    float st8[kZone], sh8[kZone], sw8[kZone];
+    s_t[lt][4 * lane + c] = stt[c];
 #pragma unroll
     for (int i = 0; i < kZone; ++i) {
-      st8[i] = i < et ? s_t[warp][i][4 * lane + c] : 0.f;
-      sh8[i] = sh[i][c];
-      sw8[i] = sw[i][c];
+      s_h[lt][i][4 * lane + c] = sh[i][c];
+      s_w[lt][i][4 * lane + c] = sw[i][c];
     }
-    vt += centred(st8, et, (float)(eh * ew)) / (float)et;
-    vh += centred(sh8, eh, (float)(et * ew)) / (float)eh;
-    vw += centred(sw8, ew, (float)(et * eh)) / (float)ew;
   }
-  vt = warp_sum_f(vt);
-  vh = warp_sum_f(vh);
-  vw = warp_sum_f(vw);
-  if (lane == 0) {
-    float* o = part + (((long long)b * nz + z) * heads + h) * 3;
-    o[0] = vt;
-    o[1] = vh;
-    o[2] = vw;
+  __syncthreads();
+  // the centred variance sums, one channel per thread: threads 0-127 take the
+  // t and h axes of channel tid, threads 128-255 the w axis of channel tid-128
+  // (slice means as sums times the reciprocal of the slice's token count)
+  {
+    const int c = threadIdx.x & 127, part_id = threadIdx.x >> 7;
+    float m8[kZone], va = 0.f, vb = 0.f;
+    if (part_id == 0) {
+      const float it = 1.f / (float)(eh * ew), ih = 1.f / (float)(et * ew);
+#pragma unroll
+      for (int i = 0; i < kZone; ++i) m8[i] = s_t[i][c] * it;
+      va = centred_means(m8, et) / (float)et;
+#pragma unroll
+      for (int i = 0; i < kZone; ++i) {
+        float hs = 0.f;
+#pragma unroll
+        for (int k = 0; k < kZone; ++k) hs += s_h[k][i][c];  // over the t-slices, in order
+        m8[i] = hs * ih;
+      }
+      vb = centred_means(m8, eh) / (float)eh;
+    } else {
+      const float iw = 1.f / (float)(et * eh);
+#pragma unroll
+      for (int i = 0; i < kZone; ++i) {
+        float ws = 0.f;
+#pragma unroll
+        for (int k = 0; k < kZone; ++k) ws += s_w[k][i][c];
+        m8[i] = ws * iw;
+      }
+      va = centred_means(m8, ew) / (float)ew;
+    }
+    // sums over the head's 128 channels: warps, then the four warps of a part
+    va = warp_sum_f(va);
+    vb = warp_sum_f(vb);
+    __shared__ float s_red[kZone][2];
+    if (lane == 0) {
+      s_red[warp][0] = va;
+      s_red[warp][1] = vb;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float vt = 0.f, vh = 0.f, vw = 0.f;
+      for (int w_ = 0; w_ < 4; ++w_) {
+        vt += s_red[w_][0];
+        vh += s_red[w_][1];
+        vw += s_red[4 + w_][0];
+      }
+      float* o = part + (((long long)b * nz + z) * heads + h) * 3;
+      o[0] = vt;
+      o[1] = vh;
+      o[2] = vw;
+    }
   }
-  if (h != 0) return;
-  // statistics of the norms a of this zone: lane l takes the tokens l, l+32, ...
+  if (h != 0 || warp != 1) return;
+  // statistics of the norms a of this zone (warp 1 of the head-0 CTA): lane l
+  // takes the tokens l, l+32, ...
   float at[kZone], ah[kZone], aw[kZone], asum = 0.f;
 #pragma unroll
   for (int i = 0; i < kZone; ++i) at[i] = ah[i] = aw[i] = 0.f;
   if (a != nullptr) {
     const int n = et * eh * ew;
     for (int i = lane; i < n; i += 32) {
-      const int lt = i / (eh * ew), r = i - lt * eh * ew, lh = r / ew, lw = r - lh * ew;
+      const int lt2 = i / (eh * ew), r = i - lt2 * eh * ew, lh = r / ew, lw = r - lh * ew;
       const float x = a[(long long)b * zg.T * zg.H * zg.W +
-                        ((long long)(t0 + lt) * zg.H + (h0 + lh)) * zg.W + (w0 + lw)];
+                        ((long long)(t0 + lt2) * zg.H + (h0 + lh)) * zg.W + (w0 + lw)];
 #pragma unroll
       for (int k = 0; k < kZone; ++k) {
-        at[k] += k == lt ? x : 0.f;
+        at[k] += k == lt2 ? x : 0.f;
         ah[k] += k == lh ? x : 0.f;
         aw[k] += k == lw ? x : 0.f;
       }
@@ -473,7 +548,15 @@ int mmdit_adaptive_plan(const void* v, const float* a_norm, const mmdit_tensor_d
   float* ast = reinterpret_cast<float*>(ws + w.ast);
   const ZoneGrid zg = zone_grid(T, H, W);
   cudaStream_t s = (cudaStream_t)stream;
-  zone_stats_kernel<<<dim3(nz, (desc->heads + 3) / 4, desc->batch), 128, 0, s>>>(
+  int dev = 0;
+  cudaError_t e0 = cudaGetDevice(&dev);
+  if (e0 == cudaSuccess)
+    e0 = once_per_device(dev, [] {
+      return cudaFuncSetAttribute(zone_stats_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  kStatsSmem);
+    });
+  if (e0 != cudaSuccess) return cuda_fail(e0, "adaptive_plan attribute");
+  zone_stats_kernel<<<dim3(desc->heads, nz, desc->batch), kStatsThreads, kStatsSmem, s>>>(
       (const __nv_bfloat16*)v, desc->stride_tok, desc->stride_batch, desc->heads, zg, a_norm,
       part, ast);
   cudaError_t e = cudaGetLastError();
