@@ -108,7 +108,8 @@ PER_CONFIG = ("480p", "720p", "720p_cond_b2", "1080p_sparse", "1080p_adaptive")
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only while the kernel
 # source is the one that was captured (sha1 of attn_tc.cu + common.cuh).
 NCU_TRAFFIC = {
-    "480p": {"src": "5ac8cc44391153b7", "bytes": 833501184},  # ncu, one joint launch
+    # ncu, one joint launch of the 720p_cond_b2 layer (1-pass DRAM counters)
+    "720p_cond_b2": {"src": "ca86e84634dcce29", "bytes": 5772729000},
 }
 
 
