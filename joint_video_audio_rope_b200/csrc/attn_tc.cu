@@ -5,17 +5,22 @@
 // the layer:
 //   * joint self-attention over the concatenated sequence (SkyReels-V4 digest,
 //     arXiv 2602.21818, workflow step 3; SkyReels-V4 blog, section 2.1);
-//   * both directions of the audio<->video cross-attention (same sources;
-//     blog section 2.2), the audio-query direction with the video keys split
-//     across CTAs and merged afterwards (split-KV);
+//   * the audio-query direction of the audio<->video cross-attention (same
+//     sources; blog section 2.2), the video keys split across CTAs and merged
+//     afterwards (split-KV); the video-query direction, over at most 256
+//     audio keys, has its own kernel (attn_short.cu);
+//   * the reinforced text cross-attention (video queries over the text keys,
+//     one-tile CTAs, two per SM);
 //   * block-sparse attention restricted to selected key blocks (Prism guide,
 //     arXiv 2610.05416, Method section 3: online-softmax attention over S_i).
 //
-// CTA organisation (320 threads, one CTA per SM):
+// CTA organisation (384 threads = 3 warpgroups, one CTA per SM, for two Q
+// tiles; the one-tile shape has 256 threads and two CTAs per SM):
 //   warps 0-3  softmax warpgroup for Q tile 0 (128 query rows; thread = row)
 //   warps 4-7  softmax warpgroup for Q tile 1
 //   warp 8     TMA producer: Q tiles once, then K/V tiles into a 4-slot ring
 //   warp 9     tensor-memory allocator and single-thread tcgen05.mma issuer
+//   warps 10-11 no role (setmaxnreg hands registers out per warpgroup)
 // Tensor memory (512 columns x 128 lanes of 32 bit):
 //   [0,128) S0 / P0   [128,256) S1 / P1   [256,384) O0   [384,512) O1
 // S = Q K^T lands in TMEM; the softmax warps read it (tcgen05.ld), write the
@@ -325,7 +330,7 @@ __device__ void rope_row_smem(uint8_t* q_tile, int r, int tok, const DevLayout& 
 // once, so no cross-item state is live).  PERSIST = true: each CTA walks items
 // blockIdx.x, blockIdx.x + gridDim.x, ... keeping TMEM and barriers alive, and
 // the next item's Q load and QK overlap the current item's epilogue.
-// ORDER: block-sparse mode, persistent CTAs walking the work items listed in
+// ORDER: block-sparse mode, CTA i taking the i-th work item listed in
 // pr.order (the items whose query group exists, in index order).
 template <int QT, int ST, bool PERSIST, bool ORDER>
 __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks)
@@ -966,10 +971,9 @@ int attn_rows_per_cta(int q_tiles) { return 128 * q_tiles; }
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
   if (p.prob.order != nullptr) {
     // block-sparse attention over a list of work items: one CTA per listed
-    // item (grid = the list's capacity; CTAs past its length exit at once),
-    // or persistent CTAs walking the list
-    if (p.q_tiles != 2) return cudaErrorInvalidValue;
-    return p.persistent ? launch_shape<2, 4, true, true>(p, s) : launch_shape<2, 4, false, true>(p, s);
+    // item (grid = the list's capacity; CTAs past its length exit at once)
+    if (p.q_tiles != 2 || p.persistent) return cudaErrorInvalidValue;
+    return launch_shape<2, 4, false, true>(p, s);
   }
   if (p.q_tiles == 1)  // one-tile CTAs are always persistent (short key sequences)
     return p.persistent ? launch_shape<1, 2, true>(p, s) : cudaErrorInvalidValue;

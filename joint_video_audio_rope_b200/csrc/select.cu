@@ -41,8 +41,8 @@
 //                      attention kernel walks the list two entries per key
 //                      tile.
 //   schedule_kernel    lists the (group, head, batch) items whose group
-//                      exists, in index order, for the persistent attention
-//                      launch.
+//                      exists, in index order, for the sparse attention
+//                      launch (CTA i takes the i-th listed item).
 #include <math.h>
 
 #include "internal.h"
@@ -536,8 +536,8 @@ __global__ void __launch_bounds__(256) union_kernel(
 
 constexpr int kSchedThreads = 1024;
 
-// The work items of the persistent sparse attention: every (group, head,
-// batch) item whose group exists, in index order (batch, head, group) --
+// The work items of the sparse attention: every (group, head, batch) item
+// whose group exists, in index order (batch, head, group) --
 // consecutive items are neighbouring query groups of one head, which select
 // largely the same key blocks, so the CTAs running side by side share their
 // K/V tiles through L2.  (Ordering by list length, longest first, measured
