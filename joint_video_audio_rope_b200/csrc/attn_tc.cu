@@ -347,6 +347,14 @@ __global__ void __launch_bounds__(Cfg<QT, ST>::kThreads, Cfg<QT, ST>::kMinBlocks
   constexpr int kStages = C::kStages;
   constexpr bool kPaired = C::kPairable && !PERSIST;
   constexpr int kUnits = kPaired ? ST / 2 : ST;  // ring units (barrier pairs)
+  if (!PERSIST) {
+    // a one-item CTA with nothing to compute or write (past the ordered
+    // list, or past its batch item's valid query rows: the masked attention
+    // sizes its grid for every video row) leaves before any set-up
+    const ItemWalk<PERSIST, ORDER> w0(P.prob);
+    if (!w0.more(P.prob)) return;
+    if (!ORDER && decode_work<false>(P, w0.cur, C::kRows).q_valid <= 0) return;
+  }
   constexpr int kQOff = C::kQOff;
   constexpr int kKVOff = C::kKVOff;
   constexpr int kBarOff = C::kBarOff;

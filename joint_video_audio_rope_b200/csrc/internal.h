@@ -61,8 +61,8 @@ struct F32AttnArgs {
 };
 cudaError_t launch_attn_f32(const F32AttnArgs& a, cudaStream_t s);
 
-// tcgen05 bf16 attention (attn_tc.cu)
-enum AttnMode { kModeDense = 0, kModeSparse = 1 };
+// tcgen05 bf16 attention (attn_tc.cu); the dense or block-sparse mode is a
+// template parameter of the kernel, chosen by whether `order` is set
 
 struct AttnProblem {
   CUtensorMap tmQ, tmK, tmV;  // 4D maps {channel, head, token, batch}, box {64,1,64,1}
@@ -77,7 +77,6 @@ struct AttnProblem {
   int n_splits;               // KV splits per (q tile pair, head, batch)
   int kv_per_split;           // tokens per split, multiple of 128
   int ctas;                   // work items: n_qtiles * H * B * n_splits
-  int mode;                   // AttnMode
   // sparse mode: the query groups and the merged key lists (n_qtiles = the
   // groups' capacity per batch item), the block table, and the list of the
   // work items that exist (ids (b H + h) n_qtiles + g, in index order)

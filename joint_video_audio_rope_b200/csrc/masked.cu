@@ -202,7 +202,6 @@ int mmdit_masked_joint_attn(const void* q, const void* k, const void* v, void* o
   pr.n_splits = 1;
   pr.kv_per_split = ((desc->n_tokens + 127) / 128) * 128;
   pr.ctas = pr.n_qtiles * pr.H * pr.B;
-  pr.mode = kModeDense;
   pr.q_count = count;
   ap.q_tiles = 2;
   ap.persistent = 0;

@@ -236,7 +236,6 @@ int short_kv_params(AttnParams& p, const void* q, const void* k, const void* v, 
   pr.n_splits = 1;
   pr.kv_per_split = ((kd.n_tokens + 127) / 128) * 128;
   pr.ctas = pr.n_qtiles * pr.H * pr.B;
-  pr.mode = kModeDense;
   p.q_tiles = kShortKvQTiles;
   p.persistent = 1;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -271,7 +270,6 @@ int launch_cross(const void* qv, const void* kv, const void* vv, const void* qa,
   a2v.n_splits = splits;
   a2v.kv_per_split = kv_per_split;
   a2v.ctas = a2v.n_qtiles * a2v.n_splits * a2v.H * a2v.B;
-  a2v.mode = kModeDense;
   pa.q_tiles = 2;
   pa.persistent = 1;
   pa.scale_log2 = scale * 1.4426950408889634f;
@@ -422,7 +420,6 @@ int mmdit_joint_attn(const void* q, const void* k, const void* v, void* o, float
   pr.n_splits = 1;
   pr.kv_per_split = ((desc->n_tokens + 127) / 128) * 128;
   pr.ctas = pr.n_qtiles * pr.H * pr.B;
-  pr.mode = kModeDense;
   pr.rope_q = rope_q != nullptr;
   p.q_tiles = kJointQTiles;
   p.persistent = 0;  // measured: one item per CTA is ~1% faster for long keys

@@ -200,7 +200,6 @@ int run_sparse(const void* q, const void* k, const void* v, void* o, const mmdit
   pr.n_splits = 1;
   pr.kv_per_split = 0;
   pr.ctas = w.maxg * pr.H * pr.B;
-  pr.mode = kModeSparse;
   pr.groups = groups;
   pr.n_groups = n_groups;
   pr.ulist = ulist;
