@@ -5,14 +5,17 @@
 
 One step is one pass of the layer's attention hot path over one batch of the
 workload: 3D RoPE of Q and K, then (dense workloads) joint self-attention over
-the whole sequence or (block-sparse workload) block selection and sparse
-video self-attention, then the bidirectional audio<->video cross-attention.
+the whole sequence or (block-sparse workloads) block selection and sparse
+video self-attention -- on the adaptive workload after the content-adaptive
+block plan and the move of Q, K, V to its storage order, O moved back after --
+then the bidirectional audio<->video cross-attention (on the adaptive
+workload with the A->V output norms for the next step's plan).
 Inputs are seeded synthetic tensors of the workload's shape, resident in HBM
 before timing; they are larger than L2 (126 MB), so no flush is needed.
 
 The headline workload (default: 720p_cond_b2, the largest dense layer that
 fits one GPU) gives the line's value; the other workloads (480p, 720p,
-1080p_sparse) follow under "per_config", timed the same way.  The JSON line
+1080p_sparse, 1080p_adaptive) follow under "per_config", timed the same way.  The JSON line
 reports algorithmic TFLOP/s (4 * Nq * Nkv * d per head for every attention;
 for sparse attention only the selected token pairs), video tokens/s, an
 end-to-end figure through the same C-ABI calls with pinned host buffers
