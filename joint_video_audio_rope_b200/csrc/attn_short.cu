@@ -181,14 +181,32 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_short_kernel(const __grid_
         if (!mbar_wait(bar(SB_QFULL + t), n & 1, err)) return false;
         if (n > 0 && !mbar_wait(bar(SB_OEMPTY + t), (n - 1) & 1, err)) return false;
         tc_fence_after();
-        const uint32_t q = sbase + kOffQ + t * kQTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t qo = (kk >> 2) * kQHalf + (kk & 3) * 32;
-          const uint32_t ko = (kk >> 2) * kKVHalf + (kk & 3) * 32;
-          tc_mma_ss(tmem + 256 * t, smem_desc_sw128(q + qo, 16, 1024),
-                    smem_desc_sw128(sbase + kOffK + ko, 16, 1024), kIdescS, kk > 0);
-        }
+        // eight MMAs of K = 16 channels in one asm block: the descriptors'
+        // start-address field (address >> 4) steps by 2 per 32 bytes and by
+        // the column-half distance >> 4 at channel 64 (addresses < 256 KB)
+        const uint64_t qd = smem_desc_sw128(sbase + kOffQ + t * kQTileBytes, 16, 1024);
+        const uint64_t kd = smem_desc_sw128(sbase + kOffK, 16, 1024);
+        asm volatile(
+            "{\n\t.reg .pred pf, pt;\n\t.reg .b64 ta, tb;\n\t"
+            "setp.ne.b32 pf, %3, %3;\n\t"
+            "setp.eq.b32 pt, %3, %3;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, pf;\n\t"
+            "add.s64 ta, %1, 2;\n\tadd.s64 tb, %2, 2;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], ta, tb, %3, pt;\n\t"
+            "add.s64 ta, %1, 4;\n\tadd.s64 tb, %2, 4;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], ta, tb, %3, pt;\n\t"
+            "add.s64 ta, %1, 6;\n\tadd.s64 tb, %2, 6;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], ta, tb, %3, pt;\n\t"
+            "add.s64 ta, %1, %4;\n\tadd.s64 tb, %2, %5;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], ta, tb, %3, pt;\n\t"
+            "add.s64 ta, ta, 2;\n\tadd.s64 tb, tb, 2;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], ta, tb, %3, pt;\n\t"
+            "add.s64 ta, ta, 2;\n\tadd.s64 tb, tb, 2;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], ta, tb, %3, pt;\n\t"
+            "add.s64 ta, ta, 2;\n\tadd.s64 tb, tb, 2;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], ta, tb, %3, pt;\n\t}"
+            ::"r"(tmem + 256 * t), "l"(qd), "l"(kd), "r"(kIdescS),
+            "l"((uint64_t)(kQHalf >> 4)), "l"((uint64_t)(kKVHalf >> 4)));
         tc_commit(bar(SB_SFULL + t));
         tc_commit(bar(SB_QEMPTY + t));
         return true;
@@ -197,10 +215,11 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_short_kernel(const __grid_
         if (!mbar_wait(bar(SB_PFULL + t), n & 1, err)) return false;
         tc_fence_after();
         const uint32_t s_tmem = tmem + 256 * t;
+        // 16 key rows (2048 bytes: 128 in the descriptor) and 8 P columns
+        // per K step
+        const uint64_t vd = smem_desc_sw128(sbase + kOffV, kKVHalf, 1024);
         for (int kk = 0; kk < n_ksteps; ++kk)
-          tc_mma_ts(s_tmem + 128, s_tmem + kk * 8,
-                    smem_desc_sw128(sbase + kOffV + kk * 2048, kKVHalf, 1024), kIdescO,
-                    kk > 0 ? 1u : 0u);
+          tc_mma_ts(s_tmem + 128, s_tmem + kk * 8, vd + 128u * kk, kIdescO, kk > 0 ? 1u : 0u);
         tc_commit(bar(SB_OFULL + t));
         return true;
       };

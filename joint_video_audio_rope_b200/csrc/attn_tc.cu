@@ -285,13 +285,33 @@ __device__ __forceinline__ void tma_tile(uint32_t dst, const CUtensorMap* map, u
 // channels moves the start address 32 bytes inside the swizzle atom, and the
 // second 64-channel half lives kHalfCol bytes further.
 __device__ __forceinline__ void mma_qk(uint32_t s_tmem, uint32_t q_smem, uint32_t k_smem) {
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    const uint32_t off = (kk >> 2) * kHalfCol + (kk & 3) * 32;
-    const uint64_t a = smem_desc_sw128(q_smem + off, 16, 1024);
-    const uint64_t b = smem_desc_sw128(k_smem + off, 16, 1024);
-    tc_mma_ss(s_tmem, a, b, kIdescQK, kk > 0);
-  }
+  // The descriptors' start-address field holds address >> 4, so stepping an
+  // operand by `off` bytes adds off >> 4 to it (every address here is below
+  // 256 KB: the 14-bit field does not wrap).  The eight MMAs go out in one
+  // asm block, the first overwriting S and the rest accumulating; the
+  // stepped descriptors are formed inside the block, two registers at a time.
+  const uint64_t a = smem_desc_sw128(q_smem, 16, 1024);
+  const uint64_t b = smem_desc_sw128(k_smem, 16, 1024);
+  asm volatile(
+      "{\n\t.reg .pred pf, pt;\n\t.reg .b64 ta, tb;\n\t"
+      "setp.ne.b32 pf, %3, %3;\n\t"
+      "setp.eq.b32 pt, %3, %3;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, pf;\n\t"
+      "add.s64 ta, %1, 2;\n\tadd.s64 tb, %2, 2;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ta, tb, %3, pt;\n\t"
+      "add.s64 ta, %1, 4;\n\tadd.s64 tb, %2, 4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ta, tb, %3, pt;\n\t"
+      "add.s64 ta, %1, 6;\n\tadd.s64 tb, %2, 6;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ta, tb, %3, pt;\n\t"
+      "add.s64 ta, %1, %4;\n\tadd.s64 tb, %2, %4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ta, tb, %3, pt;\n\t"
+      "add.s64 ta, ta, 2;\n\tadd.s64 tb, tb, 2;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ta, tb, %3, pt;\n\t"
+      "add.s64 ta, ta, 2;\n\tadd.s64 tb, tb, 2;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ta, tb, %3, pt;\n\t"
+      "add.s64 ta, ta, 2;\n\tadd.s64 tb, tb, 2;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ta, tb, %3, pt;\n\t}"
+      ::"r"(s_tmem), "l"(a), "l"(b), "r"(kIdescQK), "l"((uint64_t)(kHalfCol >> 4)));
 }
 
 // O_t (+)= P_t V : M=128, N=128 (channels), K=128 (key rows).  P comes from
@@ -301,11 +321,25 @@ __device__ __forceinline__ void mma_qk(uint32_t s_tmem, uint32_t q_smem, uint32_
 template <int K0, int K1>
 __device__ __forceinline__ void mma_pv_part(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem,
                                             bool accumulate) {
-#pragma unroll
-  for (int kk = K0; kk < K1; ++kk) {
-    const uint64_t b = smem_desc_sw128(v_smem + kk * 2048, kHalfCol, 1024);
-    tc_mma_ts(o_tmem, p_tmem + kk * 8, b, kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
-  }
+  static_assert(K1 - K0 == 4, "four K steps per part");
+  // V steps 16 key rows (2048 bytes: 128 in the descriptor) per K step; P
+  // steps 8 TMEM columns.  The first MMA accumulates only if asked (or past
+  // the first K step), the rest always.
+  const uint64_t b = smem_desc_sw128(v_smem + K0 * 2048, kHalfCol, 1024);
+  const uint32_t pa = p_tmem + K0 * 8;
+  const uint32_t acc0 = (accumulate || K0 > 0) ? 1u : 0u;
+  asm volatile(
+      "{\n\t.reg .pred p0, pt;\n\t.reg .b64 tb;\n\t.reg .b32 ta;\n\t"
+      "setp.ne.b32 p0, %4, 0;\n\t"
+      "setp.eq.b32 pt, %4, %4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p0;\n\t"
+      "add.u32 ta, %1, 8;\n\tadd.s64 tb, %2, 128;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], tb, %3, pt;\n\t"
+      "add.u32 ta, ta, 8;\n\tadd.s64 tb, tb, 128;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], tb, %3, pt;\n\t"
+      "add.u32 ta, ta, 8;\n\tadd.s64 tb, tb, 128;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], tb, %3, pt;\n\t}"
+      ::"r"(o_tmem), "r"(pa), "l"(b), "r"(kIdescPV), "r"(acc0));
 }
 
 // Rotate this thread's Q row (row r of the tile at q_smem) in place by the
