@@ -245,12 +245,21 @@ __device__ __forceinline__ float warp_max_f(float v) {
 template <int VPL>
 struct Row {
   float v[VPL];
+  // values per lane that hold blocks of the row (the rest are padding, -1):
+  // the passes skip the chunks of 8 past them (warp-uniform branches), so a
+  // row of n blocks costs ~n, not the capacity the template was sized for
+  int nv = VPL;
 
   // number of probabilities with bit pattern >= tau (tau >= 0)
   __device__ __forceinline__ int count_ge(int tau) const {
     int c = 0;
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) c += __float_as_int(v[i]) >= tau;
+    for (int i0 = 0; i0 < VPL; i0 += 8) {
+      if (i0 < nv) {  // warp-uniform
+#pragma unroll
+        for (int i = i0; i < i0 + 8 && i < VPL; ++i) c += __float_as_int(v[i]) >= tau;
+      }
+    }
     return warp_sum_i(c);
   }
   // sum of the probabilities with bit pattern >= tau: fp32 over chunks of 8
@@ -259,11 +268,13 @@ struct Row {
     double m = 0.0;
 #pragma unroll
     for (int i0 = 0; i0 < VPL; i0 += 8) {
-      float c = 0.f;
+      if (i0 < nv) {  // warp-uniform
+        float c = 0.f;
 #pragma unroll
-      for (int i = i0; i < i0 + 8 && i < VPL; ++i)
-        c += __float_as_int(v[i]) >= tau ? v[i] : 0.f;
-      m += (double)c;
+        for (int i = i0; i < i0 + 8 && i < VPL; ++i)
+          c += __float_as_int(v[i]) >= tau ? v[i] : 0.f;
+        m += (double)c;
+      }
     }
     return warp_sum_d(m);
   }
@@ -282,6 +293,7 @@ __global__ void __launch_bounds__(256) select_rows_kernel(
   const long long hb = ((long long)b * H + h) * maxb;
   const float* srow = S + (hb + row) * ld;
   Row<VPL> P;
+  P.nv = (n + 31) / 32;
   float mx = -INFINITY;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
@@ -353,16 +365,18 @@ __global__ void __launch_bounds__(256) select_rows_kernel(
   int pos = 0, ties = 0;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
-    const int j = lane + 32 * i;
-    const int vb = __float_as_int(P.v[i]);
-    const bool eq = vb == tau;  // padding (-1) never equals tau >= 0
-    const unsigned eqm = __ballot_sync(0xffffffffu, eq);
-    const int tie_rank = ties + __popc(eqm & ((1u << lane) - 1u));
-    const bool sel = vb > tau || (eq && tie_rank < take_eq);
-    const unsigned sm_ = __ballot_sync(0xffffffffu, sel);
-    if (sel) out[pos + __popc(sm_ & ((1u << lane) - 1u))] = j;
-    pos += __popc(sm_);
-    ties += __popc(eqm);
+    if (i < P.nv) {  // only padding beyond (warp-uniform)
+      const int j = lane + 32 * i;
+      const int vb = __float_as_int(P.v[i]);
+      const bool eq = vb == tau;  // padding (-1) never equals tau >= 0
+      const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+      const int tie_rank = ties + __popc(eqm & ((1u << lane) - 1u));
+      const bool sel = vb > tau || (eq && tie_rank < take_eq);
+      const unsigned sm_ = __ballot_sync(0xffffffffu, sel);
+      if (sel) out[pos + __popc(sm_ & ((1u << lane) - 1u))] = j;
+      pos += __popc(sm_);
+      ties += __popc(eqm);
+    }
   }
   if (lane == 0) cnt[hb + row] = pos;
 }
